@@ -1,0 +1,355 @@
+"""Model-level pins of the oracle (CPU only): invariants and closed forms.
+
+Each test would fail under a plausible mistake in the composition: a dropped
+residual, a wrong AdaLN order, a swapped concatenation, a wrong category index,
+a wrong self/cross alternation, an Euler step of the wrong size or sign.
+"""
+
+import dataclasses
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+TINY = synth.WORKLOADS["tiny"]
+G = TINY.geom
+rng = np.random.default_rng(77)
+
+
+@pytest.fixture(scope="module")
+def W():
+    return synth.make_weights(G)
+
+
+def _inputs(batch=1, seq=64, ids=None, seed=1):
+    w = dataclasses.replace(TINY, batch=batch, seq=seq,
+                            fixed_ids=tuple(ids) if ids is not None else (0,))
+    return synth.make_inputs(w, seed=seed)
+
+
+def _run(W, inp, K=4, g=G, **kw):
+    return oracle.get_action(W, g, inp["backbone_features"], inp["vl_mask"], inp["state"],
+                             inp["embodiment_id"], inp["init_noise"], K, **kw)
+
+
+def _copy(W):
+    return {k: np.array(v, copy=True) for k, v in W.items()}
+
+
+# ---------------------------------------------------------------- invariants
+
+def test_masked_backbone_tokens_have_no_influence(W):
+    inp = _inputs(batch=2, ids=[0, 1])
+    inp["vl_mask"][0, 40:] = 0
+    inp["vl_mask"][1, ::3] = 0
+    out = _run(W, inp)
+    feats = inp["backbone_features"].copy()
+    feats[inp["vl_mask"] == 0] = rng.normal(size=(int((inp["vl_mask"] == 0).sum()), G.backbone_dim)) * 100
+    out2 = _run(W, dict(inp, backbone_features=feats))
+    np.testing.assert_array_equal(out, out2)
+    # a valid token does matter
+    feats[0, 0] += 1.0
+    assert not np.array_equal(out, _run(W, dict(inp, backbone_features=feats)))
+
+
+def test_zero_velocity_head_leaves_noise(W):
+    W0 = _copy(W)
+    W0["act_dec.l2.W"][:] = 0
+    W0["act_dec.l2.b"][:] = 0
+    inp = _inputs(batch=2, ids=[1, 0])
+    np.testing.assert_array_equal(_run(W0, inp), inp["init_noise"].astype(np.float64))
+
+
+def test_one_step_is_noise_plus_velocity(W):
+    inp = _inputs()
+    m = oracle.Model(W, G)
+    s, kvs = oracle.prepare_sample(m, inp["backbone_features"][0], inp["vl_mask"][0], inp["state"][0], 0)
+    x0 = inp["init_noise"][0].astype(np.float64)
+    v = oracle.velocity(m, x0, 0.0, s, kvs, 0)
+    np.testing.assert_array_equal(_run(W, inp, K=1)[0], x0 + v)
+
+
+def test_decoder_bias_signature_routes_by_category():
+    g = dataclasses.replace(G, num_embodiments=4)
+    Wg = synth.make_weights(g)
+    Wg["act_dec.l1.W"][:] = 0
+    Wg["act_dec.l1.b"][:] = 0
+    Wg["act_dec.l2.W"][:] = 0
+    for c in range(4):
+        Wg["act_dec.l2.b"][c] = c
+    inp = _inputs(batch=4, ids=[2, 0, 3, 1])
+    out = _run(Wg, inp, g=g)
+    expect = inp["init_noise"].astype(np.float64) + np.array([2, 0, 3, 1], np.float64)[:, None, None]
+    np.testing.assert_array_equal(out, expect)
+
+
+def test_routing_equals_running_alone_with_category_moved_to_zero(W):
+    inp = _inputs(batch=2, ids=[1, 0])
+    mixed = _run(W, inp)
+    # sample 0 (category 1) alone, in a model whose category 0 holds category 1's weights
+    Wm = _copy(W)
+    for name, v in Wm.items():
+        if v.ndim >= 2 and v.shape[0] == G.num_embodiments and name.split(".")[0] in (
+                "state_enc", "act_enc", "act_dec"):
+            v[0] = W[name][1]
+    alone = {k: v[:1] for k, v in inp.items()}
+    alone["embodiment_id"] = np.array([0], np.int32)
+    np.testing.assert_array_equal(_run(Wm, alone)[0], mixed[0])
+    # and the category matters
+    other = dict(alone, embodiment_id=np.array([0], np.int32))
+    assert not np.array_equal(_run(W, other)[0], mixed[0])
+
+
+def test_batch_permutation_equivariance(W):
+    inp = _inputs(batch=3, ids=[0, 1, 1])
+    inp["vl_mask"][1, 10:] = 0
+    out = _run(W, inp)
+    perm = [2, 0, 1]
+    pinp = {k: v[perm] for k, v in inp.items()}
+    np.testing.assert_array_equal(_run(W, pinp), out[perm])
+
+
+def test_horizon_permutation_equivariance(W):
+    # no positional encoding over the horizon: permuting noise rows permutes the output
+    inp = _inputs()
+    out = _run(W, inp)
+    perm = rng.permutation(G.action_horizon)
+    pinp = dict(inp, init_noise=inp["init_noise"][:, perm])
+    np.testing.assert_allclose(_run(W, pinp), out[:, perm], rtol=0, atol=1e-13)
+
+
+def test_constant_velocity_integrates_exactly(W):
+    # all DiT and encoder matrices zero: v no longer depends on x or t, and K
+    # Euler steps of size 1/K add exactly v for every K
+    Wz = _copy(W)
+    for name, v in Wz.items():
+        if name.endswith((".w", ".W")) and not name.startswith("act_dec"):
+            v[:] = 0
+    inp = _inputs()
+    deltas = [(_run(Wz, inp, K=K) - inp["init_noise"])[0] for K in (1, 2, 3, 4, 8)]
+    for d in deltas[1:]:
+        np.testing.assert_allclose(d, deltas[0], rtol=0, atol=1e-14)
+    assert np.abs(deltas[0]).max() > 1e-3
+
+
+def test_alternation_even_layers_cross_odd_layers_self():
+    g = dataclasses.replace(G, num_layers=4)
+    Wg = synth.make_weights(g)
+    inp = _inputs()
+    feats2 = inp["backbone_features"] + 1.0
+    # silence the attention outputs of the even layers: the backbone no longer matters
+    We = _copy(Wg)
+    for l in (0, 2):
+        We[f"blk{l}.o.w"][:] = 0
+    np.testing.assert_array_equal(_run(We, inp, g=g), _run(We, dict(inp, backbone_features=feats2), g=g))
+    # silence only layer 0: layer 2 still reads the backbone
+    W0 = _copy(Wg)
+    W0["blk0.o.w"][:] = 0
+    assert not np.array_equal(_run(W0, inp, g=g), _run(W0, dict(inp, backbone_features=feats2), g=g))
+    # silence the odd layers: the backbone still matters
+    Wo = _copy(Wg)
+    for l in (1, 3):
+        Wo[f"blk{l}.o.w"][:] = 0
+    assert not np.array_equal(_run(Wo, inp, g=g), _run(Wo, dict(inp, backbone_features=feats2), g=g))
+
+
+def test_sample_without_valid_tokens_sees_zero_attention(W):
+    inp = _inputs()
+    inp["vl_mask"][:] = 0
+    out = _run(W, inp)
+    assert np.isfinite(out).all()
+    # same as one valid token whose values are all zero (cross V weights and biases zeroed)
+    Wv = _copy(W)
+    Wv["blk0.v.w"][:] = 0
+    Wv["blk0.v.b"][:] = 0
+    one = dict(inp, vl_mask=inp["vl_mask"].copy())
+    one["vl_mask"][0, 5] = 1
+    np.testing.assert_array_equal(_run(Wv, one), out)
+
+
+# ---------------------------------------------------------------- closed forms
+
+def _zero_block(W, layer):
+    Wb = _copy(W)
+    for n in ("q", "k", "v", "o", "ff1", "ff2", "ada"):
+        Wb[f"blk{layer}.{n}.w"][:] = 0
+    return Wb
+
+
+@pytest.mark.parametrize("layer", [0, 1])
+def test_block_residuals_closed_form(W, layer):
+    # Q = K = 0 (uniform attention), V = b_v for every key, O = identity:
+    # attention adds b_v + b_o; the MLP adds GELU(b_1) W_2 + b_2 = b_2 with W_2 = 0.
+    Wb = _zero_block(W, layer)
+    D = G.hidden
+    Wb[f"blk{layer}.o.w"][:] = np.eye(D, dtype=np.float32)
+    m = oracle.Model(Wb, G)
+    h = rng.normal(size=(G.action_horizon + 1, D))
+    temb = rng.normal(size=D)
+    kv = None
+    if layer % 2 == 0:
+        bv = m[f"blk{layer}.v.b"]
+        kv = (np.zeros((9, D)), np.repeat(bv[None], 9, axis=0))
+    out = oracle.dit_block(m, layer, h, temb, kv)
+    expect = h + m[f"blk{layer}.v.b"] + m[f"blk{layer}.o.b"] + m[f"blk{layer}.ff2.b"]
+    np.testing.assert_allclose(out, expect, rtol=0, atol=1e-12)
+
+
+def test_adaln_scale_then_shift_closed_form():
+    D = 8
+    a = 3.0
+    h = np.tile(np.array([a, -a] * (D // 2)), (2, 1))       # mean 0, variance a^2
+    s = rng.normal(size=D)
+    t = rng.normal(size=D)
+    out = oracle.ada_layer_norm(h, rng.normal(size=5), np.zeros((2 * D, 5)), np.concatenate([s, t]), 1e-5)
+    n = a / np.sqrt(a * a + 1e-5)
+    expect = np.array([n, -n] * (D // 2)) * (1.0 + s) + t
+    np.testing.assert_allclose(out, np.tile(expect, (2, 1)), rtol=1e-14, atol=1e-14)
+
+
+def test_timestep_embedding_with_zero_weights_is_output_bias(W):
+    Wz = _copy(W)
+    Wz["t_enc.l1.w"][:] = 0
+    Wz["t_enc.l1.b"][:] = 0
+    Wz["t_enc.l2.w"][:] = 0
+    m = oracle.Model(Wz, G)
+    np.testing.assert_array_equal(oracle.timestep_embedding(m, 250.0), m["t_enc.l2.b"])
+
+
+def test_action_encoder_concatenates_actions_first(W):
+    D = G.hidden
+    x = rng.normal(size=(G.action_horizon, G.action_dim))
+    # zero the first D input rows of W2: only the timestep half remains
+    Wa = _copy(W)
+    Wa["act_enc.W2.W"][:, :D, :] = 0
+    m = oracle.Model(Wa, G)
+    e1 = oracle.action_encoder(m, x, 250.0, 1)
+    e2 = oracle.action_encoder(m, x + 5.0, 250.0, 1)
+    np.testing.assert_array_equal(e1, e2)
+    assert not np.array_equal(e1, oracle.action_encoder(m, x, 500.0, 1))
+    # zero the last D rows: only the action half remains
+    Wt = _copy(W)
+    Wt["act_enc.W2.W"][:, D:, :] = 0
+    m = oracle.Model(Wt, G)
+    np.testing.assert_array_equal(oracle.action_encoder(m, x, 250.0, 1), oracle.action_encoder(m, x, 750.0, 1))
+    assert not np.array_equal(oracle.action_encoder(m, x, 250.0, 1), oracle.action_encoder(m, x + 5.0, 250.0, 1))
+
+
+def test_category_mlp_relu_between_layers(W):
+    D = G.hidden
+    Wr = _copy(W)
+    Wr["state_enc.l1.W"][:] = 0
+    b1 = np.where(np.arange(D) % 2 == 0, -1.0, 2.0).astype(np.float32)
+    Wr["state_enc.l1.b"][1] = b1
+    Wr["state_enc.l2.W"][1] = np.eye(D, dtype=np.float32)
+    m = oracle.Model(Wr, G)
+    out = oracle.state_encoder(m, rng.normal(size=(1, G.state_dim)), 1)
+    expect = np.where(np.arange(D) % 2 == 0, 0.0, 2.0) + m.cat("state_enc.l2.b", 1)
+    np.testing.assert_array_equal(out[0], expect)
+
+
+def test_state_token_comes_first(W):
+    # the decoder output of row 0 is dropped: zero the action encoder (all action
+    # tokens equal) and the state feature still reaches the actions only through
+    # attention; changing the state changes the output
+    inp = _inputs()
+    out = _run(W, inp)
+    inp2 = dict(inp, state=inp["state"] + 1.0)
+    assert not np.array_equal(out, _run(W, inp2))
+    assert out.shape == (1, G.action_horizon, G.action_dim)
+
+
+def test_bad_embodiment_id_rejected(W):
+    inp = _inputs()
+    inp["embodiment_id"] = np.array([G.num_embodiments], np.int32)
+    with pytest.raises(ValueError):
+        _run(W, inp)
+
+
+def test_dropped_row_is_the_state_token(W):
+    # With every attention and MLP output silenced and proj_out the identity, a
+    # token's velocity depends on that token alone.  Perturbing noise row i must
+    # then change output row i only: this fails if the state token were not the
+    # first row or if the wrong decoded row were dropped.
+    Wi = _copy(W)
+    for l in range(G.num_layers):
+        for n in ("o", "ff2"):
+            Wi[f"blk{l}.{n}.w"][:] = 0
+            Wi[f"blk{l}.{n}.b"][:] = 0
+    Wi["out.proj.w"][:] = np.eye(G.hidden, dtype=np.float32)
+    inp = _inputs()
+    out = _run(Wi, inp, K=1)
+    for i in (0, 3, G.action_horizon - 1):
+        noise = inp["init_noise"].copy()
+        noise[0, i] += 0.5
+        out2 = _run(Wi, dict(inp, init_noise=noise), K=1)
+        changed = np.nonzero(np.abs(out2 - out)[0].max(axis=1) > 0)[0].tolist()
+        assert changed == [i]
+
+
+def test_loop_feeds_discretised_timesteps(W):
+    # K = 2: t = 0, 0.5 -> t_discretized = 0, 500 (1000 buckets); dt = 0.5
+    inp = _inputs()
+    m = oracle.Model(W, G)
+    s, kvs = oracle.prepare_sample(m, inp["backbone_features"][0], inp["vl_mask"][0], inp["state"][0], 0)
+    x = inp["init_noise"][0].astype(np.float64)
+    x = x + 0.5 * oracle.velocity(m, x, 0.0, s, kvs, 0)
+    x = x + 0.5 * oracle.velocity(m, x, 500.0, s, kvs, 0)
+    np.testing.assert_array_equal(_run(W, inp, K=2)[0], x)
+    # the timestep does reach the network
+    x1 = inp["init_noise"][0].astype(np.float64)
+    assert not np.array_equal(oracle.velocity(m, x1, 0.0, s, kvs, 0), oracle.velocity(m, x1, 0.5, s, kvs, 0))
+
+
+def test_mlp_branch_is_gelu_of_affine_layer_norm(W):
+    # attention silenced, FF1/FF2 = identity embeddings: the block adds
+    # GELU(LN3(h)) with LN3's gain and bias (expected value from torch)
+    import torch
+    layer = 1
+    D, F = G.hidden, G.mlp_hidden
+    Wb = _copy(W)
+    p = f"blk{layer}."
+    Wb[p + "o.w"][:] = 0
+    Wb[p + "o.b"][:] = 0
+    Wb[p + "ff1.w"][:] = np.eye(F, D, dtype=np.float32)
+    Wb[p + "ff1.b"][:] = 0
+    Wb[p + "ff2.w"][:] = np.eye(D, F, dtype=np.float32)
+    Wb[p + "ff2.b"][:] = 0
+    m = oracle.Model(Wb, G)
+    h = rng.normal(size=(5, D))
+    out = oracle.dit_block(m, layer, h, rng.normal(size=D), None)
+    th = torch.from_numpy(h)
+    ln = torch.nn.functional.layer_norm(th, (D,), torch.from_numpy(m[p + "ln3.g"]),
+                                        torch.from_numpy(m[p + "ln3.b"]), eps=G.ln_eps)
+    expect = (th + torch.nn.functional.gelu(ln)).numpy()
+    np.testing.assert_allclose(out, expect, rtol=1e-12, atol=1e-12)
+
+
+def test_timestep_encoder_is_linear_silu_linear(W):
+    import torch
+    D = G.hidden
+    Wt = _copy(W)
+    Wt["t_enc.l1.w"][:] = 0
+    Wt["t_enc.l2.w"][:] = np.eye(D, dtype=np.float32)
+    m = oracle.Model(Wt, G)
+    expect = torch.nn.functional.silu(torch.from_numpy(m["t_enc.l1.b"])).numpy() + m["t_enc.l2.b"]
+    np.testing.assert_allclose(oracle.timestep_embedding(m, 750.0), expect, rtol=1e-13, atol=1e-15)
+
+
+def test_action_encoder_applies_swish_to_w2(W):
+    import torch
+    D = G.hidden
+    Wa = _copy(W)
+    for n in ("W1", "W2", "W3"):
+        Wa[f"act_enc.{n}.W"][:] = 0
+        Wa[f"act_enc.{n}.b"][:] = 0
+    Wa["act_enc.W2.W"][0, D:, :] = np.eye(D, dtype=np.float32)    # tau half -> identity
+    Wa["act_enc.W3.W"][0] = np.eye(D, dtype=np.float32)
+    m = oracle.Model(Wa, G)
+    x = rng.normal(size=(G.action_horizon, G.action_dim))
+    tau = oracle.sinusoidal_embedding(250.0, D)
+    expect = torch.nn.functional.silu(torch.from_numpy(tau)).numpy()
+    out = oracle.action_encoder(m, x, 250.0, 0)
+    np.testing.assert_allclose(out, np.broadcast_to(expect, out.shape), rtol=1e-13, atol=1e-15)
