@@ -1,0 +1,1363 @@
+// Runtime and C ABI of the flow-matching DiT action head (see include/gdit.h).
+//
+// One call of gdit_get_action enqueues, on the caller's stream:
+//   route (stable sort by embodiment id) -> pack valid backbone tokens ->
+//   gather noise / state -> K/V projection of every cross layer (one GEMM) ->
+//   state encoder -> K x { action encoder -> 32 DiT blocks -> norm_out +
+//   proj_out -> action decoder with the Euler update fused } -> scatter.
+// (Isaac-GR00T architecture page, "Inference (denoising)".)  The sequence is
+// captured once per (batch, seq, K, feature dtype) profile as a CUDA graph;
+// replays read the caller's pointers from a small device block written by a
+// one-thread kernel before each replay.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <memory>
+#include <stdexcept>
+#include <string>
+#include <tuple>
+#include <unordered_map>
+#include <vector>
+
+#include "gdit.h"
+#include "attention.cuh"
+#include "gemm_tc.cuh"
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+using namespace gdit;
+
+namespace {
+
+// ------------------------------------------------------------------ errors
+
+struct GditError : std::runtime_error {
+  int code;
+  GditError(int c, const std::string& m) : std::runtime_error(m), code(c) {}
+};
+
+std::string fmt(const char* f, ...) {
+  char buf[1024];
+  va_list ap;
+  va_start(ap, f);
+  vsnprintf(buf, sizeof(buf), f, ap);
+  va_end(ap);
+  return buf;
+}
+
+#define CUDA_TRY(expr)                                                                                  \
+  do {                                                                                                  \
+    cudaError_t e_ = (expr);                                                                            \
+    if (e_ != cudaSuccess)                                                                              \
+      throw GditError(e_ == cudaErrorMemoryAllocation ? GDIT_ENOMEM : GDIT_ECUDA,                       \
+                      fmt("%s failed: %s (%s:%d)", #expr, cudaGetErrorString(e_), __FILE__, __LINE__)); \
+  } while (0)
+
+#define REQUIRE(cond, ...)                                  \
+  do {                                                      \
+    if (!(cond)) throw GditError(GDIT_EINVAL, fmt(__VA_ARGS__)); \
+  } while (0)
+
+thread_local std::string g_create_error;
+
+// ------------------------------------------------------------------ host bf16
+
+uint16_t f32_to_bf16_rne(float f) {
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  if ((u & 0x7fffffffu) > 0x7f800000u) return (uint16_t)((u >> 16) | 0x40u);   // quiet NaN
+  const uint32_t lsb = (u >> 16) & 1u;
+  u += 0x7fffu + lsb;
+  return (uint16_t)(u >> 16);
+}
+
+float bf16_to_f32(uint16_t b) {
+  const uint32_t u = (uint32_t)b << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return f;
+}
+
+// ------------------------------------------------------------------ TMA descriptors
+
+typedef CUresult (*PFN_encodeTiled_t)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                       const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                       CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+PFN_encodeTiled_t encode_fn() {
+  static PFN_encodeTiled_t fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    CUDA_TRY(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q));
+    if (p == nullptr || q != cudaDriverEntryPointSuccess)
+      throw GditError(GDIT_ECUDA, "cuTensorMapEncodeTiled not available from the driver");
+    fn = reinterpret_cast<PFN_encodeTiled_t>(p);
+  }
+  return fn;
+}
+
+// bf16 matrix [rows, cols] with row pitch `pitch` elements; boxes of box_rows x 64,
+// 128-byte swizzle (the layout the UMMA descriptors expect).
+CUtensorMap make_tmap(const void* ptr, long long rows, long long cols, long long pitch, int box_rows) {
+  REQUIRE(((uintptr_t)ptr & 15u) == 0, "TMA base pointer not 16-byte aligned");
+  REQUIRE((pitch * 2) % 16 == 0, "TMA row pitch %lld elements is not a multiple of 16 bytes", pitch);
+  REQUIRE(box_rows >= 1 && box_rows <= 256, "TMA box rows %d", box_rows);
+  CUtensorMap m;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)std::max<long long>(rows, 1)};
+  cuuint64_t strides[1] = {(cuuint64_t)(pitch * 2)};
+  cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = encode_fn()(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) throw GditError(GDIT_ECUDA, fmt("cuTensorMapEncodeTiled failed (%d)", (int)r));
+  return m;
+}
+
+// ------------------------------------------------------------------ launch helper
+
+bool g_pdl_default = true;
+
+template <typename... KArgs, typename... Args>
+void launch_k(cudaStream_t s, bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...));
+}
+
+// ------------------------------------------------------------------ GEMM ops
+
+struct GemmOp {
+  CUtensorMap ta, tb;
+  GemmArgs args;
+  int bn = 64;
+  int grid = 1;
+  // algorithmic accounting: rows actually multiplied are known after routing
+  int rows_kind = 0;   // 0 fixed M, 1 = total valid tokens, 2 = all rows (grouped)
+  long long weight_bytes = 0;
+  int out_bytes = 2;
+};
+
+template <int BN>
+void set_gemm_attr() {
+  CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmCfg<BN>::SMEM));
+}
+
+void launch_gemm(const GemmOp& op, const GemmArgs& a, cudaStream_t s, bool pdl) {
+  switch (op.bn) {
+    case 32:
+      launch_k(s, pdl, gemm_tc_kernel<32>, dim3(op.grid), dim3(kGemmThreads), GemmCfg<32>::SMEM, op.ta, op.tb, a);
+      break;
+    case 64:
+      launch_k(s, pdl, gemm_tc_kernel<64>, dim3(op.grid), dim3(kGemmThreads), GemmCfg<64>::SMEM, op.ta, op.tb, a);
+      break;
+    case 128:
+      launch_k(s, pdl, gemm_tc_kernel<128>, dim3(op.grid), dim3(kGemmThreads), GemmCfg<128>::SMEM, op.ta, op.tb, a);
+      break;
+    case 256:
+      launch_k(s, pdl, gemm_tc_kernel<256>, dim3(op.grid), dim3(kGemmThreads), GemmCfg<256>::SMEM, op.ta, op.tb, a);
+      break;
+    default:
+      throw GditError(GDIT_EINVAL, fmt("bad GEMM tile width %d", op.bn));
+  }
+}
+
+GemmArgs default_args() {
+  GemmArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.splits = 1;
+  a.in_group = 0x7fffffff;
+  a.in_skip = 0;
+  a.out_group = 0;
+  a.out_off = 0;
+  return a;
+}
+
+constexpr long long kWsFloats = 16ll << 20;   // split-K partials (64 MB)
+constexpr int kCounters = 1 << 16;
+
+// Picks the tile width and split-K factor.  Large row counts use wide tiles;
+// small ones (weight streaming) use narrow tiles and split K so that about
+// one CTA per SM streams a slice of the weights.
+void choose_tiling(long long rows_est, int groups_est, int N, int K, int num_sms, long long ws_rows, int& bn,
+                   int& splits) {
+  if (N <= 32)
+    bn = 32;
+  else if (rows_est >= 2048 && N % 256 == 0)
+    bn = 256;
+  else if (rows_est >= 512 && N % 128 == 0)
+    bn = 128;
+  else
+    bn = 64;
+  const long long mt = (rows_est + kBM - 1) / kBM + std::max(groups_est - 1, 0);
+  const long long nt = (N + bn - 1) / bn;
+  const long long units = std::max<long long>(mt * nt, 1);
+  const int nkb = (K + kBK - 1) / kBK;
+  splits = 1;
+  if (units < num_sms) {
+    long long s = num_sms / units;
+    s = std::min<long long>(s, std::max(nkb / 2, 1));
+    while (s > 1 && s * ws_rows * (long long)N > kWsFloats) --s;
+    splits = (int)std::max<long long>(s, 1);
+  }
+}
+
+// ------------------------------------------------------------------ weights
+
+struct WeightSpec {
+  std::string name;
+  std::vector<int64_t> shape;
+};
+
+struct DevModel {
+  // bf16 matrices
+  __nv_bfloat16 *t1w, *t2w, *ada_w, *wkv, *proj_w;
+  std::vector<__nv_bfloat16*> wq;     // per layer: [3D, D] (self) or [D, D] (cross)
+  std::vector<__nv_bfloat16*> wo, wff1, wff2;
+  __nv_bfloat16 *ws1t, *ws2t, *wa1t, *wa2at, *wa2taut, *wa3t, *wd1t, *wd2t;
+  // f32 vectors
+  float *t1b, *t2b, *ada_b, *bkv, *proj_b;
+  std::vector<float*> bq, bo, ln3g, ln3b, bff1, bff2;
+  float *bs1, *bs2, *ba1, *ba2, *ba3, *bd1, *bd2;
+};
+
+struct Tables {
+  int K = 0;
+  float* ada = nullptr;   // [K][L+1][2D]
+  float* tw2 = nullptr;   // [K][C][D]
+  std::vector<float> td;  // host copy
+};
+
+struct Profile {
+  int B, S, K, bf16;
+  GemmOp kv, st1, st2, a1, a2, a3, proj, d1, d2;
+  std::vector<GemmOp> q, o, ff1, ff2;
+  cudaGraphExec_t exec = nullptr;
+};
+
+struct KStat {
+  std::string name;
+  int launches = 0;
+  double ms = 0, flops = 0, bytes = 0;
+};
+
+struct Recorder {
+  struct Ev {
+    int cls;
+    cudaEvent_t a, b;
+    double flops, bytes;
+    const GemmOp* op;
+  };
+  std::vector<Ev> evs;
+  std::vector<std::string> names;
+  int cls(const std::string& n) {
+    for (size_t i = 0; i < names.size(); ++i)
+      if (names[i] == n) return (int)i;
+    names.push_back(n);
+    return (int)names.size() - 1;
+  }
+};
+
+}  // namespace
+
+struct gdit_handle {
+  gdit_config cfg;
+  int L, D, F, Dvl, A, Sd, H, C, Tf, N, Lc;
+  int num_sms = 148;
+  bool pdl = true;
+  bool use_graph = true;
+  bool strict = false;
+  std::string last_error;
+
+  // device memory
+  std::vector<void*> allocs;
+  DevModel w;
+  __nv_bfloat16 *xp, *kv, *u, *qkv, *o, *f, *xb, *abf, *zbf, *ybf, *rbf, *sb, *s1;
+  float *h, *x, *sfeat, *ws;
+  int *perm, *seg, *vofs, *counters;
+  uint8_t* bad;
+  unsigned* status;
+  IoPtrs* io;
+  long long max_tok;
+
+  // per-K tables and per-profile plans
+  std::map<int, Tables> tables;
+  std::map<std::tuple<int, int, int, int>, std::unique_ptr<Profile>> profiles;
+  cudaStream_t cap_stream = nullptr;
+  cudaStream_t last_stream = nullptr;
+
+  // host-buffer staging (gdit_get_action_host)
+  void* st_feats = nullptr;
+  size_t st_feats_bytes = 0;
+  uint8_t* st_mask = nullptr;
+  float *st_state = nullptr, *st_noise = nullptr, *st_out = nullptr;
+  int32_t* st_ids = nullptr;
+
+  Recorder* rec = nullptr;   // non-null during gdit_profile_get_action
+  int last_B = 0;
+
+  template <typename T>
+  T* dalloc(size_t count) {
+    void* p = nullptr;
+    CUDA_TRY(cudaMalloc(&p, std::max<size_t>(count * sizeof(T), 256)));
+    allocs.push_back(p);
+    return static_cast<T*>(p);
+  }
+};
+
+namespace {
+
+// ------------------------------------------------------------------ validation
+
+void validate_config(const gdit_config& c) {
+  REQUIRE(c.num_layers >= 2 && c.num_layers % 2 == 0, "num_layers must be even and >= 2 (got %d)", c.num_layers);
+  REQUIRE(c.head_dim == 32 || c.head_dim == 64, "head_dim must be 32 or 64 (got %d)", c.head_dim);
+  REQUIRE(c.num_heads >= 1 && c.hidden == c.num_heads * c.head_dim, "hidden (%d) must equal num_heads * head_dim",
+          c.hidden);
+  REQUIRE(c.hidden == 128 || c.hidden == 256 || c.hidden == 512 || c.hidden == 1024 || c.hidden == 2048,
+          "hidden must be one of 128, 256, 512, 1024, 2048 (got %d)", c.hidden);
+  REQUIRE(c.mlp_hidden >= 64 && c.mlp_hidden % 64 == 0, "mlp_hidden must be a positive multiple of 64");
+  REQUIRE(c.backbone_dim >= 64 && c.backbone_dim % 64 == 0, "backbone_dim must be a positive multiple of 64");
+  REQUIRE(c.action_dim >= 32 && c.action_dim <= 256 && c.action_dim % 32 == 0,
+          "action_dim must be a multiple of 32 in [32, 256] (got %d)", c.action_dim);
+  REQUIRE(c.state_dim >= 32 && c.state_dim <= 256 && c.state_dim % 32 == 0,
+          "state_dim must be a multiple of 32 in [32, 256] (got %d)", c.state_dim);
+  REQUIRE(c.action_horizon >= 1 && c.action_horizon + 1 <= 64, "action_horizon must be in [1, 63] (got %d)",
+          c.action_horizon);
+  REQUIRE(c.num_embodiments >= 1 && c.num_embodiments <= kMaxGroups, "num_embodiments must be in [1, %d]",
+          kMaxGroups);
+  REQUIRE(c.max_batch >= 1 && c.max_batch <= kMaxBatch, "max_batch must be in [1, %d]", kMaxBatch);
+  REQUIRE(c.max_backbone_seq >= 1 && c.max_backbone_seq <= 65536, "max_backbone_seq must be in [1, 65536]");
+  REQUIRE(c.time_freq_dim >= 2 && c.time_freq_dim % 2 == 0, "time_freq_dim must be even and >= 2");
+  REQUIRE(c.num_timestep_buckets >= 1, "num_timestep_buckets must be >= 1");
+  REQUIRE(c.ln_eps > 0.0f, "ln_eps must be > 0");
+}
+
+std::vector<WeightSpec> weight_specs(const gdit_config& c) {
+  const int64_t D = c.hidden, F = c.mlp_hidden, C = c.num_embodiments;
+  std::vector<WeightSpec> v;
+  auto add = [&](const std::string& n, std::vector<int64_t> s) { v.push_back({n, s}); };
+  add("t_enc.l1.w", {D, c.time_freq_dim});
+  add("t_enc.l1.b", {D});
+  add("t_enc.l2.w", {D, D});
+  add("t_enc.l2.b", {D});
+  for (int l = 0; l < c.num_layers; ++l) {
+    const int64_t din = (l % 2 == 0) ? c.backbone_dim : D;
+    const std::string p = "blk" + std::to_string(l) + ".";
+    add(p + "ada.w", {2 * D, D});
+    add(p + "ada.b", {2 * D});
+    add(p + "q.w", {D, D});
+    add(p + "q.b", {D});
+    add(p + "k.w", {D, din});
+    add(p + "k.b", {D});
+    add(p + "v.w", {D, din});
+    add(p + "v.b", {D});
+    add(p + "o.w", {D, D});
+    add(p + "o.b", {D});
+    add(p + "ln3.g", {D});
+    add(p + "ln3.b", {D});
+    add(p + "ff1.w", {F, D});
+    add(p + "ff1.b", {F});
+    add(p + "ff2.w", {D, F});
+    add(p + "ff2.b", {D});
+  }
+  add("out.ada.w", {2 * D, D});
+  add("out.ada.b", {2 * D});
+  add("out.proj.w", {D, D});
+  add("out.proj.b", {D});
+  add("state_enc.l1.W", {C, c.state_dim, D});
+  add("state_enc.l1.b", {C, D});
+  add("state_enc.l2.W", {C, D, D});
+  add("state_enc.l2.b", {C, D});
+  add("act_enc.W1.W", {C, c.action_dim, D});
+  add("act_enc.W1.b", {C, D});
+  add("act_enc.W2.W", {C, 2 * D, D});
+  add("act_enc.W2.b", {C, D});
+  add("act_enc.W3.W", {C, D, D});
+  add("act_enc.W3.b", {C, D});
+  add("act_dec.l1.W", {C, D, D});
+  add("act_dec.l1.b", {C, D});
+  add("act_dec.l2.W", {C, D, c.action_dim});
+  add("act_dec.l2.b", {C, c.action_dim});
+  return v;
+}
+
+// Host view of one weight as f32 values (converted from bf16 if needed).
+struct HostW {
+  const gdit_tensor* t;
+  int64_t numel;
+  float at(int64_t i) const {
+    if (t->dtype == GDIT_F32) return static_cast<const float*>(t->host_ptr)[i];
+    return bf16_to_f32(static_cast<const uint16_t*>(t->host_ptr)[i]);
+  }
+};
+
+std::unordered_map<std::string, HostW> check_weights(const gdit_config& c, const gdit_tensor* ws, int n) {
+  REQUIRE(ws != nullptr || n == 0, "weights is NULL");
+  std::unordered_map<std::string, HostW> got;
+  for (int i = 0; i < n; ++i) {
+    const gdit_tensor& t = ws[i];
+    REQUIRE(t.name != nullptr, "weight %d has no name", i);
+    REQUIRE(got.find(t.name) == got.end(), "weight '%s' given twice", t.name);
+    REQUIRE(t.dtype == GDIT_F32 || t.dtype == GDIT_BF16, "weight '%s': dtype must be GDIT_F32 or GDIT_BF16",
+            t.name);
+    REQUIRE(t.ndim >= 1 && t.ndim <= 4 && t.shape != nullptr, "weight '%s': bad ndim/shape", t.name);
+    REQUIRE(t.host_ptr != nullptr, "weight '%s': host_ptr is NULL", t.name);
+    int64_t numel = 1;
+    for (int d = 0; d < t.ndim; ++d) numel *= t.shape[d];
+    got[t.name] = HostW{&t, numel};
+  }
+  const auto specs = weight_specs(c);
+  for (const auto& s : specs) {
+    auto it = got.find(s.name);
+    REQUIRE(it != got.end(), "missing weight '%s'", s.name.c_str());
+    const gdit_tensor* t = it->second.t;
+    bool ok = t->ndim == (int)s.shape.size();
+    for (int d = 0; ok && d < t->ndim; ++d) ok = t->shape[d] == s.shape[d];
+    if (!ok) {
+      std::string want, have;
+      for (auto x : s.shape) want += std::to_string(x) + ",";
+      for (int d = 0; d < t->ndim; ++d) have += std::to_string(t->shape[d]) + ",";
+      throw GditError(GDIT_EINVAL, fmt("weight '%s' has shape [%s] but [%s] is required", s.name.c_str(),
+                                       have.c_str(), want.c_str()));
+    }
+  }
+  REQUIRE(got.size() == specs.size(), "%zu unknown weight name(s) given (expected exactly %zu tensors)",
+          got.size() - specs.size(), specs.size());
+  return got;
+}
+
+// ------------------------------------------------------------------ upload
+
+struct Uploader {
+  gdit_handle* h;
+  std::vector<uint16_t> hb;
+  std::vector<float> hf;
+
+  __nv_bfloat16* mat(size_t n) { return h->dalloc<__nv_bfloat16>(n); }
+
+  // rows of `src` (a [rows, cols] row-major weight) -> bf16 at dst + row_off * cols
+  void put_rows(__nv_bfloat16* dst, const HostW& w, size_t count) {
+    hb.resize(count);
+    for (size_t i = 0; i < count; ++i) hb[i] = f32_to_bf16_rne(w.at((int64_t)i));
+    CUDA_TRY(cudaMemcpy(dst, hb.data(), count * 2, cudaMemcpyHostToDevice));
+  }
+  __nv_bfloat16* matrix(const HostW& w) {
+    __nv_bfloat16* d = mat((size_t)w.numel);
+    put_rows(d, w, (size_t)w.numel);
+    return d;
+  }
+  // [C, in, out] -> [C, out, in] restricted to input rows [in0, in0 + nin)
+  __nv_bfloat16* cat_transposed(const HostW& w, int C, int in, int out, int in0, int nin) {
+    __nv_bfloat16* d = mat((size_t)C * out * nin);
+    hb.resize((size_t)C * out * nin);
+    for (int c = 0; c < C; ++c)
+      for (int o = 0; o < out; ++o)
+        for (int i = 0; i < nin; ++i)
+          hb[((size_t)c * out + o) * nin + i] = f32_to_bf16_rne(w.at(((int64_t)c * in + in0 + i) * out + o));
+    CUDA_TRY(cudaMemcpy(d, hb.data(), hb.size() * 2, cudaMemcpyHostToDevice));
+    return d;
+  }
+  float* vec(const HostW& w) {
+    float* d = h->dalloc<float>((size_t)w.numel);
+    hf.resize((size_t)w.numel);
+    for (int64_t i = 0; i < w.numel; ++i) hf[i] = w.at(i);
+    CUDA_TRY(cudaMemcpy(d, hf.data(), hf.size() * 4, cudaMemcpyHostToDevice));
+    return d;
+  }
+  void vec_into(float* d, const HostW& w) {
+    hf.resize((size_t)w.numel);
+    for (int64_t i = 0; i < w.numel; ++i) hf[i] = w.at(i);
+    CUDA_TRY(cudaMemcpy(d, hf.data(), hf.size() * 4, cudaMemcpyHostToDevice));
+  }
+};
+
+void upload_model(gdit_handle* h, const std::unordered_map<std::string, HostW>& W) {
+  Uploader up{h, {}, {}};
+  const int D = h->D, F = h->F, L = h->L, C = h->C, Dvl = h->Dvl, A = h->A, Sd = h->Sd;
+  DevModel& m = h->w;
+  auto get = [&](const std::string& n) -> const HostW& { return W.at(n); };
+  m.t1w = up.matrix(get("t_enc.l1.w"));
+  m.t1b = up.vec(get("t_enc.l1.b"));
+  m.t2w = up.matrix(get("t_enc.l2.w"));
+  m.t2b = up.vec(get("t_enc.l2.b"));
+  // AdaLN weights of the L blocks and of norm_out, contiguous: [(L+1)][2D][D]
+  m.ada_w = up.mat((size_t)(L + 1) * 2 * D * D);
+  m.ada_b = h->dalloc<float>((size_t)(L + 1) * 2 * D);
+  for (int l = 0; l <= L; ++l) {
+    const std::string p = l < L ? "blk" + std::to_string(l) + ".ada" : std::string("out.ada");
+    up.put_rows(m.ada_w + (size_t)l * 2 * D * D, get(p + ".w"), (size_t)2 * D * D);
+    up.vec_into(m.ada_b + (size_t)l * 2 * D, get(p + ".b"));
+  }
+  // K/V weights of all cross layers: [Lc][2][D][Dvl] rows, biases [Lc][2D]
+  m.wkv = up.mat((size_t)h->Lc * 2 * D * Dvl);
+  m.bkv = h->dalloc<float>((size_t)h->Lc * 2 * D);
+  m.wq.resize(L);
+  m.bq.resize(L);
+  m.wo.resize(L);
+  m.bo.resize(L);
+  m.ln3g.resize(L);
+  m.ln3b.resize(L);
+  m.wff1.resize(L);
+  m.bff1.resize(L);
+  m.wff2.resize(L);
+  m.bff2.resize(L);
+  for (int l = 0; l < L; ++l) {
+    const std::string p = "blk" + std::to_string(l) + ".";
+    if (l % 2 == 0) {
+      const int li = l / 2;
+      up.put_rows(m.wkv + (size_t)li * 2 * D * Dvl, get(p + "k.w"), (size_t)D * Dvl);
+      up.put_rows(m.wkv + (size_t)li * 2 * D * Dvl + (size_t)D * Dvl, get(p + "v.w"), (size_t)D * Dvl);
+      up.vec_into(m.bkv + (size_t)li * 2 * D, get(p + "k.b"));
+      up.vec_into(m.bkv + (size_t)li * 2 * D + D, get(p + "v.b"));
+      m.wq[l] = up.matrix(get(p + "q.w"));
+      m.bq[l] = up.vec(get(p + "q.b"));
+    } else {
+      m.wq[l] = up.mat((size_t)3 * D * D);
+      up.put_rows(m.wq[l], get(p + "q.w"), (size_t)D * D);
+      up.put_rows(m.wq[l] + (size_t)D * D, get(p + "k.w"), (size_t)D * D);
+      up.put_rows(m.wq[l] + (size_t)2 * D * D, get(p + "v.w"), (size_t)D * D);
+      m.bq[l] = h->dalloc<float>((size_t)3 * D);
+      up.vec_into(m.bq[l], get(p + "q.b"));
+      up.vec_into(m.bq[l] + D, get(p + "k.b"));
+      up.vec_into(m.bq[l] + 2 * D, get(p + "v.b"));
+    }
+    m.wo[l] = up.matrix(get(p + "o.w"));
+    m.bo[l] = up.vec(get(p + "o.b"));
+    m.ln3g[l] = up.vec(get(p + "ln3.g"));
+    m.ln3b[l] = up.vec(get(p + "ln3.b"));
+    m.wff1[l] = up.matrix(get(p + "ff1.w"));
+    m.bff1[l] = up.vec(get(p + "ff1.b"));
+    m.wff2[l] = up.matrix(get(p + "ff2.w"));
+    m.bff2[l] = up.vec(get(p + "ff2.b"));
+  }
+  m.proj_w = up.matrix(get("out.proj.w"));
+  m.proj_b = up.vec(get("out.proj.b"));
+  // category-specific weights, transposed to [C][out][in] (K-major for the GEMM)
+  m.ws1t = up.cat_transposed(get("state_enc.l1.W"), C, Sd, D, 0, Sd);
+  m.bs1 = up.vec(get("state_enc.l1.b"));
+  m.ws2t = up.cat_transposed(get("state_enc.l2.W"), C, D, D, 0, D);
+  m.bs2 = up.vec(get("state_enc.l2.b"));
+  m.wa1t = up.cat_transposed(get("act_enc.W1.W"), C, A, D, 0, A);
+  m.ba1 = up.vec(get("act_enc.W1.b"));
+  m.wa2at = up.cat_transposed(get("act_enc.W2.W"), C, 2 * D, D, 0, D);       // action half
+  m.wa2taut = up.cat_transposed(get("act_enc.W2.W"), C, 2 * D, D, D, D);     // timestep half
+  m.ba2 = up.vec(get("act_enc.W2.b"));
+  m.wa3t = up.cat_transposed(get("act_enc.W3.W"), C, D, D, 0, D);
+  m.ba3 = up.vec(get("act_enc.W3.b"));
+  m.wd1t = up.cat_transposed(get("act_dec.l1.W"), C, D, D, 0, D);
+  m.bd1 = up.vec(get("act_dec.l1.b"));
+  m.wd2t = up.cat_transposed(get("act_dec.l2.W"), C, D, A, 0, D);
+  m.bd2 = up.vec(get("act_dec.l2.b"));
+}
+
+void alloc_workspace(gdit_handle* h) {
+  const long long Bm = h->cfg.max_batch, Sm = h->cfg.max_backbone_seq;
+  const int D = h->D, F = h->F, N = h->N, H = h->H, A = h->A;
+  h->max_tok = Bm * Sm;
+  h->xp = h->dalloc<__nv_bfloat16>((size_t)h->max_tok * h->Dvl);
+  h->kv = h->dalloc<__nv_bfloat16>((size_t)h->Lc * h->max_tok * 2 * D);
+  h->h = h->dalloc<float>((size_t)Bm * N * D);
+  h->u = h->dalloc<__nv_bfloat16>((size_t)Bm * N * D);
+  h->qkv = h->dalloc<__nv_bfloat16>((size_t)Bm * N * 3 * D);
+  h->o = h->dalloc<__nv_bfloat16>((size_t)Bm * N * D);
+  h->f = h->dalloc<__nv_bfloat16>((size_t)Bm * N * F);
+  h->x = h->dalloc<float>((size_t)Bm * H * A);
+  h->xb = h->dalloc<__nv_bfloat16>((size_t)Bm * H * A);
+  h->abf = h->dalloc<__nv_bfloat16>((size_t)Bm * H * D);
+  h->zbf = h->dalloc<__nv_bfloat16>((size_t)Bm * H * D);
+  h->ybf = h->dalloc<__nv_bfloat16>((size_t)Bm * H * D);
+  h->rbf = h->dalloc<__nv_bfloat16>((size_t)Bm * H * D);
+  h->sb = h->dalloc<__nv_bfloat16>((size_t)Bm * h->Sd);
+  h->s1 = h->dalloc<__nv_bfloat16>((size_t)Bm * D);
+  h->sfeat = h->dalloc<float>((size_t)Bm * D);
+  h->perm = h->dalloc<int>((size_t)Bm);
+  h->seg = h->dalloc<int>((size_t)h->C + 1);
+  h->vofs = h->dalloc<int>((size_t)Bm + 1);
+  h->bad = h->dalloc<uint8_t>((size_t)Bm);
+  h->status = h->dalloc<unsigned>(1);
+  h->io = h->dalloc<IoPtrs>(1);
+  h->ws = h->dalloc<float>((size_t)kWsFloats);
+  h->counters = h->dalloc<int>((size_t)kCounters);
+  CUDA_TRY(cudaMemset(h->counters, 0, sizeof(int) * kCounters));
+  CUDA_TRY(cudaMemset(h->status, 0, sizeof(unsigned)));
+  CUDA_TRY(cudaMemset(h->h, 0, sizeof(float) * (size_t)Bm * N * D));
+}
+
+void set_kernel_attrs() {
+  static bool done = false;
+  if (done) return;
+  set_gemm_attr<32>();
+  set_gemm_attr<64>();
+  set_gemm_attr<128>();
+  set_gemm_attr<256>();
+  CUDA_TRY(cudaFuncSetAttribute(attention_kernel<2, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                AttnSmem<2, 64>::TOTAL));
+  CUDA_TRY(cudaFuncSetAttribute(attention_kernel<4, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                AttnSmem<4, 64>::TOTAL));
+  CUDA_TRY(cudaFuncSetAttribute(attention_kernel<2, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                AttnSmem<2, 32>::TOTAL));
+  CUDA_TRY(cudaFuncSetAttribute(attention_kernel<4, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                AttnSmem<4, 32>::TOTAL));
+  done = true;
+}
+
+// ------------------------------------------------------------------ tables
+
+void compute_tables(gdit_handle* h, int K, cudaStream_t s) {
+  if (h->tables.count(K)) return;
+  Tables t;
+  t.K = K;
+  const int D = h->D, L = h->L, C = h->C, Tf = h->Tf;
+  // t_k = k / K; t_discretized = floor(t_k * buckets), in double (Isaac-GR00T
+  // architecture page, "Inference (denoising)"; GR00T model class page,
+  // num_timestep_buckets).
+  for (int k = 0; k < K; ++k) {
+    const double tk = (double)k / (double)K;
+    t.td.push_back((float)std::floor(tk * (double)h->cfg.num_timestep_buckets));
+  }
+  t.ada = h->dalloc<float>((size_t)K * (L + 1) * 2 * D);
+  t.tw2 = h->dalloc<float>((size_t)K * C * D);
+  float* td = h->dalloc<float>((size_t)K);
+  float* phiT = h->dalloc<float>((size_t)K * Tf);
+  float* phiD = h->dalloc<float>((size_t)K * D);
+  float* t1 = h->dalloc<float>((size_t)K * D);
+  float* temb = h->dalloc<float>((size_t)K * D);
+  CUDA_TRY(cudaMemcpyAsync(td, t.td.data(), sizeof(float) * K, cudaMemcpyHostToDevice, s));
+  const int thr = 256;
+  sinusoid_kernel<<<(K * Tf + thr - 1) / thr, thr, 0, s>>>(td, K, Tf, phiT);
+  sinusoid_kernel<<<(K * D + thr - 1) / thr, thr, 0, s>>>(td, K, D, phiD);
+  // TimestepEncoder: temb = L2(SiLU(L1(phi_Tf(td))))
+  gemv_rows_kernel<<<(D + 7) / 8, 256, 0, s>>>(h->w.t1w, D, Tf, phiT, K, h->w.t1b, 0, 1, t1, D);
+  gemv_rows_kernel<<<(D + 7) / 8, 256, 0, s>>>(h->w.t2w, D, D, t1, K, h->w.t2b, 0, 0, temb, D);
+  // AdaLN modulation of every block and of norm_out: Lin_l(SiLU(temb)) -> [K][L+1][2D]
+  const int R = (L + 1) * 2 * D;
+  gemv_rows_kernel<<<(R + 7) / 8, 256, 0, s>>>(h->w.ada_w, R, D, temb, K, h->w.ada_b, 1, 0, t.ada, R);
+  // timestep half of the action encoder's W2 (+ its bias): phi_D(td) W2[c][D:2D] + b2[c] -> [K][C][D]
+  gemv_rows_kernel<<<(C * D + 7) / 8, 256, 0, s>>>(h->w.wa2taut, C * D, D, phiD, K, h->w.ba2, 0, 0, t.tw2,
+                                                  (long long)C * D);
+  CUDA_TRY(cudaGetLastError());
+  h->tables[K] = std::move(t);
+}
+
+// ------------------------------------------------------------------ planning
+
+GemmOp plan_gemm(gdit_handle* h, const void* A, long long a_rows, int K, const void* Bw, long long b_rows, int N,
+                 int epi, long long rows_est, int groups, int rows_per_sample, int groups_est) {
+  GemmOp op;
+  op.args = default_args();
+  GemmArgs& a = op.args;
+  a.M = (int)a_rows;
+  a.N = N;
+  a.K = K;
+  a.num_groups = groups;
+  a.seg = groups ? h->seg : nullptr;
+  a.rows_per_sample = rows_per_sample;
+  a.b_group_rows = N;
+  a.epi = epi;
+  a.ws = h->ws;
+  a.counters = h->counters;
+  a.err = h->status;
+  int bn, splits;
+  choose_tiling(rows_est, groups_est, N, K, h->num_sms, a_rows, bn, splits);
+  op.bn = bn;
+  a.splits = splits;
+  op.ta = make_tmap(A, a_rows, K, K, kBM);
+  op.tb = make_tmap(Bw, b_rows, K, K, bn);
+  const long long nt = (N + bn - 1) / bn;
+  long long max_units = ((a_rows + kBM - 1) / kBM + (groups ? std::min<long long>(groups, a_rows) : 0)) * nt;
+  if (splits > 1 && max_units > kCounters) throw GditError(GDIT_EINVAL, "too many split-K tiles");
+  op.grid = (int)std::max<long long>(1, std::min<long long>(max_units * splits, h->num_sms));
+  op.out_bytes = (epi <= EPI_SWISH_VEC_BF16) ? 2 : 4;
+  return op;
+}
+
+std::unique_ptr<Profile> build_profile(gdit_handle* h, int B, int S, int K, int bf16) {
+  auto p = std::make_unique<Profile>();
+  p->B = B;
+  p->S = S;
+  p->K = K;
+  p->bf16 = bf16;
+  const int D = h->D, F = h->F, N = h->N, H = h->H, A = h->A, C = h->C, Dvl = h->Dvl, Sd = h->Sd, L = h->L;
+  const long long rows = (long long)B * N;
+  const long long arows = (long long)B * H;
+  const int gest = std::min(B, C);
+  DevModel& m = h->w;
+
+  // cross-attention K/V of every cross layer, over the packed valid tokens:
+  // [tok, Dvl] x [Lc*2D, Dvl]^T -> KV [Lc][tok][2D] (column blocks of 2D)
+  p->kv = plan_gemm(h, h->xp, (long long)B * S, Dvl, m.wkv, (long long)h->Lc * 2 * D, h->Lc * 2 * D, EPI_BF16,
+                    (long long)B * S, 0, 0, 1);
+  p->kv.args.m_dev = h->vofs + B;
+  p->kv.args.bias = m.bkv;
+  p->kv.args.out = h->kv;
+  p->kv.args.ldo = 2 * D;
+  p->kv.args.nblk = 2 * D;
+  p->kv.args.blk_stride = h->max_tok * 2 * D;
+  p->kv.rows_kind = 1;
+  p->kv.weight_bytes = (long long)h->Lc * 2 * D * Dvl * 2;
+
+  // state encoder (CategorySpecificMLP, ReLU)
+  p->st1 = plan_gemm(h, h->sb, B, Sd, m.ws1t, (long long)C * D, D, EPI_RELU_BF16, B, C, 1, gest);
+  p->st1.args.bias = m.bs1;
+  p->st1.args.bias_gstride = D;
+  p->st1.args.out = h->s1;
+  p->st1.args.ldo = D;
+  p->st1.rows_kind = 2;
+  p->st2 = plan_gemm(h, h->s1, B, D, m.ws2t, (long long)C * D, D, EPI_F32, B, C, 1, gest);
+  p->st2.args.bias = m.bs2;
+  p->st2.args.bias_gstride = D;
+  p->st2.args.out = h->sfeat;
+  p->st2.args.ldo = D;
+  p->st2.rows_kind = 2;
+
+  // action encoder: a = x W1[c] + b1; z = swish(a W2a[c] + (phi(td) W2tau[c] + b2)); e = z W3[c] + b3 -> h rows 1..H
+  p->a1 = plan_gemm(h, h->xb, arows, A, m.wa1t, (long long)C * D, D, EPI_BF16, arows, C, H, gest);
+  p->a1.args.bias = m.ba1;
+  p->a1.args.bias_gstride = D;
+  p->a1.args.out = h->abf;
+  p->a1.args.ldo = D;
+  p->a1.rows_kind = 2;
+  p->a2 = plan_gemm(h, h->abf, arows, D, m.wa2at, (long long)C * D, D, EPI_SWISH_VEC_BF16, arows, C, H, gest);
+  p->a2.args.vec_gstride = D;   // vec set per step
+  p->a2.args.out = h->zbf;
+  p->a2.args.ldo = D;
+  p->a2.rows_kind = 2;
+  p->a3 = plan_gemm(h, h->zbf, arows, D, m.wa3t, (long long)C * D, D, EPI_F32, arows, C, H, gest);
+  p->a3.args.bias = m.ba3;
+  p->a3.args.bias_gstride = D;
+  p->a3.args.out = h->h;
+  p->a3.args.ldo = D;
+  p->a3.args.in_group = H;
+  p->a3.args.out_group = N;
+  p->a3.args.out_off = 1;
+  p->a3.rows_kind = 2;
+
+  // DiT blocks
+  p->q.resize(L);
+  p->o.resize(L);
+  p->ff1.resize(L);
+  p->ff2.resize(L);
+  for (int l = 0; l < L; ++l) {
+    const int nq = (l % 2 == 1) ? 3 * D : D;
+    p->q[l] = plan_gemm(h, h->u, rows, D, m.wq[l], nq, nq, EPI_BF16, rows, 0, 0, 1);
+    p->q[l].args.bias = m.bq[l];
+    p->q[l].args.out = h->qkv;
+    p->q[l].args.ldo = nq;
+    p->q[l].weight_bytes = (long long)nq * D * 2;
+    p->o[l] = plan_gemm(h, h->o, rows, D, m.wo[l], D, D, EPI_RESID_F32, rows, 0, 0, 1);
+    p->o[l].args.bias = m.bo[l];
+    p->o[l].args.out = h->h;
+    p->o[l].args.ldo = D;
+    p->o[l].weight_bytes = (long long)D * D * 2;
+    p->ff1[l] = plan_gemm(h, h->u, rows, D, m.wff1[l], F, F, EPI_GELU_BF16, rows, 0, 0, 1);
+    p->ff1[l].args.bias = m.bff1[l];
+    p->ff1[l].args.out = h->f;
+    p->ff1[l].args.ldo = F;
+    p->ff1[l].weight_bytes = (long long)F * D * 2;
+    p->ff2[l] = plan_gemm(h, h->f, rows, F, m.wff2[l], D, D, EPI_RESID_F32, rows, 0, 0, 1);
+    p->ff2[l].args.bias = m.bff2[l];
+    p->ff2[l].args.out = h->h;
+    p->ff2[l].args.ldo = D;
+    p->ff2[l].weight_bytes = (long long)D * F * 2;
+  }
+  // norm_out + proj_out on every token; only the H action rows are kept (compact)
+  p->proj = plan_gemm(h, h->u, rows, D, m.proj_w, D, D, EPI_BF16, rows, 0, 0, 1);
+  p->proj.args.bias = m.proj_b;
+  p->proj.args.out = h->ybf;
+  p->proj.args.ldo = D;
+  p->proj.args.in_group = N;
+  p->proj.args.in_skip = 1;
+  p->proj.args.out_group = H;
+  p->proj.weight_bytes = (long long)D * D * 2;
+  // action decoder (CategorySpecificMLP, ReLU), Euler update fused into layer 2
+  p->d1 = plan_gemm(h, h->ybf, arows, D, m.wd1t, (long long)C * D, D, EPI_RELU_BF16, arows, C, H, gest);
+  p->d1.args.bias = m.bd1;
+  p->d1.args.bias_gstride = D;
+  p->d1.args.out = h->rbf;
+  p->d1.args.ldo = D;
+  p->d1.rows_kind = 2;
+  p->d2 = plan_gemm(h, h->rbf, arows, D, m.wd2t, (long long)C * A, A, EPI_EULER, arows, C, H, gest);
+  p->d2.args.bias = m.bd2;
+  p->d2.args.bias_gstride = A;
+  p->d2.args.out = h->x;
+  p->d2.args.ldo = A;
+  p->d2.args.out2 = h->xb;
+  p->d2.args.ldo2 = A;
+  p->d2.args.alpha = 1.0f / (float)K;
+  p->d2.rows_kind = 2;
+  for (GemmOp* g : {&p->st1, &p->st2, &p->a1, &p->a2, &p->a3, &p->d1, &p->d2})
+    g->weight_bytes = (long long)g->args.N * g->args.K * 2;   // per category used
+  return p;
+}
+
+// ------------------------------------------------------------------ enqueue
+
+struct Launcher {
+  gdit_handle* h;
+  cudaStream_t s;
+  Recorder* rec;
+
+  template <typename F>
+  void timed(const char* name, double flops, double bytes, const GemmOp* op, F&& fn) {
+    if (rec == nullptr) {
+      fn();
+      return;
+    }
+    Recorder::Ev e;
+    e.cls = rec->cls(name);
+    e.flops = flops;
+    e.bytes = bytes;
+    e.op = op;
+    CUDA_TRY(cudaEventCreate(&e.a));
+    CUDA_TRY(cudaEventCreate(&e.b));
+    CUDA_TRY(cudaEventRecord(e.a, s));
+    fn();
+    CUDA_TRY(cudaEventRecord(e.b, s));
+    rec->evs.push_back(e);
+  }
+  void gemm(const char* name, const GemmOp& op, const GemmArgs* over = nullptr) {
+    timed(name, 0, 0, &op, [&] { launch_gemm(op, over ? *over : op.args, s, h->pdl); });
+  }
+};
+
+void enqueue_forward(gdit_handle* h, Profile& p, cudaStream_t s, Recorder* rec) {
+  Launcher lx{h, s, rec};
+  const int B = p.B, S = p.S, K = p.K;
+  const int D = h->D, N = h->N, H = h->H, A = h->A, L = h->L, C = h->C, Dvl = h->Dvl;
+  const int rows = B * N;
+  const Tables& t = h->tables.at(K);
+  const bool pdl = h->pdl;
+  const int vec = D / 128;
+  const float eps = h->cfg.ln_eps;
+  auto ln = [&](const float* p0, const float* p1, int mode, const float* restore) {
+    const dim3 grid((rows + 7) / 8);
+    lx.timed("layernorm", 0, (double)rows * D * 6, nullptr, [&] {
+      switch (vec) {
+        case 1: launch_k(s, pdl, layernorm_kernel<1>, grid, dim3(256), 0, h->h, rows, p0, p1, mode, eps, h->u, restore, N); break;
+        case 2: launch_k(s, pdl, layernorm_kernel<2>, grid, dim3(256), 0, h->h, rows, p0, p1, mode, eps, h->u, restore, N); break;
+        case 4: launch_k(s, pdl, layernorm_kernel<4>, grid, dim3(256), 0, h->h, rows, p0, p1, mode, eps, h->u, restore, N); break;
+        case 8: launch_k(s, pdl, layernorm_kernel<8>, grid, dim3(256), 0, h->h, rows, p0, p1, mode, eps, h->u, restore, N); break;
+        default: launch_k(s, pdl, layernorm_kernel<16>, grid, dim3(256), 0, h->h, rows, p0, p1, mode, eps, h->u, restore, N); break;
+      }
+    });
+  };
+  auto attn = [&](const char* name, const AttnArgs& aa) {
+    const dim3 grid(B * h->cfg.num_heads), block(kAttnThreads);
+    lx.timed(name, 0, 0, nullptr, [&] {
+      if (h->cfg.head_dim == 64) {
+        if (N <= 32) launch_k(s, pdl, attention_kernel<2, 64>, grid, block, AttnSmem<2, 64>::TOTAL, aa);
+        else launch_k(s, pdl, attention_kernel<4, 64>, grid, block, AttnSmem<4, 64>::TOTAL, aa);
+      } else {
+        if (N <= 32) launch_k(s, pdl, attention_kernel<2, 32>, grid, block, AttnSmem<2, 32>::TOTAL, aa);
+        else launch_k(s, pdl, attention_kernel<4, 32>, grid, block, AttnSmem<4, 32>::TOTAL, aa);
+      }
+    });
+  };
+
+  // routing, packing, gathers
+  lx.timed("route_pack", 0, 0, nullptr, [&] {
+    launch_k(s, pdl, route_kernel, dim3(1), dim3(kRouteThreads), 0, (const IoPtrs*)h->io, B, S, C, h->perm, h->seg,
+             h->vofs, h->bad, h->status);
+  });
+  lx.timed("route_pack", 0, (double)B * S * Dvl * (p.bf16 ? 4 : 6), nullptr, [&] {
+    launch_k(s, pdl, pack_features_kernel, dim3(B, (S + 31) / 32), dim3(kPackThreads), 0, (const IoPtrs*)h->io,
+             p.bf16, S, Dvl, (const int*)h->perm, (const int*)h->vofs, h->xp);
+  });
+  lx.timed("route_pack", 0, 0, nullptr, [&] {
+    launch_k(s, pdl, gather_inputs_kernel, dim3(B), dim3(128), 0, (const IoPtrs*)h->io, B, H * A, h->Sd,
+             (const int*)h->perm, h->x, h->xb, h->sb);
+  });
+  lx.gemm("gemm_kv_proj", p.kv);
+  lx.gemm("gemm_embodiment", p.st1);
+  lx.gemm("gemm_embodiment", p.st2);
+
+  const float scale_log2 = 1.4426950408889634f / std::sqrt((float)h->cfg.head_dim);
+  for (int k = 0; k < K; ++k) {
+    GemmArgs a2 = p.a2.args;
+    a2.vec = t.tw2 + (size_t)k * C * D;
+    lx.gemm("gemm_embodiment", p.a1);
+    lx.gemm("gemm_embodiment", p.a2, &a2);
+    lx.gemm("gemm_embodiment", p.a3);
+    const float* ada_k = t.ada + (size_t)k * (L + 1) * 2 * D;
+    for (int l = 0; l < L; ++l) {
+      const float* ada = ada_k + (size_t)l * 2 * D;
+      ln(ada, ada + D, 0, l == 0 ? h->sfeat : nullptr);
+      lx.gemm("gemm_dit", p.q[l]);
+      AttnArgs aa;
+      aa.q = h->qkv;
+      aa.n_tok = N;
+      aa.num_heads = h->cfg.num_heads;
+      aa.out = h->o;
+      aa.out_ld = D;
+      aa.scale_log2 = scale_log2;
+      if (l % 2 == 1) {
+        aa.q_ld = 3 * D;
+        aa.k = h->qkv + D;
+        aa.v = h->qkv + 2 * D;
+        aa.kv_ld = 3 * D;
+        aa.kofs = nullptr;
+        attn("attn_self", aa);
+      } else {
+        const __nv_bfloat16* kvl = h->kv + (size_t)(l / 2) * h->max_tok * 2 * D;
+        aa.q_ld = D;
+        aa.k = kvl;
+        aa.v = kvl + D;
+        aa.kv_ld = 2 * D;
+        aa.kofs = h->vofs;
+        attn("attn_cross", aa);
+      }
+      lx.gemm("gemm_dit", p.o[l]);
+      ln(h->w.ln3g[l], h->w.ln3b[l], 1, nullptr);
+      lx.gemm("gemm_dit", p.ff1[l]);
+      lx.gemm("gemm_dit", p.ff2[l]);
+    }
+    const float* ada = ada_k + (size_t)L * 2 * D;
+    ln(ada, ada + D, 0, nullptr);
+    lx.gemm("gemm_dit", p.proj);
+    lx.gemm("gemm_embodiment", p.d1);
+    lx.gemm("gemm_embodiment", p.d2);
+  }
+  lx.timed("route_pack", 0, 0, nullptr, [&] {
+    launch_k(s, pdl, scatter_out_kernel, dim3(B), dim3(128), 0, (const IoPtrs*)h->io, H * A, (const int*)h->perm,
+             (const uint8_t*)h->bad, (const float*)h->x);
+  });
+}
+
+Profile& get_profile(gdit_handle* h, int B, int S, int K, int bf16, bool allow_build) {
+  const auto key = std::make_tuple(B, S, K, bf16);
+  auto it = h->profiles.find(key);
+  if (it != h->profiles.end()) return *it->second;
+  if (!allow_build)
+    throw GditError(GDIT_EPROFILE, fmt("profile (batch=%d, seq=%d, steps=%d, bf16=%d) was not prepared", B, S, K, bf16));
+  auto p = build_profile(h, B, S, K, bf16);
+  if (h->use_graph) {
+    if (h->cap_stream == nullptr) CUDA_TRY(cudaStreamCreateWithFlags(&h->cap_stream, cudaStreamNonBlocking));
+    cudaGraph_t graph = nullptr;
+    CUDA_TRY(cudaStreamBeginCapture(h->cap_stream, cudaStreamCaptureModeThreadLocal));
+    try {
+      enqueue_forward(h, *p, h->cap_stream, nullptr);
+    } catch (...) {
+      cudaStreamEndCapture(h->cap_stream, &graph);
+      if (graph) cudaGraphDestroy(graph);
+      throw;
+    }
+    CUDA_TRY(cudaStreamEndCapture(h->cap_stream, &graph));
+    cudaError_t e = cudaGraphInstantiate(&p->exec, graph, 0);
+    cudaGraphDestroy(graph);
+    CUDA_TRY(e);
+  }
+  Profile& ref = *p;
+  h->profiles[key] = std::move(p);
+  return ref;
+}
+
+void check_call(gdit_handle* h, const void* feats, int bb_dtype, const void* mask, const void* state, const void* ids,
+                const void* noise, int K, const void* out, int B, int S) {
+  REQUIRE(h != nullptr, "handle is NULL");
+  REQUIRE(feats && mask && state && ids && noise && out, "a required pointer argument is NULL");
+  REQUIRE(bb_dtype == GDIT_F32 || bb_dtype == GDIT_BF16, "bb_dtype must be GDIT_F32 or GDIT_BF16");
+  REQUIRE(K >= 1 && K <= 64, "num_steps must be in [1, 64] (got %d)", K);
+  REQUIRE(B >= 1 && B <= h->cfg.max_batch, "batch %d outside [1, max_batch=%d]", B, h->cfg.max_batch);
+  REQUIRE(S >= 1 && S <= h->cfg.max_backbone_seq, "seq %d outside [1, max_backbone_seq=%d]", S,
+          h->cfg.max_backbone_seq);
+  REQUIRE(((uintptr_t)feats & 15u) == 0, "backbone_features must be 16-byte aligned");
+}
+
+void run_call(gdit_handle* h, const void* feats, int bb_dtype, const uint8_t* mask, const float* state,
+              const int32_t* ids, const float* noise, int K, float* out, int B, int S, cudaStream_t s) {
+  CUDA_TRY(cudaSetDevice(h->cfg.device));
+  compute_tables(h, K, s);
+  Profile& p = get_profile(h, B, S, K, bb_dtype == GDIT_BF16, !h->strict);
+  IoPtrs io{feats, mask, state, ids, noise, out};
+  set_io_kernel<<<1, 1, 0, s>>>(h->io, io);
+  CUDA_TRY(cudaGetLastError());
+  if (p.exec != nullptr)
+    CUDA_TRY(cudaGraphLaunch(p.exec, s));
+  else
+    enqueue_forward(h, p, s, h->rec);
+  h->last_stream = s;
+  h->last_B = B;
+}
+
+template <typename F>
+int guarded(gdit_handle* h, F&& fn) {
+  try {
+    fn();
+    return GDIT_OK;
+  } catch (const GditError& e) {
+    if (h) h->last_error = e.what();
+    else g_create_error = e.what();
+    return e.code;
+  } catch (const std::bad_alloc&) {
+    if (h) h->last_error = "host allocation failed";
+    else g_create_error = "host allocation failed";
+    return GDIT_ENOMEM;
+  } catch (const std::exception& e) {
+    if (h) h->last_error = e.what();
+    else g_create_error = e.what();
+    return GDIT_ECUDA;
+  }
+}
+
+void free_handle(gdit_handle* h) {
+  if (!h) return;
+  cudaSetDevice(h->cfg.device);
+  cudaDeviceSynchronize();
+  for (auto& kv : h->profiles)
+    if (kv.second->exec) cudaGraphExecDestroy(kv.second->exec);
+  if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
+  for (void* p : h->allocs) cudaFree(p);
+  delete h;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+
+extern "C" {
+
+const char* gdit_version(void) { return "gdit 0.1 (sm_100a)"; }
+
+const char* gdit_strerror(int code) {
+  switch (code) {
+    case GDIT_OK: return "ok";
+    case GDIT_EINVAL: return "invalid argument";
+    case GDIT_ENOMEM: return "out of memory";
+    case GDIT_ECUDA: return "CUDA error";
+    case GDIT_EPROFILE: return "profile not prepared";
+    case GDIT_ETIMEOUT: return "device wait timed out";
+    case GDIT_EDEVICE: return "invalid input detected on the device";
+    case GDIT_ENODEV: return "no sm_100 device";
+    default: return "unknown error";
+  }
+}
+
+const char* gdit_last_error(const gdit_handle* h) { return h ? h->last_error.c_str() : g_create_error.c_str(); }
+
+int gdit_create(const gdit_config* cfg, const gdit_tensor* weights, int n_weights, gdit_handle** out) {
+  if (out) *out = nullptr;
+  gdit_handle* h = nullptr;
+  g_create_error.clear();
+  int rc = guarded(nullptr, [&] {
+    REQUIRE(cfg != nullptr && out != nullptr, "cfg and out must not be NULL");
+    validate_config(*cfg);
+    auto W = check_weights(*cfg, weights, n_weights);   // host-only checks first
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) throw GditError(GDIT_ENODEV, "no CUDA device");
+    REQUIRE(cfg->device >= 0 && cfg->device < ndev, "device %d out of range", cfg->device);
+    cudaDeviceProp prop;
+    CUDA_TRY(cudaGetDeviceProperties(&prop, cfg->device));
+    if (prop.major != 10) throw GditError(GDIT_ENODEV, fmt("device %d is sm_%d%d, sm_100 required", cfg->device, prop.major, prop.minor));
+    CUDA_TRY(cudaSetDevice(cfg->device));
+    h = new gdit_handle();
+    h->cfg = *cfg;
+    h->L = cfg->num_layers;
+    h->D = cfg->hidden;
+    h->F = cfg->mlp_hidden;
+    h->Dvl = cfg->backbone_dim;
+    h->A = cfg->action_dim;
+    h->Sd = cfg->state_dim;
+    h->H = cfg->action_horizon;
+    h->C = cfg->num_embodiments;
+    h->Tf = cfg->time_freq_dim;
+    h->N = cfg->action_horizon + 1;
+    h->Lc = cfg->num_layers / 2;
+    h->num_sms = prop.multiProcessorCount;
+    h->use_graph = (cfg->flags & GDIT_FLAG_NO_GRAPH) == 0;
+    h->strict = (cfg->flags & GDIT_FLAG_STRICT_PROFILES) != 0;
+    const char* pdl_env = getenv("GDIT_PDL");
+    h->pdl = !(pdl_env && pdl_env[0] == '0');
+    set_kernel_attrs();
+    upload_model(h, W);
+    alloc_workspace(h);
+    CUDA_TRY(cudaDeviceSynchronize());
+  });
+  if (rc != GDIT_OK) {
+    if (h) {
+      std::string msg = g_create_error;
+      free_handle(h);
+      g_create_error = msg;
+    }
+    return rc;
+  }
+  *out = h;
+  return GDIT_OK;
+}
+
+void gdit_destroy(gdit_handle* h) { free_handle(h); }
+
+int gdit_get_action(gdit_handle* h, const void* backbone_features, int bb_dtype, const uint8_t* vl_mask,
+                    const float* state, const int32_t* embodiment_id, const float* init_noise, int num_steps,
+                    float* out_actions, int batch, int seq, void* cuda_stream) {
+  if (!h) return GDIT_EINVAL;
+  return guarded(h, [&] {
+    check_call(h, backbone_features, bb_dtype, vl_mask, state, embodiment_id, init_noise, num_steps, out_actions,
+               batch, seq);
+    run_call(h, backbone_features, bb_dtype, vl_mask, state, embodiment_id, init_noise, num_steps, out_actions, batch,
+             seq, (cudaStream_t)cuda_stream);
+  });
+}
+
+int gdit_get_action_host(gdit_handle* h, const void* backbone_features, int bb_dtype, const uint8_t* vl_mask,
+                         const float* state, const int32_t* embodiment_id, const float* init_noise, int num_steps,
+                         float* out_actions, int batch, int seq, void* cuda_stream) {
+  if (!h) return GDIT_EINVAL;
+  return guarded(h, [&] {
+    check_call(h, backbone_features, GDIT_BF16, vl_mask, state, embodiment_id, init_noise, num_steps, out_actions,
+               batch, seq);
+    REQUIRE(bb_dtype == GDIT_F32 || bb_dtype == GDIT_BF16, "bb_dtype must be GDIT_F32 or GDIT_BF16");
+    CUDA_TRY(cudaSetDevice(h->cfg.device));
+    cudaStream_t s = (cudaStream_t)cuda_stream;
+    const size_t Bm = h->cfg.max_batch, Sm = h->cfg.max_backbone_seq;
+    const size_t esz = bb_dtype == GDIT_BF16 ? 2 : 4;
+    if (h->st_mask == nullptr) {
+      h->st_mask = h->dalloc<uint8_t>(Bm * Sm);
+      h->st_state = h->dalloc<float>(Bm * h->Sd);
+      h->st_ids = h->dalloc<int32_t>(Bm);
+      h->st_noise = h->dalloc<float>(Bm * h->H * h->A);
+      h->st_out = h->dalloc<float>(Bm * h->H * h->A);
+    }
+    const size_t fbytes = (size_t)batch * seq * h->Dvl * esz;
+    if (h->st_feats_bytes < fbytes) {
+      const size_t cap = Bm * Sm * h->Dvl * esz;
+      h->st_feats = h->dalloc<uint8_t>(std::max(cap, fbytes));
+      h->st_feats_bytes = std::max(cap, fbytes);
+    }
+    const size_t ha = (size_t)batch * h->H * h->A;
+    CUDA_TRY(cudaMemcpyAsync(h->st_feats, backbone_features, fbytes, cudaMemcpyHostToDevice, s));
+    CUDA_TRY(cudaMemcpyAsync(h->st_mask, vl_mask, (size_t)batch * seq, cudaMemcpyHostToDevice, s));
+    CUDA_TRY(cudaMemcpyAsync(h->st_state, state, (size_t)batch * h->Sd * 4, cudaMemcpyHostToDevice, s));
+    CUDA_TRY(cudaMemcpyAsync(h->st_ids, embodiment_id, (size_t)batch * 4, cudaMemcpyHostToDevice, s));
+    CUDA_TRY(cudaMemcpyAsync(h->st_noise, init_noise, ha * 4, cudaMemcpyHostToDevice, s));
+    run_call(h, h->st_feats, bb_dtype, h->st_mask, h->st_state, h->st_ids, h->st_noise, num_steps, h->st_out, batch,
+             seq, s);
+    CUDA_TRY(cudaMemcpyAsync(out_actions, h->st_out, ha * 4, cudaMemcpyDeviceToHost, s));
+    CUDA_TRY(cudaStreamSynchronize(s));
+  });
+}
+
+int gdit_prepare(gdit_handle* h, int batch, int seq, int num_steps, int bb_dtype, void* cuda_stream) {
+  if (!h) return GDIT_EINVAL;
+  return guarded(h, [&] {
+    REQUIRE(num_steps >= 1 && num_steps <= 64, "num_steps must be in [1, 64]");
+    REQUIRE(batch >= 1 && batch <= h->cfg.max_batch, "batch out of range");
+    REQUIRE(seq >= 1 && seq <= h->cfg.max_backbone_seq, "seq out of range");
+    REQUIRE(bb_dtype == GDIT_F32 || bb_dtype == GDIT_BF16, "bad bb_dtype");
+    CUDA_TRY(cudaSetDevice(h->cfg.device));
+    compute_tables(h, num_steps, (cudaStream_t)cuda_stream);
+    get_profile(h, batch, seq, num_steps, bb_dtype == GDIT_BF16, true);
+  });
+}
+
+int gdit_sync_status(gdit_handle* h) {
+  if (!h) return GDIT_EINVAL;
+  unsigned st = 0;
+  int rc = guarded(h, [&] {
+    CUDA_TRY(cudaSetDevice(h->cfg.device));
+    CUDA_TRY(cudaStreamSynchronize(h->last_stream));
+    CUDA_TRY(cudaMemcpy(&st, h->status, sizeof(unsigned), cudaMemcpyDeviceToHost));
+    CUDA_TRY(cudaMemset(h->status, 0, sizeof(unsigned)));
+    if (st & DEV_ERR_TIMEOUT) CUDA_TRY(cudaMemset(h->counters, 0, sizeof(int) * kCounters));
+  });
+  if (rc != GDIT_OK) return rc;
+  if (st & DEV_ERR_TIMEOUT) {
+    h->last_error = "a device-side wait timed out";
+    return GDIT_ETIMEOUT;
+  }
+  if (st & DEV_ERR_BAD_ID) {
+    h->last_error = "embodiment_id out of range (those samples are NaN)";
+    return GDIT_EDEVICE;
+  }
+  return GDIT_OK;
+}
+
+int gdit_debug_routing(gdit_handle* h, int32_t* perm, int32_t* seg, int32_t* vofs) {
+  if (!h) return GDIT_EINVAL;
+  return guarded(h, [&] {
+    REQUIRE(perm && seg && vofs, "NULL output");
+    REQUIRE(h->last_B > 0, "no call has run on this handle");
+    CUDA_TRY(cudaSetDevice(h->cfg.device));
+    CUDA_TRY(cudaStreamSynchronize(h->last_stream));
+    CUDA_TRY(cudaMemcpy(perm, h->perm, sizeof(int) * h->last_B, cudaMemcpyDeviceToHost));
+    CUDA_TRY(cudaMemcpy(seg, h->seg, sizeof(int) * (h->C + 1), cudaMemcpyDeviceToHost));
+    CUDA_TRY(cudaMemcpy(vofs, h->vofs, sizeof(int) * (h->last_B + 1), cudaMemcpyDeviceToHost));
+  });
+}
+
+int gdit_debug_kv(gdit_handle* h, int layer, float* k_out, float* v_out, int* total_valid) {
+  if (!h) return GDIT_EINVAL;
+  return guarded(h, [&] {
+    REQUIRE(total_valid != nullptr, "total_valid is NULL");
+    REQUIRE(layer >= 0 && layer < h->L && layer % 2 == 0, "layer %d is not a cross-attention layer", layer);
+    REQUIRE(h->last_B > 0, "no call has run on this handle");
+    CUDA_TRY(cudaSetDevice(h->cfg.device));
+    CUDA_TRY(cudaStreamSynchronize(h->last_stream));
+    int tot = 0;
+    CUDA_TRY(cudaMemcpy(&tot, h->vofs + h->last_B, sizeof(int), cudaMemcpyDeviceToHost));
+    *total_valid = tot;
+    if (k_out == nullptr && v_out == nullptr) return;
+    const int D = h->D;
+    std::vector<uint16_t> buf((size_t)tot * 2 * D);
+    if (tot > 0)
+      CUDA_TRY(cudaMemcpy(buf.data(), h->kv + (size_t)(layer / 2) * h->max_tok * 2 * D, buf.size() * 2,
+                          cudaMemcpyDeviceToHost));
+    for (int r = 0; r < tot; ++r)
+      for (int c = 0; c < D; ++c) {
+        if (k_out) k_out[(size_t)r * D + c] = bf16_to_f32(buf[(size_t)r * 2 * D + c]);
+        if (v_out) v_out[(size_t)r * D + c] = bf16_to_f32(buf[(size_t)r * 2 * D + D + c]);
+      }
+  });
+}
+
+int gdit_profile_get_action(gdit_handle* h, const void* backbone_features, int bb_dtype, const uint8_t* vl_mask,
+                            const float* state, const int32_t* embodiment_id, const float* init_noise, int num_steps,
+                            float* out_actions, int batch, int seq, void* cuda_stream, gdit_kernel_stat* stats,
+                            int max_stats) {
+  if (!h) return GDIT_EINVAL;
+  int count = 0;
+  Recorder rec;
+  int rc = guarded(h, [&] {
+    REQUIRE(stats != nullptr && max_stats > 0, "stats buffer required");
+    check_call(h, backbone_features, bb_dtype, vl_mask, state, embodiment_id, init_noise, num_steps, out_actions,
+               batch, seq);
+    CUDA_TRY(cudaSetDevice(h->cfg.device));
+    cudaStream_t s = (cudaStream_t)cuda_stream;
+    compute_tables(h, num_steps, s);
+    Profile& p = get_profile(h, batch, seq, num_steps, bb_dtype == GDIT_BF16, true);
+    IoPtrs io{backbone_features, vl_mask, state, embodiment_id, init_noise, out_actions};
+    set_io_kernel<<<1, 1, 0, s>>>(h->io, io);
+    CUDA_TRY(cudaGetLastError());
+    CUDA_TRY(cudaStreamSynchronize(s));
+    enqueue_forward(h, p, s, &rec);
+    h->last_stream = s;
+    h->last_B = batch;
+    CUDA_TRY(cudaStreamSynchronize(s));
+    // algorithmic work, now that the routing is known
+    std::vector<int> seg(h->C + 1), vofs(batch + 1);
+    CUDA_TRY(cudaMemcpy(seg.data(), h->seg, sizeof(int) * (h->C + 1), cudaMemcpyDeviceToHost));
+    CUDA_TRY(cudaMemcpy(vofs.data(), h->vofs, sizeof(int) * (batch + 1), cudaMemcpyDeviceToHost));
+    int used = 0;
+    for (int c = 0; c < h->C; ++c) used += seg[c + 1] > seg[c];
+    const double tok = vofs[batch];
+    std::vector<KStat> agg(rec.names.size());
+    for (size_t i = 0; i < rec.names.size(); ++i) agg[i].name = rec.names[i];
+    const int N = h->N, D = h->D;
+    for (auto& e : rec.evs) {
+      float ms = 0.0f;
+      CUDA_TRY(cudaEventElapsedTime(&ms, e.a, e.b));
+      KStat& k = agg[e.cls];
+      k.launches += 1;
+      k.ms += ms;
+      double fl = e.flops, by = e.bytes;
+      if (e.op != nullptr) {
+        const GemmArgs& a = e.op->args;
+        double m = a.M;
+        double wb = (double)e.op->weight_bytes;
+        if (e.op->rows_kind == 1) m = tok;
+        if (e.op->rows_kind == 2) wb *= used;
+        fl = 2.0 * m * a.N * a.K;
+        by = wb + m * a.K * 2.0 + m * a.N * e.op->out_bytes * (a.epi == EPI_RESID_F32 || a.epi == EPI_EULER ? 2 : 1);
+      }
+      if (rec.names[e.cls] == "attn_cross") {
+        fl = 4.0 * N * tok * D;
+        by = tok * 2.0 * D * 2.0 + 2.0 * batch * N * D * 2.0;
+      } else if (rec.names[e.cls] == "attn_self") {
+        fl = 4.0 * batch * (double)N * N * D;
+        by = batch * (double)N * 3 * D * 2.0 + batch * (double)N * D * 2.0;
+      }
+      k.flops += fl;
+      k.bytes += by;
+      cudaEventDestroy(e.a);
+      cudaEventDestroy(e.b);
+    }
+    rec.evs.clear();
+    for (auto& k : agg) {
+      if (count >= max_stats) break;
+      gdit_kernel_stat& o = stats[count++];
+      std::memset(&o, 0, sizeof(o));
+      std::snprintf(o.name, sizeof(o.name), "%s", k.name.c_str());
+      o.launches = k.launches;
+      o.total_ms = k.ms;
+      o.flops = k.flops;
+      o.bytes = k.bytes;
+    }
+  });
+  for (auto& e : rec.evs) {
+    cudaEventDestroy(e.a);
+    cudaEventDestroy(e.b);
+  }
+  return rc == GDIT_OK ? count : rc;
+}
+
+int gdit_test_gemm(const void* A, const void* B, const float* bias, float* C, int M, int N, int K, int bn, int splits,
+                   void* cuda_stream) {
+  g_create_error.clear();
+  return guarded(nullptr, [&] {
+    REQUIRE(A && B && C, "NULL matrix");
+    REQUIRE(M >= 1 && N >= 32 && N % 32 == 0 && K >= 8 && K % 8 == 0, "need M >= 1, N %% 32 == 0, K %% 8 == 0");
+    REQUIRE(bn == 32 || bn == 64 || bn == 128 || bn == 256, "bn must be 32, 64, 128 or 256");
+    const int nkb = (K + kBK - 1) / kBK;
+    REQUIRE(splits >= 1 && splits <= nkb, "splits must be in [1, %d]", nkb);
+    set_kernel_attrs();
+    int dev = 0;
+    CUDA_TRY(cudaGetDevice(&dev));
+    int sms = 0;
+    CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    cudaStream_t s = (cudaStream_t)cuda_stream;
+    float* ws = nullptr;
+    int* counters = nullptr;
+    unsigned* err = nullptr;
+    const long long nt = (N + bn - 1) / bn, mt = (M + kBM - 1) / kBM;
+    CUDA_TRY(cudaMalloc(&err, sizeof(unsigned)));
+    CUDA_TRY(cudaMemset(err, 0, sizeof(unsigned)));
+    if (splits > 1) {
+      CUDA_TRY(cudaMalloc(&ws, sizeof(float) * (size_t)splits * M * N));
+      CUDA_TRY(cudaMalloc(&counters, sizeof(int) * (size_t)(mt * nt)));
+      CUDA_TRY(cudaMemset(counters, 0, sizeof(int) * (size_t)(mt * nt)));
+    }
+    GemmOp op;
+    op.args = default_args();
+    op.args.M = M;
+    op.args.N = N;
+    op.args.K = K;
+    op.args.splits = splits;
+    op.args.ws = ws;
+    op.args.counters = counters;
+    op.args.epi = EPI_F32;
+    op.args.bias = bias;
+    op.args.out = C;
+    op.args.ldo = N;
+    op.args.err = err;
+    op.bn = bn;
+    op.ta = make_tmap(A, M, K, K, kBM);
+    op.tb = make_tmap(B, N, K, K, bn);
+    op.grid = (int)std::min<long long>(mt * nt * splits, sms);
+    launch_gemm(op, op.args, s, false);
+    CUDA_TRY(cudaStreamSynchronize(s));
+    unsigned e = 0;
+    CUDA_TRY(cudaMemcpy(&e, err, sizeof(unsigned), cudaMemcpyDeviceToHost));
+    cudaFree(err);
+    if (ws) cudaFree(ws);
+    if (counters) cudaFree(counters);
+    if (e) throw GditError(GDIT_ETIMEOUT, "GEMM wait timed out");
+  });
+}
+
+}  // extern "C"

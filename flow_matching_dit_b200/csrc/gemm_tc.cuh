@@ -1,0 +1,472 @@
+// Persistent bf16 GEMM on the 5th-generation tensor cores (tcgen05 + TMEM),
+// fed by TMA, with the action head's epilogues fused in.
+//
+//   C[m, n] = sum_k A[m, k] * B[n, k]      (A: activations, B: weights, both K-major)
+//
+// Used for every dense contraction of the action head: the cross-attention
+// K/V projection of the backbone features, the Q/QKV, O, FF1, FF2 and
+// proj_out linears of the DiT blocks (Isaac-GR00T architecture page,
+// "Transformer block structure"), and the CategorySpecificLinear layers of the
+// state encoder, action encoder and action decoder ("Embodiment-specific
+// projectors"), which run grouped: rows are sorted by embodiment and each
+// group multiplies by its own category's weights.
+//
+// CTA = 6 warps: warp 0 issues TMA loads into a STAGES-deep shared-memory
+// ring, warp 1 allocates TMEM and one thread issues tcgen05.mma (128 x BN x 16
+// per instruction) into one of two TMEM accumulators, warps 2-5 drain the
+// other accumulator through tcgen05.ld and run the epilogue.  Tiles are
+// 128 x BN (BN in {32, 64, 128, 256}) with 64-wide K blocks in the 128-byte
+// swizzled layout.  Split-K is deterministic: every split writes an f32
+// partial, and the last split to finish (per-tile counter) sums the partials
+// in split order and runs the epilogue.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace gdit {
+
+enum Epi : int {
+  EPI_BF16 = 0,            // out(bf16) = acc + bias
+  EPI_GELU_BF16 = 1,       // out(bf16) = gelu(acc + bias)           (FF1)
+  EPI_RELU_BF16 = 2,       // out(bf16) = relu(acc + bias)           (CategorySpecificMLP layer 1)
+  EPI_SWISH_VEC_BF16 = 3,  // out(bf16) = swish(acc + vec[g])        (action encoder W2)
+  EPI_F32 = 4,             // out(f32)  = acc + bias
+  EPI_RESID_F32 = 5,       // out(f32) += acc + bias                 (residual adds)
+  EPI_EULER = 6,           // x = out + alpha * (acc + bias); out = x; out2(bf16) = x   (velocity -> Euler)
+};
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kGemmThreads = 192;
+constexpr int kMaxGroups = 64;
+
+struct GemmArgs {
+  int M;                    // rows of A (dense) or row capacity (grouped)
+  int N, K;
+  const int* m_dev;         // dense: optional device row count (<= M)
+  int num_groups;           // 0 = dense
+  const int* seg;           // grouped: [num_groups + 1] sample offsets (device)
+  int rows_per_sample;      // grouped: rows of A per sample
+  int b_group_rows;         // grouped: rows of B per group (= N)
+  int splits;               // split-K factor
+  float* ws;                // split-K partials [splits][M][N]
+  int* counters;            // split-K per-unit arrival counters (zero between launches)
+  int epi;
+  const float* bias;
+  long long bias_gstride;   // bias of group g at bias + g * bias_gstride
+  const float* vec;
+  long long vec_gstride;
+  void* out;
+  long long ldo;
+  __nv_bfloat16* out2;
+  long long ldo2;
+  float alpha;
+  int in_group, in_skip, out_group, out_off;   // output row = (m / in_group) * out_group + m % in_group - in_skip + out_off
+  int nblk;                 // > 0: columns blocked by nblk, block j at out + j * blk_stride
+  long long blk_stride;
+  unsigned* err;
+};
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int A_BYTES = kBM * kBK * 2;
+  static constexpr int B_BYTES = BN * kBK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
+  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 256;
+  static constexpr uint32_t IDESC = idesc_bf16_f32(kBM, BN);
+};
+
+struct GemmSched {
+  int units;          // output tiles (without the split factor)
+  int nt;             // column tiles
+  int mt;             // dense: row tiles
+  int rows;           // dense: valid rows
+  int uprefix[kMaxGroups + 1];
+  int rstart[kMaxGroups];
+  int rend[kMaxGroups];
+};
+
+struct TileInfo {
+  int g, m0, m_end, n_idx, kb0, kb1, unit, split;   // n_idx: column tile index
+};
+
+__device__ __forceinline__ void gemm_decode(const GemmArgs& a, const GemmSched& s, int t, TileInfo& ti) {
+  const int u = t / a.splits;
+  ti.split = t - u * a.splits;
+  ti.unit = u;
+  int m_idx, n_idx;
+  if (a.num_groups == 0) {
+    constexpr int GM = 16;   // row-tile groups for L2 reuse of the B tiles
+    const int group_size = GM * s.nt;
+    const int gid = u / group_size;
+    const int first_m = gid * GM;
+    const int gm = min(s.mt - first_m, GM);
+    const int r = u - gid * group_size;
+    m_idx = first_m + r % gm;
+    n_idx = r / gm;
+    ti.g = 0;
+    ti.m0 = m_idx * kBM;
+    ti.m_end = s.rows;
+  } else {
+    int g = 0;
+    while (g + 1 < a.num_groups && s.uprefix[g + 1] <= u) ++g;
+    const int r = u - s.uprefix[g];
+    const int mt_g = (s.rend[g] - s.rstart[g] + kBM - 1) / kBM;
+    m_idx = r % mt_g;
+    n_idx = r / mt_g;
+    ti.g = g;
+    ti.m0 = s.rstart[g] + m_idx * kBM;
+    ti.m_end = s.rend[g];
+  }
+  ti.n_idx = n_idx;
+  const int nkb = (a.K + kBK - 1) / kBK;
+  ti.kb0 = (int)(((long long)ti.split * nkb) / a.splits);
+  ti.kb1 = (int)(((long long)(ti.split + 1) * nkb) / a.splits);
+}
+
+__device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
+__device__ __forceinline__ float swish_f(float x) { return x / (1.0f + __expf(-x)); }
+
+// Epilogue of 32 consecutive columns [n, n + 32) of row m (group g).
+__device__ __forceinline__ void gemm_epilogue32(const GemmArgs& a, int g, int m, int n, float (&v)[32]) {
+  const int gi = m / a.in_group;
+  const int ri = m - gi * a.in_group;
+  if (ri < a.in_skip) return;
+  const long long orow = (long long)gi * a.out_group + (ri - a.in_skip) + a.out_off;
+  long long col = n;
+  long long blk_off = 0;
+  if (a.nblk > 0) {
+    const int blk = n / a.nblk;
+    col = n - (long long)blk * a.nblk;
+    blk_off = (long long)blk * a.blk_stride;
+  }
+  const int epi = a.epi;
+  if (epi == EPI_SWISH_VEC_BF16) {
+    const float4* vp = reinterpret_cast<const float4*>(a.vec + (long long)g * a.vec_gstride + n);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float4 b = vp[j];
+      v[4 * j + 0] = swish_f(v[4 * j + 0] + b.x);
+      v[4 * j + 1] = swish_f(v[4 * j + 1] + b.y);
+      v[4 * j + 2] = swish_f(v[4 * j + 2] + b.z);
+      v[4 * j + 3] = swish_f(v[4 * j + 3] + b.w);
+    }
+  } else if (a.bias != nullptr) {
+    const float4* bp = reinterpret_cast<const float4*>(a.bias + (long long)g * a.bias_gstride + n);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float4 b = bp[j];
+      v[4 * j + 0] += b.x;
+      v[4 * j + 1] += b.y;
+      v[4 * j + 2] += b.z;
+      v[4 * j + 3] += b.w;
+    }
+  }
+  if (epi == EPI_GELU_BF16) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = gelu_erf(v[j]);
+  } else if (epi == EPI_RELU_BF16) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = fmaxf(v[j], 0.0f);
+  }
+  if (epi <= EPI_SWISH_VEC_BF16) {
+    __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) + blk_off + orow * a.ldo + col;
+    uint4* o4 = reinterpret_cast<uint4*>(o);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint4 w;
+      w.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
+      w.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+      w.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+      w.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+      o4[j] = w;
+    }
+    return;
+  }
+  float* o = reinterpret_cast<float*>(a.out) + blk_off + orow * a.ldo + col;
+  float4* o4 = reinterpret_cast<float4*>(o);
+  if (epi == EPI_F32) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) o4[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+  } else if (epi == EPI_RESID_F32) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float4 r = o4[j];
+      r.x += v[4 * j];
+      r.y += v[4 * j + 1];
+      r.z += v[4 * j + 2];
+      r.w += v[4 * j + 3];
+      o4[j] = r;
+    }
+  } else {  // EPI_EULER
+    uint4* x2 = reinterpret_cast<uint4*>(a.out2 + orow * a.ldo2 + col);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float4 r = o4[j];
+      r.x += a.alpha * v[4 * j];
+      r.y += a.alpha * v[4 * j + 1];
+      r.z += a.alpha * v[4 * j + 2];
+      r.w += a.alpha * v[4 * j + 3];
+      o4[j] = r;
+      v[4 * j] = r.x;
+      v[4 * j + 1] = r.y;
+      v[4 * j + 2] = r.z;
+      v[4 * j + 3] = r.w;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint4 w;
+      w.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
+      w.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+      w.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+      w.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+      x2[j] = w;
+    }
+  }
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const GemmArgs a) {
+  using Cfg = GemmCfg<BN>;
+  constexpr int STAGES = Cfg::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ GemmSched sched;
+  __shared__ uint32_t tmem_holder;
+  __shared__ int s_last;
+  __shared__ volatile int s_abort;
+
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * Cfg::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 128);
+    }
+    fence_mbar_init();
+    s_abort = 0;
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_holder, Cfg::TMEM_COLS);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  // Inputs (A, seg, m_dev, residuals) come from earlier kernels on the stream.
+  pdl_wait();
+  if (threadIdx.x == 0) {
+    sched.nt = (a.N + BN - 1) / BN;
+    if (a.num_groups == 0) {
+      int rows = a.M;
+      if (a.m_dev != nullptr) rows = min(rows, *a.m_dev);
+      rows = max(rows, 0);
+      sched.rows = rows;
+      sched.mt = (rows + kBM - 1) / kBM;
+      sched.units = sched.mt * sched.nt;
+    } else {
+      int u = 0;
+      for (int g = 0; g < a.num_groups; ++g) {
+        const int rs = a.seg[g] * a.rows_per_sample;
+        const int re = a.seg[g + 1] * a.rows_per_sample;
+        sched.rstart[g] = rs;
+        sched.rend[g] = re;
+        sched.uprefix[g] = u;
+        u += ((re - rs + kBM - 1) / kBM) * sched.nt;
+      }
+      sched.uprefix[a.num_groups] = u;
+      sched.units = u;
+    }
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_holder;
+  const int total = sched.units * a.splits;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        TileInfo ti;
+        gemm_decode(a, sched, t, ti);
+        const int brow = ti.g * a.b_group_rows + ti.n_idx * BN;
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, a.err)) { ok = false; s_abort = 1; break; }
+          if (s_abort) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
+          tma_load_2d(sA + stage * Cfg::A_BYTES, &tmA, &full[stage], kb * kBK, ti.m0);
+          tma_load_2d(sB + stage * Cfg::B_BYTES, &tmB, &full[stage], kb * kBK, brow);
+          ++issued;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (ok) {
+        // Producer tail: wait until the MMA warp has released every stage, so
+        // no tcgen05.commit arrival is still pending when the CTA exits.
+        for (int i = 0; i < STAGES; ++i) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, a.err)) break;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      } else {
+        // Let the loads already in flight land before the CTA can exit.
+        const unsigned long long t0 = globaltimer_ns();
+        for (int i = 0; i < min(issued, STAGES); ++i) {
+          if (--stage < 0) { stage = STAGES - 1; phase ^= 1u; }
+          while (!mbar_try_wait(&full[stage], phase) && globaltimer_ns() - t0 < 10000000ull) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
+        TileInfo ti;
+        gemm_decode(a, sched, t, ti);
+        const int buf = it & 1;
+        const uint32_t aphase = (it >> 1) & 1;
+        if (!mbar_wait(&tempty[buf], aphase ^ 1u, a.err)) { s_abort = 1; break; }
+        tc_fence_after();
+        const uint32_t d = tmem_base + buf * BN;
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
+          if (!mbar_wait(&full[stage], phase, a.err) || s_abort) { ok = false; s_abort = 1; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * Cfg::A_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * Cfg::B_BYTES);
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            umma_bf16(d, smem_desc_sw128(a_addr + k * 32), smem_desc_sw128(b_addr + k * 32), Cfg::IDESC,
+                      (kb > ti.kb0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        umma_commit(&tfull[buf]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;             // TMEM lane quarter this warp may access
+    const int row = q * 32 + lane;
+    int it = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+      TileInfo ti;
+      gemm_decode(a, sched, t, ti);
+      const int buf = it & 1;
+      const uint32_t aphase = (it >> 1) & 1;
+      int ready = 0;
+      if (lane == 0) ready = mbar_wait(&tfull[buf], aphase, a.err) && !s_abort;
+      ready = __shfl_sync(0xffffffffu, ready, 0);   // keep the warp converged for tcgen05.ld
+      if (!ready) { s_abort = 1; break; }
+      tc_fence_after();
+      const int m = ti.m0 + row;
+      const bool row_ok = m < ti.m_end;
+      const int n0 = ti.n_idx * BN;
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
+      if (a.splits == 1) {
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(taddr + c * 32, r);
+          tmem_ld_wait();
+          const int n = n0 + c * 32;
+          if (row_ok && n < a.N) {
+            float v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+            gemm_epilogue32(a, ti.g, m, n, v);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&tempty[buf]);
+      } else {
+        // write this split's partial, then the last split reduces in split order
+        float* wsp = a.ws + ((long long)ti.split * a.M + m) * a.N;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(taddr + c * 32, r);
+          tmem_ld_wait();
+          const int n = n0 + c * 32;
+          if (row_ok && n < a.N) {
+            float4* w4 = reinterpret_cast<float4*>(wsp + n);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              w4[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                  __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&tempty[buf]);
+        __threadfence();
+        named_bar_sync(1, 128);
+        if (threadIdx.x == 64) {
+          const int old = atomicAdd(&a.counters[ti.unit], 1);
+          s_last = (old == a.splits - 1);
+          if (s_last) a.counters[ti.unit] = 0;
+        }
+        named_bar_sync(1, 128);
+        if (s_last) {
+          __threadfence();
+          if (row_ok) {
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+              const int n = n0 + c * 32;
+              if (n >= a.N) break;
+              float v[32];
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+              for (int s = 0; s < a.splits; ++s) {
+                const float4* p4 = reinterpret_cast<const float4*>(a.ws + ((long long)s * a.M + m) * a.N + n);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                  const float4 x = __ldcg(p4 + j);
+                  v[4 * j] += x.x;
+                  v[4 * j + 1] += x.y;
+                  v[4 * j + 2] += x.z;
+                  v[4 * j + 3] += x.w;
+                }
+              }
+              gemm_epilogue32(a, ti.g, m, n, v);
+            }
+          }
+        }
+        named_bar_sync(1, 128);   // s_last is reused by the next tile
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+}  // namespace gdit

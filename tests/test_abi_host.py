@@ -1,0 +1,134 @@
+"""The C-ABI library builds, loads and exports every entry point that
+include/gdit.h declares; host-side argument validation works without a GPU."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import synth
+from flow_matching_dit_b200 import _lib
+from flow_matching_dit_b200.build import HEADER, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build()
+    return _lib.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdit_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("gdit_create", "gdit_get_action", "gdit_destroy", "gdit_sync_status", "gdit_strerror"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    assert set(declared_functions()) == set(_lib.exported_names())
+
+
+def test_strings(L):
+    assert L.gdit_version().startswith(b"gdit")
+    assert L.gdit_strerror(_lib.GDIT_EINVAL) == b"invalid argument"
+    assert L.gdit_strerror(-1234) == b"unknown error"
+
+
+def _cfg(g, **over):
+    c = _lib.gdit_config()
+    for f in ("num_layers", "hidden", "num_heads", "head_dim", "mlp_hidden", "backbone_dim", "action_dim",
+              "state_dim", "action_horizon", "num_embodiments", "time_freq_dim", "num_timestep_buckets"):
+        setattr(c, f, getattr(g, f))
+    c.ln_eps = g.ln_eps
+    c.max_batch = 4
+    c.max_backbone_seq = 64
+    for k, v in over.items():
+        setattr(c, k, v)
+    return c
+
+
+def _tensors(W):
+    keep = []
+    arr = (_lib.gdit_tensor * len(W))()
+    for i, (n, a) in enumerate(W.items()):
+        a = np.ascontiguousarray(a)
+        shp = (ctypes.c_int64 * a.ndim)(*a.shape)
+        nm = n.encode()
+        keep += [a, shp, nm]
+        arr[i].name, arr[i].ndim, arr[i].shape, arr[i].host_ptr = nm, a.ndim, shp, a.ctypes.data
+        arr[i].dtype = _lib.GDIT_BF16 if a.dtype == np.uint16 else _lib.GDIT_F32
+    return arr, keep
+
+
+@pytest.fixture(scope="module")
+def tinyW():
+    return synth.make_weights(synth.GEOM_TINY)
+
+
+def _create(L, cfg, W):
+    arr, keep = _tensors(W)
+    h = ctypes.c_void_p()
+    rc = L.gdit_create(ctypes.byref(cfg), arr, len(W), ctypes.byref(h))
+    return rc, h, L.gdit_last_error(None).decode()
+
+
+@pytest.mark.parametrize("field,value,msg", [
+    ("num_layers", 3, "num_layers"),
+    ("head_dim", 48, "head_dim"),
+    ("hidden", 96, "hidden"),
+    ("action_dim", 30, "action_dim"),
+    ("action_horizon", 64, "action_horizon"),
+    ("num_embodiments", 65, "num_embodiments"),
+    ("max_batch", 0, "max_batch"),
+])
+def test_bad_config_rejected_on_host(L, tinyW, field, value, msg):
+    cfg = _cfg(synth.GEOM_TINY, **{field: value})
+    rc, h, err = _create(L, cfg, tinyW)
+    assert rc == _lib.GDIT_EINVAL and not h.value
+    assert msg in err
+
+
+def test_missing_weight_is_named(L, tinyW):
+    W = dict(tinyW)
+    del W["blk1.ff2.b"]
+    rc, h, err = _create(L, _cfg(synth.GEOM_TINY), W)
+    assert rc == _lib.GDIT_EINVAL and "blk1.ff2.b" in err
+
+
+def test_misshaped_weight_is_named(L, tinyW):
+    W = dict(tinyW)
+    W["act_enc.W2.W"] = np.zeros((2, 128, 128), np.float32)
+    rc, h, err = _create(L, _cfg(synth.GEOM_TINY), W)
+    assert rc == _lib.GDIT_EINVAL and "act_enc.W2.W" in err
+
+
+def test_unknown_weight_rejected(L, tinyW):
+    W = dict(tinyW)
+    W["blk9.extra"] = np.zeros(3, np.float32)
+    rc, h, err = _create(L, _cfg(synth.GEOM_TINY), W)
+    assert rc == _lib.GDIT_EINVAL and "unknown" in err
+
+
+def test_valid_table_without_gpu_reports_no_device(L, tinyW):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    rc, h, err = _create(L, _cfg(synth.GEOM_TINY), tinyW)
+    assert rc in (_lib.GDIT_ENODEV, _lib.GDIT_ECUDA) and not h.value
+
+
+def test_null_handle_calls_are_rejected(L):
+    assert L.gdit_get_action(None, None, 0, None, None, None, None, 4, None, 1, 1, None) == _lib.GDIT_EINVAL
+    assert L.gdit_sync_status(None) == _lib.GDIT_EINVAL
+    L.gdit_destroy(None)

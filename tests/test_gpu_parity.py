@@ -1,0 +1,253 @@
+"""End-to-end parity of gdit_get_action (CUDA, through the C ABI) with the fp64
+CPU oracle on the same seeded inputs, for every workload, plus edge cases.
+
+Samples are independent, so at full batch sizes the oracle is run on a few
+sampled batch rows (covering different embodiments) and compared row by row.
+"""
+
+import dataclasses
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests.gpu_util import DELTA_REL_L2, MAX_ABS, REL_L2, parity_stats, require_gpu, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def full_weights():
+    return synth.make_weights(synth.GEOM_FULL)
+
+
+@pytest.fixture(scope="module")
+def full_model(full_weights):
+    return oracle.Model(full_weights, synth.GEOM_FULL)
+
+
+@pytest.fixture(scope="module")
+def head_full(full_weights):
+    require_gpu()
+    from flow_matching_dit_b200 import ActionHead
+    h = ActionHead(synth.GEOM_FULL, full_weights, max_batch=256, max_seq=600)
+    yield h
+    h.close()
+
+
+@pytest.fixture(scope="module")
+def tiny_weights():
+    return synth.make_weights(synth.GEOM_TINY)
+
+
+@pytest.fixture(scope="module")
+def head_tiny(tiny_weights):
+    require_gpu()
+    from flow_matching_dit_b200 import ActionHead
+    h = ActionHead(synth.GEOM_TINY, tiny_weights, max_batch=8, max_seq=64)
+    yield h
+    h.close()
+
+
+def run_gpu(head, inp, K):
+    out = head.get_action(*to_dev(inp), num_steps=K)
+    st = head.sync_status()
+    return out.cpu().numpy(), st
+
+
+def run_oracle(W, g, inp, K, samples=None, model=None):
+    return oracle.get_action(W, g, inp["backbone_features"], inp["vl_mask"], inp["state"], inp["embodiment_id"],
+                             inp["init_noise"], K, samples=samples, model=model)
+
+
+def assert_parity(gpu, ref, noise, what):
+    max_abs, rel, drel = parity_stats(gpu, ref, noise)
+    print(f"{what}: max_abs={max_abs:.3e} rel_l2={rel:.3e} delta_rel_l2={drel:.3e}")
+    assert np.isfinite(gpu).all(), what
+    assert max_abs <= MAX_ABS, (what, max_abs)
+    assert rel <= REL_L2, (what, rel)
+    assert drel <= DELTA_REL_L2, (what, drel)
+
+
+# ---------------------------------------------------------------- tiny workload
+
+@pytest.mark.parametrize("emb", [0, 1])
+def test_tiny_parity(head_tiny, tiny_weights, emb):
+    w = synth.workload("tiny", fixed_ids=(emb,))
+    inp = synth.make_inputs(w)
+    gpu, st = run_gpu(head_tiny, inp, 4)
+    assert st == 0
+    ref = run_oracle(tiny_weights, w.geom, inp, 4)
+    assert_parity(gpu, ref, inp["init_noise"], f"tiny id={emb}")
+
+
+def test_tiny_mixed_batch_ragged_masks(head_tiny, tiny_weights):
+    w = synth.workload("tiny", batch=5, valid_min=1, fixed_ids=None, id_low=0, id_high=1)
+    inp = synth.make_inputs(w, seed=5)
+    inp["vl_mask"][2] = 0                          # a sample with no valid token
+    inp["vl_mask"][3] = 0
+    inp["vl_mask"][3, 17] = 1                      # exactly one valid token
+    inp["vl_mask"][4, ::2] = 0                     # not a prefix
+    gpu, st = run_gpu(head_tiny, inp, 4)
+    assert st == 0
+    ref = run_oracle(tiny_weights, w.geom, inp, 4)
+    assert_parity(gpu, ref, inp["init_noise"], "tiny mixed")
+
+
+@pytest.mark.parametrize("K", [1, 3, 8])
+def test_tiny_step_counts(head_tiny, tiny_weights, K):
+    w = synth.workload("tiny", batch=2, fixed_ids=(1, 0))
+    inp = synth.make_inputs(w, seed=9)
+    gpu, st = run_gpu(head_tiny, inp, K)
+    ref = run_oracle(tiny_weights, w.geom, inp, K)
+    assert_parity(gpu, ref, inp["init_noise"], f"tiny K={K}")
+
+
+def test_tiny_masked_tokens_do_not_matter(head_tiny):
+    w = synth.workload("tiny", batch=2, fixed_ids=(0, 1))
+    inp = synth.make_inputs(w, seed=3)
+    inp["vl_mask"][:, 40:] = 0
+    a, _ = run_gpu(head_tiny, inp, 4)
+    inp2 = dict(inp, backbone_features=inp["backbone_features"].copy())
+    inp2["backbone_features"][:, 40:] = 1e3
+    b, _ = run_gpu(head_tiny, inp2, 4)
+    np.testing.assert_array_equal(a, b)
+
+
+def test_bad_embodiment_id_gives_nan_and_status(head_tiny, tiny_weights):
+    from flow_matching_dit_b200._lib import GDIT_EDEVICE
+    w = synth.workload("tiny", batch=3, fixed_ids=(0, 7, 1))
+    inp = synth.make_inputs(w, seed=4)
+    gpu, st = run_gpu(head_tiny, inp, 4)
+    assert st == GDIT_EDEVICE
+    assert np.isnan(gpu[1]).all()
+    ok = dict(inp)
+    for k in ok:
+        ok[k] = ok[k][[0, 2]]
+    ref = run_oracle(tiny_weights, w.geom, ok, 4)
+    assert_parity(gpu[[0, 2]], ref, ok["init_noise"], "tiny valid rows next to a bad id")
+    assert head_tiny.sync_status() == 0   # cleared
+
+
+def test_decoder_signature_routes_exactly():
+    """act_dec weights zero and b2[c] = c: every sample moves by exactly its
+    category index, so the output names the category that was used."""
+    require_gpu()
+    from flow_matching_dit_b200 import ActionHead
+    g = dataclasses.replace(synth.GEOM_TINY, num_embodiments=6)
+    W = synth.make_weights(g)
+    W["act_dec.l1.W"][:] = 0
+    W["act_dec.l1.b"][:] = 0
+    W["act_dec.l2.W"][:] = 0
+    for c in range(6):
+        W["act_dec.l2.b"][c] = c
+    ids = np.array([5, 0, 3, 3, 1, 4, 2, 0], np.int32)
+    w = synth.workload("tiny", geom=g, batch=8, fixed_ids=tuple(ids))
+    inp = synth.make_inputs(w, seed=11)
+    with ActionHead(g, W, max_batch=8, max_seq=64) as head:
+        gpu, st = run_gpu(head, inp, 4)
+        perm, seg, vofs = head.routing(8)
+    assert st == 0
+    moved = gpu - inp["init_noise"]
+    np.testing.assert_allclose(moved, np.broadcast_to(ids[:, None, None].astype(np.float64), moved.shape),
+                               rtol=0, atol=1e-5)
+    # routing arrays: stable counting sort by id
+    assert perm.tolist() == np.argsort(ids, kind="stable").tolist()
+    assert seg.tolist() == [int((ids < c).sum()) for c in range(7)]
+    assert vofs.tolist() == [64 * i for i in range(9)]
+
+
+def test_host_buffer_entry_point_matches_device_entry_point(head_tiny):
+    w = synth.workload("tiny", batch=3, fixed_ids=(1, 0, 1))
+    inp = synth.make_inputs(w, seed=21)
+    dev, _ = run_gpu(head_tiny, inp, 4)
+    host = head_tiny.get_action_host(inp["backbone_features"], inp["vl_mask"], inp["state"],
+                                     inp["embodiment_id"], inp["init_noise"], 4)
+    np.testing.assert_array_equal(dev, host)
+
+
+def test_eager_and_graph_paths_agree(tiny_weights):
+    require_gpu()
+    from flow_matching_dit_b200 import GDIT_FLAG_NO_GRAPH, ActionHead
+    w = synth.workload("tiny", batch=2, fixed_ids=(0, 1))
+    inp = synth.make_inputs(w, seed=2)
+    with ActionHead(synth.GEOM_TINY, tiny_weights, max_batch=2, max_seq=64, flags=GDIT_FLAG_NO_GRAPH) as eager:
+        a, _ = run_gpu(eager, inp, 4)
+    with ActionHead(synth.GEOM_TINY, tiny_weights, max_batch=2, max_seq=64) as graph:
+        b, _ = run_gpu(graph, inp, 4)
+        c, _ = run_gpu(graph, inp, 4)     # graph replay
+    np.testing.assert_array_equal(a, b)
+    np.testing.assert_array_equal(b, c)
+
+
+def test_strict_profiles(tiny_weights):
+    require_gpu()
+    from flow_matching_dit_b200 import GDIT_FLAG_STRICT_PROFILES, ActionHead, GditError
+    from flow_matching_dit_b200._lib import GDIT_EPROFILE
+    w = synth.workload("tiny", batch=2, fixed_ids=(0, 1))
+    inp = synth.make_inputs(w, seed=2)
+    with ActionHead(synth.GEOM_TINY, tiny_weights, max_batch=2, max_seq=64, flags=GDIT_FLAG_STRICT_PROFILES) as h:
+        with pytest.raises(GditError) as e:
+            run_gpu(h, inp, 4)
+        assert e.value.code == GDIT_EPROFILE
+        h.prepare(2, 64, 4, bf16=False)
+        run_gpu(h, inp, 4)
+
+
+# ---------------------------------------------------------------- full-size workloads
+
+def test_latency_workload_full_oracle(head_full, full_weights, full_model):
+    w = synth.WORKLOADS["latency"]
+    inp = synth.make_inputs(w)
+    gpu, st = run_gpu(head_full, inp, w.num_steps)
+    assert st == 0
+    ref = run_oracle(full_weights, w.geom, inp, w.num_steps, model=full_model)
+    assert_parity(gpu, ref, inp["init_noise"], "latency B=1 S=300")
+
+
+def test_cross_kv_projection_matches_oracle(head_full, full_model):
+    w = synth.WORKLOADS["latency"]
+    inp = synth.make_inputs(w)
+    run_gpu(head_full, inp, w.num_steps)
+    valid = oracle.to_f64(inp["backbone_features"][0])[inp["vl_mask"][0] == 1]
+    for layer in (0, 30):
+        k, v = head_full.debug_kv(layer)
+        kr, vr = oracle.cross_kv(full_model, layer, valid)
+        for got, ref in ((k, kr), (v, vr)):
+            # bf16 storage of f32-accumulated exact products: <= 2^-8 relative
+            np.testing.assert_allclose(got, ref, rtol=2 ** -8, atol=1e-3)
+
+
+def test_batched_workload_sampled(head_full, full_weights, full_model):
+    w = synth.WORKLOADS["batched"]
+    inp = synth.make_inputs(w)
+    gpu, st = run_gpu(head_full, inp, w.num_steps)
+    assert st == 0
+    rows = [0, 13, 27, 31]
+    ref = run_oracle(full_weights, w.geom, inp, w.num_steps, samples=rows, model=full_model)
+    assert_parity(gpu[rows], ref, inp["init_noise"][rows], "batched B=32 S<=600 (rows 0,13,27,31)")
+
+
+def test_sweep256_workload_sampled(head_full, full_weights, full_model):
+    w = synth.WORKLOADS["sweep256"]
+    inp = synth.make_inputs(w)
+    gpu, st = run_gpu(head_full, inp, w.num_steps)
+    assert st == 0
+    assert np.isfinite(gpu).all()
+    rows = [0, 100, 255]
+    ref = run_oracle(full_weights, w.geom, inp, w.num_steps, samples=rows, model=full_model)
+    assert_parity(gpu[rows], ref, inp["init_noise"][rows], "sweep B=256 (rows 0,100,255)")
+
+
+def test_long_chunk_workload_sampled(full_weights):
+    require_gpu()
+    from flow_matching_dit_b200 import ActionHead
+    w = synth.WORKLOADS["long_chunk"]
+    inp = synth.make_inputs(w)
+    with ActionHead(w.geom, full_weights, max_batch=8, max_seq=512) as head:
+        gpu, st = run_gpu(head, inp, w.num_steps)
+    assert st == 0
+    rows = [5]
+    ref = run_oracle(full_weights, w.geom, inp, w.num_steps, samples=rows)
+    assert_parity(gpu[rows], ref, inp["init_noise"][rows], "long chunk B=8 H=50 K=8 (row 5)")
