@@ -1,0 +1,352 @@
+#!/usr/bin/env python
+"""Benchmark of the flow-matching DiT action head (get_action) on B200.
+
+One step = one gdit_get_action call over a batch of synthetic inputs:
+B = 256 action chunks, backbone features [256, 256, 2048] bf16 (all valid),
+embodiment ids uniform over 32 categories, K = 4 Euler steps, 32-layer DiT
+(hidden 1024, 16 x 64 heads, MLP 4096), inputs resident in HBM.
+value = chunks/s of the whole job (all ranks).  Also reported: p50/p99
+latency of a B = 1 call (backbone [1, 300, 2048], K = 4), the dominant
+kernel's roofline, an end-to-end number through the host-buffer entry point,
+and the CPU oracle timed on a bounded sample.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+For N > 1 launch with torch.distributed.run; every rank runs its own replica
+on its own batch (the samples are independent: no collective on the data
+path), timing is taken as the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "DiT action chunks/s at B=256 and p50 get_action latency at B=1 (4 steps)"
+UNIT = "chunks/s"
+THROUGHPUT = "sweep256"
+LATENCY = "latency"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--latency-calls", type=int, default=200)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-profile", action="store_true")
+    p.add_argument("--oracle-samples", type=int, default=2)
+    p.add_argument("--batch", type=int, default=None, help="override the throughput batch (profiling runs)")
+    p.add_argument("--seq", type=int, default=None, help="override the throughput backbone length (profiling runs)")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), d.get("bf16_tflops_sustained", 1400.0), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.device = device
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.device)],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def time_oracle(W, w, samples: int):
+    """The fp64 oracle, as it stands, on `samples` batch rows of workload w
+    (one untimed row first: it converts the weights it touches)."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+    except Exception:
+        threadpool_info = None
+    inp = synth.make_inputs(w)
+    model = oracle.Model(W, w.geom)
+    args = (W, w.geom, inp["backbone_features"], inp["vl_mask"], inp["state"], inp["embodiment_id"],
+            inp["init_noise"], w.num_steps)
+    oracle.get_action(*args, samples=[0], model=model)
+    rows = list(range(1, 1 + samples))
+    t0 = time.perf_counter()
+    oracle.get_action(*args, samples=rows, model=model)
+    dt = time.perf_counter() - t0
+    cores = os.cpu_count() or 1
+    if threadpool_info is not None:
+        n = [p.get("num_threads", 0) for p in threadpool_info() if p.get("user_api") == "blas"]
+        if n:
+            cores = max(n)
+    return samples / dt, cores, dt
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    w = synth.WORKLOADS[THROUGHPUT]
+    W = synth.make_weights(w.geom)
+    samples = 1
+    times = []
+    import oracle
+    inp = synth.make_inputs(w)
+    model = oracle.Model(W, w.geom)
+    a = (W, w.geom, inp["backbone_features"], inp["vl_mask"], inp["state"], inp["embodiment_id"],
+         inp["init_noise"], w.num_steps)
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        oracle.get_action(*a, samples=[i % w.batch], model=model)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    per = float(np.mean(times))
+    value = samples / per
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([p.get("num_threads", 0) for p in threadpool_info() if p.get("user_api") == "blas"] or [os.cpu_count()])
+    except Exception:
+        cores = os.cpu_count()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "DiT action head B=256 S=256 K=4 (throughput sweep); each step one sampled chunk",
+                   "batch": w.batch, "seq": w.seq, "num_steps": w.num_steps},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"1 chunk of the B=256 workload per step ({args.steps} steps)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank)
+
+    import torch
+    import torch.distributed as dist
+    from flow_matching_dit_b200 import ActionHead
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev)
+
+    w = synth.WORKLOADS[THROUGHPUT]
+    if args.batch or args.seq:
+        w = synth.workload(THROUGHPUT, batch=args.batch or w.batch, seq=args.seq or w.seq)
+    wl = synth.WORKLOADS[LATENCY]
+    g = w.geom
+    W = synth.make_weights(g)
+    max_seq = max(w.seq, wl.seq) if args.latency_calls > 0 else w.seq
+    head = ActionHead(g, W, max_batch=w.batch, max_seq=max_seq, device=local)
+
+    def dev_inputs(wk, seed):
+        inp = synth.make_inputs(wk, seed=seed)
+        f = torch.from_numpy(inp["backbone_features"].view(np.int16)).to(dev).view(torch.bfloat16)
+        return inp, (f, torch.from_numpy(inp["vl_mask"]).to(dev), torch.from_numpy(inp["state"]).to(dev),
+                     torch.from_numpy(inp["embodiment_id"]).to(dev), torch.from_numpy(inp["init_noise"]).to(dev))
+
+    inp, d = dev_inputs(w, 1 + rank)
+    out = torch.empty_like(d[4])
+    stream = torch.cuda.current_stream(dev)
+    K = w.num_steps
+    for _ in range(max(args.warmup, 1)):
+        head.get_action(*d, num_steps=K, out=out)
+    assert head.sync_status() == 0
+
+    # ---- timed region: K steps, device-resident inputs
+    clocks = Clocks(local)
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        head.get_action(*d, num_steps=K, out=out)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    assert head.sync_status() == 0
+    ms_per_step = ms / args.steps
+    value = world * w.batch * args.steps / (ms / 1e3)
+
+    # ---- B = 1 latency (device inputs, one call at a time)
+    lat = None
+    if rank == 0 and args.latency_calls > 0:
+        _, dl = dev_inputs(wl, 7)
+        outl = torch.empty_like(dl[4])
+        for _ in range(20):
+            head.get_action(*dl, num_steps=wl.num_steps, out=outl)
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(args.latency_calls):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            head.get_action(*dl, num_steps=wl.num_steps, out=outl)
+            b.record(stream)
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        ts = np.array(ts)
+        lat = {"p50_ms": float(np.percentile(ts, 50)), "p99_ms": float(np.percentile(ts, 99)),
+               "mean_ms": float(ts.mean()), "calls": int(len(ts)),
+               "workload": "B=1, backbone [1,300,2048] bf16 all valid, id 0, K=4"}
+
+    # ---- end to end through the host-buffer entry point (pinned host memory)
+    e2e = None
+    if not args.no_e2e:
+        pin = {k: torch.from_numpy(np.ascontiguousarray(v)).pin_memory() for k, v in inp.items()}
+        hf = pin["backbone_features"].numpy()
+        hout = torch.empty(d[4].shape, dtype=torch.float32).pin_memory().numpy()
+        hargs = (hf, pin["vl_mask"].numpy(), pin["state"].numpy(), pin["embodiment_id"].numpy(),
+                 pin["init_noise"].numpy())
+        st = stream.cuda_stream
+        for _ in range(2):
+            head.get_action_host(*hargs, num_steps=K, out=hout, stream=st)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        n_e2e = max(3, args.steps // 2)
+        for _ in range(n_e2e):
+            head.get_action_host(*hargs, num_steps=K, out=hout, stream=st)
+        sec = time.perf_counter() - t0
+        if world > 1:
+            t = torch.tensor([sec], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            sec = float(t.item())
+        h2d = sum(int(v.nbytes) for v in hargs)
+        e2e = {"value": world * w.batch * n_e2e / sec, "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": int(hout.nbytes), "steps": n_e2e,
+               "api": "gdit_get_action_host (pinned host buffers, copies and sync inside)"}
+
+    # ---- per-kernel-class timing of one instrumented (eager) call
+    roof = None
+    launches_per_call = None
+    kstats = None
+    if rank == 0 and not args.no_profile:
+        kstats = head.profile(*d, num_steps=K, out=out)
+        launches_per_call = sum(k["launches"] for k in kstats) + 1    # + the pointer-setting kernel
+        top = max(kstats, key=lambda k: k["total_ms"])
+        hbm, tf_burst, tf_sus, src = load_peaks()
+        traffic = None
+        tpath = os.path.join(ROOT, "profiles", "traffic.json")
+        if os.path.exists(tpath):
+            traffic = json.load(open(tpath)).get(top["name"])
+        if top["name"].startswith("gemm"):
+            ach = top["flops"] / (top["total_ms"] / 1e3) / 1e12
+            roof = {"bound": "tensor", "kernel": top["name"], "achieved": ach, "peak": tf_sus, "unit": "TFLOP/s",
+                    "frac": ach / tf_sus, "frac_of_burst": ach / tf_burst, "peak_kind": f"sustained bf16 ({src})",
+                    "traffic": traffic, "launches": top["launches"], "ms": top["total_ms"]}
+        else:
+            ach = top["bytes"] / (top["total_ms"] / 1e3) / 1e9
+            roof = {"bound": "hbm", "kernel": top["name"], "achieved": ach, "peak": hbm, "unit": "GB/s",
+                    "frac": ach / hbm, "peak_kind": f"HBM copy ({src})", "traffic": traffic,
+                    "launches": top["launches"], "ms": top["total_ms"]}
+
+    # ---- CPU oracle on a bounded sample
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, secs = time_oracle(W, w, args.oracle_samples)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{args.oracle_samples} chunks of the B=256 workload (rows 1..{args.oracle_samples}), "
+                         f"fp64 numpy, {secs:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"DiT action head B={w.batch} S={w.seq} K={K} (throughput sweep)", "batch": w.batch,
+                       "seq": w.seq, "num_steps": K, "layers": g.num_layers, "hidden": g.hidden,
+                       "embodiments": g.num_embodiments, "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (1.36 GB bf16 weights, 4.3 GB KV cache per call)"},
+            "latency_b1": lat, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": (launches_per_call * args.steps) if launches_per_call else None,
+            "clocks": clk,
+        }
+        if kstats is not None:
+            line["kernel_classes"] = [{k: (round(v, 4) if isinstance(v, float) else v) for k, v in s.items()}
+                                      for s in kstats]
+        print(json.dumps(line), flush=True)
+    head.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
