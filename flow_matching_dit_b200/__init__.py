@@ -178,3 +178,17 @@ def test_gemm(A, B, bias, bn: int = 128, splits: int = 1, stream=None):
     check(_lib.gdit_test_gemm(_ptr(A), _ptr(B), _ptr(bias) if bias is not None else None, _ptr(C),
                               M, N, K, bn, splits, st), None)
     return C
+
+
+def gemm_static_scratch(A, B, bias, C=None, bn: int = 64, splits: int = 1, stream=None):
+    """Same as test_gemm, through the entry point that allocates no device
+    memory (its scratch is a fixed array inside the library).  C may be given."""
+    import torch
+    M, K = A.shape
+    N = B.shape[0]
+    if C is None:
+        C = torch.empty((M, N), dtype=torch.float32, device=A.device)
+    st = stream if stream is not None else torch.cuda.current_stream().cuda_stream
+    check(_lib.gdit_gemm_static_scratch(_ptr(A), _ptr(B), _ptr(bias) if bias is not None else None, _ptr(C),
+                                        M, N, K, bn, splits, st), None)
+    return C

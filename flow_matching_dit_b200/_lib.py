@@ -62,6 +62,7 @@ _SIGS = {
     "gdit_profile_get_action": (_I, [_P, _P, _I, _P, _P, _P, _P, _I, _P, _I, _I, _P,
                                      ctypes.POINTER(gdit_kernel_stat), _I]),
     "gdit_test_gemm": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "gdit_gemm_static_scratch": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
 }
 
 _lock = threading.Lock()
@@ -153,3 +154,7 @@ def gdit_profile_get_action(*a):
 
 def gdit_test_gemm(*a):
     return lib().gdit_test_gemm(*a)
+
+
+def gdit_gemm_static_scratch(*a):
+    return lib().gdit_gemm_static_scratch(*a)

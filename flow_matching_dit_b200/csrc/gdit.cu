@@ -18,6 +18,7 @@
 #include <cstdio>
 #include <cstring>
 #include <map>
+#include <mutex>
 #include <memory>
 #include <stdexcept>
 #include <string>
@@ -1361,3 +1362,94 @@ int gdit_test_gemm(const void* A, const void* B, const float* bias, float* C, in
 }
 
 }  // extern "C"
+
+// ====================================================================== no-allocation GEMM
+//
+// A variant of the split-K GEMM for callers that must not allocate device
+// memory at call time.  A robot's control loop is the typical case: cudaMalloc
+// and cudaFree can synchronise the whole device and take unbounded time, and
+// deployments with a fixed memory budget route every buffer through their own
+// pool.  Such callers pass inputs and outputs; the split-K partial sums, the
+// per-tile arrival counters and the status word live in the fixed array below,
+// which every GPU that loads this library holds until the process exits.
+namespace {
+
+constexpr long long kStaticPartialFloats = 1ll << 20;   // 4 MiB of split-K partials
+constexpr int kStaticCounters = 4096;                   // output tiles per call
+
+struct StaticScratch {
+  unsigned status;
+  unsigned pad[63];
+  int counters[kStaticCounters];
+  float partials[kStaticPartialFloats];
+};
+
+static __device__ __align__(256) StaticScratch g_static_scratch;
+
+// Device address of g_static_scratch, looked up once per device.
+std::mutex g_static_mu;
+StaticScratch* g_static_ptr[64] = {};
+
+StaticScratch* static_scratch_for_current_device() {
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  REQUIRE(dev >= 0 && dev < 64, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (g_static_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    CUDA_TRY(cudaGetSymbolAddress(&p, g_static_scratch));
+    g_static_ptr[dev] = static_cast<StaticScratch*>(p);
+  }
+  return g_static_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" int gdit_gemm_static_scratch(const void* A, const void* B, const float* bias, float* C, int M, int N,
+                                        int K, int bn, int splits, void* cuda_stream) {
+  g_create_error.clear();
+  return guarded(nullptr, [&] {
+    REQUIRE(A && B && C, "NULL matrix");
+    REQUIRE(M >= 1 && N >= 32 && N % 32 == 0 && K >= 8 && K % 8 == 0, "need M >= 1, N %% 32 == 0, K %% 8 == 0");
+    REQUIRE(bn == 32 || bn == 64 || bn == 128 || bn == 256, "bn must be 32, 64, 128 or 256");
+    const int nkb = (K + kBK - 1) / kBK;
+    REQUIRE(splits >= 1 && splits <= nkb, "splits must be in [1, %d]", nkb);
+    const long long nt = (N + bn - 1) / bn, mt = (M + kBM - 1) / kBM;
+    REQUIRE(mt * nt <= kStaticCounters, "%lld output tiles exceed the fixed scratch's %d tile counters", mt * nt,
+            kStaticCounters);
+    REQUIRE(splits == 1 || (long long)splits * M * N <= kStaticPartialFloats,
+            "split-K partials need %lld floats; the fixed scratch holds %lld (reduce splits, M or N)",
+            (long long)splits * M * N, kStaticPartialFloats);
+    set_kernel_attrs();
+    StaticScratch* sc = static_scratch_for_current_device();
+    cudaStream_t s = (cudaStream_t)cuda_stream;
+    int dev = 0, sms = 0;
+    CUDA_TRY(cudaGetDevice(&dev));
+    CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    // the status word and the tile counters must start at zero
+    CUDA_TRY(cudaMemsetAsync(&sc->status, 0, sizeof(unsigned), s));
+    CUDA_TRY(cudaMemsetAsync(sc->counters, 0, sizeof(int) * (size_t)(mt * nt), s));
+    GemmOp op;
+    op.args = default_args();
+    op.args.M = M;
+    op.args.N = N;
+    op.args.K = K;
+    op.args.splits = splits;
+    op.args.ws = sc->partials;
+    op.args.counters = sc->counters;
+    op.args.epi = EPI_F32;
+    op.args.bias = bias;
+    op.args.out = C;
+    op.args.ldo = N;
+    op.args.err = &sc->status;
+    op.bn = bn;
+    op.ta = make_tmap(A, M, K, K, kBM);
+    op.tb = make_tmap(B, N, K, K, bn);
+    op.grid = (int)std::min<long long>(mt * nt * splits, sms);
+    launch_gemm(op, op.args, s, false);
+    unsigned e = 0;
+    CUDA_TRY(cudaMemcpyAsync(&e, &sc->status, sizeof(unsigned), cudaMemcpyDeviceToHost, s));
+    CUDA_TRY(cudaStreamSynchronize(s));
+    if (e) throw GditError(GDIT_ETIMEOUT, "GEMM wait timed out");
+  });
+}

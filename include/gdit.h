@@ -220,6 +220,28 @@ int gdit_profile_get_action(gdit_handle* h, const void* backbone_features, int b
 int gdit_test_gemm(const void* A, const void* B, const float* bias, float* C,
                    int M, int N, int K, int bn, int splits, void* cuda_stream);
 
+/* Split-K GEMM that allocates nothing (no counterpart in the source pages: it
+ * serves callers, not the method).  Same operation, layouts and limits as
+ * gdit_test_gemm: C[M,N] (f32) = A[M,K] B[N,K]^T + bias[N], A and B bf16 device
+ * matrices (row-major, K contiguous), bias f32 device or NULL, C f32 device;
+ * all owned by the caller.
+ * For callers that cannot call cudaMalloc at call time, for example a robot's
+ * control loop, where cudaMalloc/cudaFree may synchronise the device and take
+ * unbounded time, or a deployment whose memory budget is fixed up front.  The
+ * split-K partials, per-tile counters and status word live in one fixed
+ * device array inside the library (4 MiB of partials, 4096 output tiles),
+ * which every GPU that loads the library keeps until the process exits.
+ * Limits (else GDIT_EINVAL): ceil(M/128) * ceil(N/bn) <= 4096 and, when
+ * splits > 1, splits * M * N <= 1048576.
+ * The first call on each device looks up the array's device address; make
+ * that first call before any stream capture on that device.  Every call
+ * shares the array and leaves its contents behind: calls that overlap on the
+ * GPU (several streams, several host threads) race and give wrong results.
+ * The call clears the status word and the counters itself, then synchronizes
+ * cuda_stream.  Returns GDIT_OK, GDIT_EINVAL or GDIT_ETIMEOUT. */
+int gdit_gemm_static_scratch(const void* A, const void* B, const float* bias, float* C,
+                             int M, int N, int K, int bn, int splits, void* cuda_stream);
+
 #ifdef __cplusplus
 }
 #endif
