@@ -3,14 +3,19 @@
 //   cross layers (even): the N = H + 1 state/action tokens of a sample attend to
 //     that sample's valid backbone tokens, whose K/V were projected once per call;
 //   self layers (odd): the N tokens attend to each other (no mask).
-// out_h = softmax(q_h k_h^T / sqrt(head_dim)) v_h per head, heads concatenated; a
-// sample with no key gets a zero output.
+// out_h = softmax(q_h k_h^T / sqrt(head_dim)) v_h per head, heads concatenated;
+// a sample with no key gets a zero output.
 //
-// One CTA per (sample, head); its 4 warps split the keys in chunks of 16
-// (flash-decoding inside the CTA) and keep an online softmax, then combine
-// through shared memory.  Scores and P*V use bf16 mma.sync m16n8k16 with f32
-// accumulation: the op is bound by the K/V reads (about 17 FLOP per byte at
-// N = 17), which this path keeps up with; queries are padded to 16-row tiles.
+// A warp streams 16-key chunks of K and V through a 3-deep cp.async ring in
+// shared memory and keeps an online (base-2) softmax.  Scores and P*V use bf16
+// mma.sync m16n8k16 with f32 accumulation: the op is bound by the K/V reads
+// (about 17 FLOP per byte at N = 17), which this path keeps up with; queries
+// are padded to 16-row tiles.  Two schedules share that routine:
+//   attention_split_kernel: one CTA per (sample, head), the 4 warps split the
+//     keys (flash-decoding inside the CTA) and combine through shared memory;
+//     for few samples with long key lists.
+//   attention_warp_kernel: every warp owns one (sample, head) and all its keys;
+//     for many samples, and for self-attention (N keys).
 #pragma once
 
 #include "ptx.cuh"
@@ -24,10 +29,12 @@ struct AttnArgs {
   long long q_ld;
   const __nv_bfloat16* k;
   const __nv_bfloat16* v;
-  long long kv_ld;
+  long long kv_ld;          // row stride of K and V
+  long long kv_head_stride; // offset between heads of K (and of V)
   const int* kofs;      // cross: keys of sample b are rows [kofs[b], kofs[b+1]); nullptr: self (rows of q's sample)
   int n_tok;            // queries (tokens) per sample
   int num_heads;
+  int num_items;        // samples * heads
   __nv_bfloat16* out;
   long long out_ld;
   float scale_log2;     // log2(e) / sqrt(head_dim)
@@ -38,13 +45,16 @@ struct AttnArgs {
 template <int MT, int DH>
 struct AttnSmem {
   static constexpr int ROW = DH + 8;
-  static constexpr int Q_BYTES = MT * 16 * ROW * 2;
-  static constexpr int CHUNK_BYTES = 16 * ROW * 2;                // 16 keys x DH dims (padded)
+  static constexpr int Q_ELEMS = MT * 16 * ROW;
+  static constexpr int CHUNK_ELEMS = 16 * ROW;                    // 16 keys x DH dims (padded)
   static constexpr int RING = 3;                                  // chunks in flight per warp
-  static constexpr int KV_BYTES = 4 * RING * 2 * CHUNK_BYTES;     // 4 warps x ring x (K, V)
-  static constexpr int O_BYTES = 4 * MT * 16 * DH * 4;
-  static constexpr int ML_BYTES = 4 * MT * 16 * 2 * 4;
-  static constexpr int TOTAL = Q_BYTES + KV_BYTES + O_BYTES + ML_BYTES;
+  static constexpr int RING_ELEMS = RING * 2 * CHUNK_ELEMS;       // (K, V) per slot
+  // split schedule: one Q tile, 4 rings, per-warp partials
+  static constexpr int SPLIT_O_BYTES = 4 * MT * 16 * DH * 4;
+  static constexpr int SPLIT_ML_BYTES = 4 * MT * 16 * 2 * 4;
+  static constexpr int SPLIT_TOTAL = (Q_ELEMS + 4 * RING_ELEMS) * 2 + SPLIT_O_BYTES + SPLIT_ML_BYTES;
+  // warp schedule: a Q tile and a ring per warp
+  static constexpr int WARP_TOTAL = 4 * (Q_ELEMS + RING_ELEMS) * 2;
 };
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid) {
@@ -71,49 +81,33 @@ __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t& r0, uint32_t& r1, ui
                : "r"(smem_u32(p)));
 }
 
-template <int MT, int DH>
-__global__ void __launch_bounds__(kAttnThreads) attention_kernel(const AttnArgs a) {
-  using SM = AttnSmem<MT, DH>;
-  constexpr int kRowPad = SM::ROW;
-  constexpr int kHeadDim = DH;
-  extern __shared__ __align__(16) uint8_t smem[];
-  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem);
-  __nv_bfloat16* sKV = reinterpret_cast<__nv_bfloat16*>(smem + SM::Q_BYTES);
-  float* sO = reinterpret_cast<float*>(smem + SM::Q_BYTES + SM::KV_BYTES);
-  float* sML = reinterpret_cast<float*>(smem + SM::Q_BYTES + SM::KV_BYTES + SM::O_BYTES);
-
-  const int b = blockIdx.x / a.num_heads;
-  const int h = blockIdx.x - b * a.num_heads;
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int g = lane >> 2;     // row group of the mma fragments
-  const int tig = lane & 3;    // thread in group
-
-  pdl_wait();
-
-  int k_begin, k_end;
+__device__ __forceinline__ void attn_key_range(const AttnArgs& a, int b, int& k_begin, int& n_keys) {
   if (a.kofs != nullptr) {
     k_begin = a.kofs[b];
-    k_end = a.kofs[b + 1];
+    n_keys = a.kofs[b + 1] - k_begin;
   } else {
     k_begin = b * a.n_tok;
-    k_end = k_begin + a.n_tok;
+    n_keys = a.n_tok;
   }
-  const int n_keys = k_end - k_begin;
+}
 
-  // ---- queries -> shared memory (rows >= n_tok are zero)
-  const __nv_bfloat16* qbase = a.q + (long long)b * a.n_tok * a.q_ld + h * kHeadDim;
+// Q rows of (b, h) -> shared tile [MT*16][DH+8]; rows >= n_tok are zero.
+// Thread t of `nthreads` cooperating threads copies every nthreads-th piece.
+template <int MT, int DH>
+__device__ __forceinline__ void attn_load_q(const AttnArgs& a, int b, int h, __nv_bfloat16* sQ, int t, int nthreads) {
+  constexpr int ROW = DH + 8;
   constexpr int PIECES = DH / 8;   // 16-byte pieces per row
-  for (int i = threadIdx.x; i < MT * 16 * PIECES; i += kAttnThreads) {
+  const __nv_bfloat16* qbase = a.q + (long long)b * a.n_tok * a.q_ld + h * DH;
+  for (int i = t; i < MT * 16 * PIECES; i += nthreads) {
     const int r = i / PIECES, c = (i % PIECES) * 8;
     uint4 val = make_uint4(0, 0, 0, 0);
     if (r < a.n_tok) val = *reinterpret_cast<const uint4*>(qbase + (long long)r * a.q_ld + c);
-    *reinterpret_cast<uint4*>(sQ + r * kRowPad + c) = val;
+    *reinterpret_cast<uint4*>(sQ + r * ROW + c) = val;
   }
-  __syncthreads();
+}
 
-  float o[MT][DH / 8][4];
-  float mrow[MT][2], lrow[MT][2];
+template <int MT, int DH>
+__device__ __forceinline__ void attn_init(float (&o)[MT][DH / 8][4], float (&mrow)[MT][2], float (&lrow)[MT][2]) {
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) {
 #pragma unroll
@@ -123,16 +117,29 @@ __global__ void __launch_bounds__(kAttnThreads) attention_kernel(const AttnArgs 
     mrow[mt][0] = mrow[mt][1] = -INFINITY;
     lrow[mt][0] = lrow[mt][1] = 0.0f;
   }
+}
 
+// One warp: chunks c0, c0 + cstep, ... of the keys [k_begin, k_begin + n_keys)
+// of head h, folded into (o, mrow, lrow) with an online softmax.
+template <int MT, int DH>
+__device__ __forceinline__ void attn_stream_chunks(const AttnArgs& a, int h, int k_begin, int n_keys, int c0,
+                                                   int cstep, const __nv_bfloat16* sQ, __nv_bfloat16* ring,
+                                                   float (&o)[MT][DH / 8][4], float (&mrow)[MT][2],
+                                                   float (&lrow)[MT][2]) {
+  using SM = AttnSmem<MT, DH>;
+  constexpr int ROW = SM::ROW;
+  constexpr int PIECES = DH / 8;
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2;     // row group of the mma fragments
+  const int tig = lane & 3;    // thread in group
   const int n_chunks = (n_keys + 15) >> 4;
-  __nv_bfloat16* ring = sKV + warp * SM::RING * 2 * (16 * kRowPad);
-  const __nv_bfloat16* kbase = a.k + h * kHeadDim;
-  const __nv_bfloat16* vbase = a.v + h * kHeadDim;
+  const __nv_bfloat16* kbase = a.k + h * a.kv_head_stride;
+  const __nv_bfloat16* vbase = a.v + h * a.kv_head_stride;
 
   // each lane copies DH/16 x 16 bytes of K and of V per chunk
   auto issue = [&](int chunk, int slot) {
-    __nv_bfloat16* dk = ring + slot * 2 * (16 * kRowPad);
-    __nv_bfloat16* dv = dk + 16 * kRowPad;
+    __nv_bfloat16* dk = ring + slot * 2 * SM::CHUNK_ELEMS;
+    __nv_bfloat16* dv = dk + SM::CHUNK_ELEMS;
 #pragma unroll
     for (int i = 0; i < DH / 16; ++i) {
       const int idx = lane + 32 * i;      // 16 rows x PIECES pieces
@@ -140,31 +147,30 @@ __global__ void __launch_bounds__(kAttnThreads) attention_kernel(const AttnArgs 
       const int key = chunk * 16 + r;
       const bool valid = key < n_keys;
       const long long row = (long long)(k_begin + (valid ? key : 0));
-      cp_async16(dk + r * kRowPad + c, kbase + row * a.kv_ld + c, valid);
-      cp_async16(dv + r * kRowPad + c, vbase + row * a.kv_ld + c, valid);
+      cp_async16(dk + r * ROW + c, kbase + row * a.kv_ld + c, valid);
+      cp_async16(dv + r * ROW + c, vbase + row * a.kv_ld + c, valid);
     }
   };
 
-  // chunks of this warp: warp, warp + 4, ...
   int my_n = 0;
-  for (int c = warp; c < n_chunks; c += 4) ++my_n;
+  for (int c = c0; c < n_chunks; c += cstep) ++my_n;
 #pragma unroll
   for (int p = 0; p < SM::RING - 1; ++p) {
-    if (p < my_n) issue(warp + 4 * p, p);
+    if (p < my_n) issue(c0 + cstep * p, p);
     cp_async_commit();
   }
 
   for (int it = 0; it < my_n; ++it) {
-    const int chunk = warp + 4 * it;
+    const int chunk = c0 + cstep * it;
     {
       const int nxt = it + SM::RING - 1;
-      if (nxt < my_n) issue(warp + 4 * nxt, nxt % SM::RING);
+      if (nxt < my_n) issue(c0 + cstep * nxt, nxt % SM::RING);
       cp_async_commit();
     }
     cp_async_wait<SM::RING - 1>();
     __syncwarp();
-    const __nv_bfloat16* sk = ring + (it % SM::RING) * 2 * (16 * kRowPad);
-    const __nv_bfloat16* sv = sk + 16 * kRowPad;
+    const __nv_bfloat16* sk = ring + (it % SM::RING) * 2 * SM::CHUNK_ELEMS;
+    const __nv_bfloat16* sv = sk + SM::CHUNK_ELEMS;
 
     // S = Q K^T for 16 keys (two n-tiles of 8)
     float s[MT][2][4];
@@ -179,17 +185,17 @@ __global__ void __launch_bounds__(kAttnThreads) attention_kernel(const AttnArgs 
       uint32_t kb[2][2];
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
-        const __nv_bfloat16* kr = sk + (nt * 8 + g) * kRowPad + ks * 16 + tig * 2;
+        const __nv_bfloat16* kr = sk + (nt * 8 + g) * ROW + ks * 16 + tig * 2;
         kb[nt][0] = *reinterpret_cast<const uint32_t*>(kr);
         kb[nt][1] = *reinterpret_cast<const uint32_t*>(kr + 8);
       }
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
-        const __nv_bfloat16* qr = sQ + (mt * 16 + g) * kRowPad + ks * 16 + tig * 2;
+        const __nv_bfloat16* qr = sQ + (mt * 16 + g) * ROW + ks * 16 + tig * 2;
         const uint32_t a0 = *reinterpret_cast<const uint32_t*>(qr);
-        const uint32_t a1 = *reinterpret_cast<const uint32_t*>(qr + 8 * kRowPad);
+        const uint32_t a1 = *reinterpret_cast<const uint32_t*>(qr + 8 * ROW);
         const uint32_t a2 = *reinterpret_cast<const uint32_t*>(qr + 8);
-        const uint32_t a3 = *reinterpret_cast<const uint32_t*>(qr + 8 * kRowPad + 8);
+        const uint32_t a3 = *reinterpret_cast<const uint32_t*>(qr + 8 * ROW + 8);
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) mma_bf16_16816(s[mt][nt], a0, a1, a2, a3, kb[nt][0], kb[nt][1]);
       }
@@ -242,7 +248,7 @@ __global__ void __launch_bounds__(kAttnThreads) attention_kernel(const AttnArgs 
       uint32_t vb0, vb1, vb2, vb3;
       const int r = lane & 7;
       const int mtx = lane >> 3;          // matrix 0..3: (keys 0-7 | 8-15) x (dims nd | nd+1)
-      const __nv_bfloat16* vp = sv + ((mtx & 1) * 8 + r) * kRowPad + (nd2 * 2 + (mtx >> 1)) * 8;
+      const __nv_bfloat16* vp = sv + ((mtx & 1) * 8 + r) * ROW + (nd2 * 2 + (mtx >> 1)) * 8;
       ldmatrix_x4_trans(vb0, vb1, vb2, vb3, vp);
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
@@ -257,8 +263,38 @@ __global__ void __launch_bounds__(kAttnThreads) attention_kernel(const AttnArgs 
     __syncwarp();   // the slot is refilled by a later issue
   }
   cp_async_wait<0>();
+}
 
-  // ---- per-warp partial results -> shared memory
+// ---------------------------------------------------------------- split schedule
+template <int MT, int DH>
+__global__ void __launch_bounds__(kAttnThreads) attention_split_kernel(const AttnArgs a) {
+  using SM = AttnSmem<MT, DH>;
+  extern __shared__ __align__(16) uint8_t smem[];
+  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem);
+  __nv_bfloat16* sKV = sQ + SM::Q_ELEMS;
+  float* sO = reinterpret_cast<float*>(smem + (SM::Q_ELEMS + 4 * SM::RING_ELEMS) * 2);
+  float* sML = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(sO) + SM::SPLIT_O_BYTES);
+
+  const int b = blockIdx.x / a.num_heads;
+  const int h = blockIdx.x - b * a.num_heads;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2;
+  const int tig = lane & 3;
+
+  pdl_wait();
+  pdl_launch_dependents();
+  int k_begin, n_keys;
+  attn_key_range(a, b, k_begin, n_keys);
+  attn_load_q<MT, DH>(a, b, h, sQ, threadIdx.x, kAttnThreads);
+  __syncthreads();
+
+  float o[MT][DH / 8][4];
+  float mrow[MT][2], lrow[MT][2];
+  attn_init<MT, DH>(o, mrow, lrow);
+  attn_stream_chunks<MT, DH>(a, h, k_begin, n_keys, warp, 4, sQ, sKV + warp * SM::RING_ELEMS, o, mrow, lrow);
+
+  // per-warp partial results -> shared memory
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) {
 #pragma unroll
@@ -271,7 +307,7 @@ __global__ void __launch_bounds__(kAttnThreads) attention_kernel(const AttnArgs 
         sML[(warp * MT * 16 + row) * 2 + 0] = mrow[mt][hr];
         sML[(warp * MT * 16 + row) * 2 + 1] = l;
       }
-      float* orow = sO + (warp * MT * 16 + row) * kHeadDim;
+      float* orow = sO + (warp * MT * 16 + row) * DH;
 #pragma unroll
       for (int nd = 0; nd < DH / 8; ++nd) {
         orow[nd * 8 + tig * 2 + 0] = o[mt][nd][hr * 2 + 0];
@@ -281,11 +317,11 @@ __global__ void __launch_bounds__(kAttnThreads) attention_kernel(const AttnArgs 
   }
   __syncthreads();
 
-  // ---- combine the 4 warps and write bf16 rows
-  __nv_bfloat16* obase = a.out + (long long)b * a.n_tok * a.out_ld + h * kHeadDim;
-  for (int i = threadIdx.x; i < a.n_tok * (kHeadDim / 2); i += kAttnThreads) {
-    const int row = i / (kHeadDim / 2);
-    const int d = (i - row * (kHeadDim / 2)) * 2;
+  // combine the 4 warps and write bf16 rows
+  __nv_bfloat16* obase = a.out + (long long)b * a.n_tok * a.out_ld + h * DH;
+  for (int i = threadIdx.x; i < a.n_tok * (DH / 2); i += kAttnThreads) {
+    const int row = i / (DH / 2);
+    const int d = (i - row * (DH / 2)) * 2;
     float mt = -INFINITY;
 #pragma unroll
     for (int w = 0; w < 4; ++w) mt = fmaxf(mt, sML[(w * MT * 16 + row) * 2]);
@@ -297,14 +333,61 @@ __global__ void __launch_bounds__(kAttnThreads) attention_kernel(const AttnArgs 
         const float mw = sML[(w * MT * 16 + row) * 2];
         const float f = (mw == -INFINITY) ? 0.0f : exp2f(mw - mt);
         l += f * sML[(w * MT * 16 + row) * 2 + 1];
-        r0 += f * sO[(w * MT * 16 + row) * kHeadDim + d];
-        r1 += f * sO[(w * MT * 16 + row) * kHeadDim + d + 1];
+        r0 += f * sO[(w * MT * 16 + row) * DH + d];
+        r1 += f * sO[(w * MT * 16 + row) * DH + d + 1];
       }
       const float inv = 1.0f / l;
       r0 *= inv;
       r1 *= inv;
     }
     *reinterpret_cast<uint32_t*>(obase + (long long)row * a.out_ld + d) = pack_bf16x2(r0, r1);
+  }
+}
+
+// ---------------------------------------------------------------- warp schedule
+template <int MT, int DH>
+__global__ void __launch_bounds__(kAttnThreads) attention_warp_kernel(const AttnArgs a) {
+  using SM = AttnSmem<MT, DH>;
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2;
+  const int tig = lane & 3;
+  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem) + warp * (SM::Q_ELEMS + SM::RING_ELEMS);
+  __nv_bfloat16* ring = sQ + SM::Q_ELEMS;
+
+  pdl_wait();
+  pdl_launch_dependents();
+  const int item = blockIdx.x * 4 + warp;
+  if (item >= a.num_items) return;
+  const int b = item / a.num_heads;
+  const int h = item - b * a.num_heads;
+  int k_begin, n_keys;
+  attn_key_range(a, b, k_begin, n_keys);
+  attn_load_q<MT, DH>(a, b, h, sQ, lane, 32);
+  __syncwarp();
+
+  float o[MT][DH / 8][4];
+  float mrow[MT][2], lrow[MT][2];
+  attn_init<MT, DH>(o, mrow, lrow);
+  attn_stream_chunks<MT, DH>(a, h, k_begin, n_keys, 0, 1, sQ, ring, o, mrow, lrow);
+
+  __nv_bfloat16* obase = a.out + (long long)b * a.n_tok * a.out_ld + h * DH;
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      float l = lrow[mt][hr];
+      l += __shfl_xor_sync(0xffffffffu, l, 1);
+      l += __shfl_xor_sync(0xffffffffu, l, 2);
+      const int row = mt * 16 + g + hr * 8;
+      if (row >= a.n_tok) continue;
+      const float inv = l > 0.0f ? 1.0f / l : 0.0f;   // no key: zero output
+#pragma unroll
+      for (int nd = 0; nd < DH / 8; ++nd)
+        *reinterpret_cast<uint32_t*>(obase + (long long)row * a.out_ld + nd * 8 + tig * 2) =
+            pack_bf16x2(o[mt][nd][hr * 2 + 0] * inv, o[mt][nd][hr * 2 + 1] * inv);
+    }
   }
 }
 

@@ -601,21 +601,49 @@ void alloc_workspace(gdit_handle* h) {
   CUDA_TRY(cudaMemset(h->h, 0, sizeof(float) * (size_t)Bm * N * D));
 }
 
+template <typename K>
+void max_shared_carveout(K* kern) {
+  CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                (int)cudaSharedmemCarveoutMaxShared));
+}
+
+template <int MT, int DH>
+void set_attn_attrs() {
+  CUDA_TRY(cudaFuncSetAttribute(attention_split_kernel<MT, DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                AttnSmem<MT, DH>::SPLIT_TOTAL));
+  CUDA_TRY(cudaFuncSetAttribute(attention_warp_kernel<MT, DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                AttnSmem<MT, DH>::WARP_TOTAL));
+  max_shared_carveout(attention_split_kernel<MT, DH>);
+  max_shared_carveout(attention_warp_kernel<MT, DH>);
+}
+
 void set_kernel_attrs() {
   static bool done = false;
   if (done) return;
+  // One shared-memory carveout for every kernel, so consecutive launches never
+  // wait for an SM to repartition L1 / shared memory.
+  max_shared_carveout(route_kernel);
+  max_shared_carveout(pack_features_kernel);
+  max_shared_carveout(gather_inputs_kernel);
+  max_shared_carveout(scatter_out_kernel);
+  max_shared_carveout(set_io_kernel);
+  max_shared_carveout(layernorm_kernel<1>);
+  max_shared_carveout(layernorm_kernel<2>);
+  max_shared_carveout(layernorm_kernel<4>);
+  max_shared_carveout(layernorm_kernel<8>);
+  max_shared_carveout(layernorm_kernel<16>);
+  max_shared_carveout(gemm_tc_kernel<32>);
+  max_shared_carveout(gemm_tc_kernel<64>);
+  max_shared_carveout(gemm_tc_kernel<128>);
+  max_shared_carveout(gemm_tc_kernel<256>);
   set_gemm_attr<32>();
   set_gemm_attr<64>();
   set_gemm_attr<128>();
   set_gemm_attr<256>();
-  CUDA_TRY(cudaFuncSetAttribute(attention_kernel<2, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                AttnSmem<2, 64>::TOTAL));
-  CUDA_TRY(cudaFuncSetAttribute(attention_kernel<4, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                AttnSmem<4, 64>::TOTAL));
-  CUDA_TRY(cudaFuncSetAttribute(attention_kernel<2, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                AttnSmem<2, 32>::TOTAL));
-  CUDA_TRY(cudaFuncSetAttribute(attention_kernel<4, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                AttnSmem<4, 32>::TOTAL));
+  set_attn_attrs<2, 64>();
+  set_attn_attrs<4, 64>();
+  set_attn_attrs<2, 32>();
+  set_attn_attrs<4, 32>();
   done = true;
 }
 
@@ -709,8 +737,12 @@ std::unique_ptr<Profile> build_profile(gdit_handle* h, int B, int S, int K, int 
   p->kv.args.bias = m.bkv;
   p->kv.args.out = h->kv;
   p->kv.args.ldo = 2 * D;
+  // head-major cache: layer block [K | V][head][token][head_dim], so the
+  // attention of one (sample, head) streams contiguous rows
   p->kv.args.nblk = 2 * D;
   p->kv.args.blk_stride = h->max_tok * 2 * D;
+  p->kv.args.head_cols = h->cfg.head_dim;
+  p->kv.args.head_stride = h->max_tok * h->cfg.head_dim;
   p->kv.rows_kind = 1;
   p->kv.weight_bytes = (long long)h->Lc * 2 * D * Dvl * 2;
 
@@ -859,18 +891,30 @@ void enqueue_forward(gdit_handle* h, Profile& p, cudaStream_t s, Recorder* rec) 
       }
     });
   };
-  auto attn = [&](const char* name, const AttnArgs& aa) {
-    const dim3 grid(B * h->cfg.num_heads), block(kAttnThreads);
+  // Attention schedule: one warp per (sample, head) when there are enough of
+  // them to fill the GPU (and always for self-attention: N keys); otherwise
+  // one CTA per (sample, head) with the keys split across its warps.
+  auto attn = [&](const char* name, const AttnArgs& aa, bool warp_sched) {
+    const dim3 block(kAttnThreads);
+    const int MT = N <= 32 ? 2 : 4;
+    const int DH = h->cfg.head_dim;
     lx.timed(name, 0, 0, nullptr, [&] {
-      if (h->cfg.head_dim == 64) {
-        if (N <= 32) launch_k(s, pdl, attention_kernel<2, 64>, grid, block, AttnSmem<2, 64>::TOTAL, aa);
-        else launch_k(s, pdl, attention_kernel<4, 64>, grid, block, AttnSmem<4, 64>::TOTAL, aa);
+      if (warp_sched) {
+        const dim3 grid((aa.num_items + 3) / 4);
+        if (DH == 64 && MT == 2) launch_k(s, pdl, attention_warp_kernel<2, 64>, grid, block, AttnSmem<2, 64>::WARP_TOTAL, aa);
+        else if (DH == 64) launch_k(s, pdl, attention_warp_kernel<4, 64>, grid, block, AttnSmem<4, 64>::WARP_TOTAL, aa);
+        else if (MT == 2) launch_k(s, pdl, attention_warp_kernel<2, 32>, grid, block, AttnSmem<2, 32>::WARP_TOTAL, aa);
+        else launch_k(s, pdl, attention_warp_kernel<4, 32>, grid, block, AttnSmem<4, 32>::WARP_TOTAL, aa);
       } else {
-        if (N <= 32) launch_k(s, pdl, attention_kernel<2, 32>, grid, block, AttnSmem<2, 32>::TOTAL, aa);
-        else launch_k(s, pdl, attention_kernel<4, 32>, grid, block, AttnSmem<4, 32>::TOTAL, aa);
+        const dim3 grid(aa.num_items);
+        if (DH == 64 && MT == 2) launch_k(s, pdl, attention_split_kernel<2, 64>, grid, block, AttnSmem<2, 64>::SPLIT_TOTAL, aa);
+        else if (DH == 64) launch_k(s, pdl, attention_split_kernel<4, 64>, grid, block, AttnSmem<4, 64>::SPLIT_TOTAL, aa);
+        else if (MT == 2) launch_k(s, pdl, attention_split_kernel<2, 32>, grid, block, AttnSmem<2, 32>::SPLIT_TOTAL, aa);
+        else launch_k(s, pdl, attention_split_kernel<4, 32>, grid, block, AttnSmem<4, 32>::SPLIT_TOTAL, aa);
       }
     });
   };
+  const bool cross_warp_sched = B * h->cfg.num_heads >= 4 * h->num_sms;
 
   // routing, packing, gathers
   lx.timed("route_pack", 0, 0, nullptr, [&] {
@@ -905,6 +949,7 @@ void enqueue_forward(gdit_handle* h, Profile& p, cudaStream_t s, Recorder* rec) 
       aa.q = h->qkv;
       aa.n_tok = N;
       aa.num_heads = h->cfg.num_heads;
+      aa.num_items = B * h->cfg.num_heads;
       aa.out = h->o;
       aa.out_ld = D;
       aa.scale_log2 = scale_log2;
@@ -913,16 +958,18 @@ void enqueue_forward(gdit_handle* h, Profile& p, cudaStream_t s, Recorder* rec) 
         aa.k = h->qkv + D;
         aa.v = h->qkv + 2 * D;
         aa.kv_ld = 3 * D;
+        aa.kv_head_stride = h->cfg.head_dim;
         aa.kofs = nullptr;
-        attn("attn_self", aa);
+        attn("attn_self", aa, true);
       } else {
         const __nv_bfloat16* kvl = h->kv + (size_t)(l / 2) * h->max_tok * 2 * D;
         aa.q_ld = D;
         aa.k = kvl;
-        aa.v = kvl + D;
-        aa.kv_ld = 2 * D;
+        aa.v = kvl + (size_t)h->cfg.num_heads * h->max_tok * h->cfg.head_dim;
+        aa.kv_ld = h->cfg.head_dim;
+        aa.kv_head_stride = h->max_tok * h->cfg.head_dim;
         aa.kofs = h->vofs;
-        attn("attn_cross", aa);
+        attn("attn_cross", aa, cross_warp_sched);
       }
       lx.gemm("gemm_dit", p.o[l]);
       ln(h->w.ln3g[l], h->w.ln3b[l], 1, nullptr);
@@ -1214,15 +1261,16 @@ int gdit_debug_kv(gdit_handle* h, int layer, float* k_out, float* v_out, int* to
     CUDA_TRY(cudaMemcpy(&tot, h->vofs + h->last_B, sizeof(int), cudaMemcpyDeviceToHost));
     *total_valid = tot;
     if (k_out == nullptr && v_out == nullptr) return;
-    const int D = h->D;
-    std::vector<uint16_t> buf((size_t)tot * 2 * D);
-    if (tot > 0)
-      CUDA_TRY(cudaMemcpy(buf.data(), h->kv + (size_t)(layer / 2) * h->max_tok * 2 * D, buf.size() * 2,
-                          cudaMemcpyDeviceToHost));
+    const int D = h->D, dh = h->cfg.head_dim, nh = h->cfg.num_heads;
+    // layer block: [K | V][head][token (max_tok)][head_dim]
+    std::vector<uint16_t> buf((size_t)2 * nh * h->max_tok * dh);
+    CUDA_TRY(cudaMemcpy(buf.data(), h->kv + (size_t)(layer / 2) * h->max_tok * 2 * D, buf.size() * 2,
+                        cudaMemcpyDeviceToHost));
     for (int r = 0; r < tot; ++r)
       for (int c = 0; c < D; ++c) {
-        if (k_out) k_out[(size_t)r * D + c] = bf16_to_f32(buf[(size_t)r * 2 * D + c]);
-        if (v_out) v_out[(size_t)r * D + c] = bf16_to_f32(buf[(size_t)r * 2 * D + D + c]);
+        const int hd = c / dh, d = c % dh;
+        if (k_out) k_out[(size_t)r * D + c] = bf16_to_f32(buf[((size_t)hd * h->max_tok + r) * dh + d]);
+        if (v_out) v_out[(size_t)r * D + c] = bf16_to_f32(buf[((size_t)(nh + hd) * h->max_tok + r) * dh + d]);
       }
   });
 }

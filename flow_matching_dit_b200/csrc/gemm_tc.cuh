@@ -64,6 +64,9 @@ struct GemmArgs {
   int in_group, in_skip, out_group, out_off;   // output row = (m / in_group) * out_group + m % in_group - in_skip + out_off
   int nblk;                 // > 0: columns blocked by nblk, block j at out + j * blk_stride
   long long blk_stride;
+  int head_cols;            // > 0 (with nblk): inside a block, column c goes to sub-matrix c / head_cols,
+  long long head_stride;    //   stored [rows][head_cols] at block + (c / head_cols) * head_stride
+
   unsigned* err;
 };
 
@@ -126,6 +129,31 @@ __device__ __forceinline__ void gemm_decode(const GemmArgs& a, const GemmSched& 
   ti.kb1 = (int)(((long long)(ti.split + 1) * nkb) / a.splits);
 }
 
+template <int BN>
+__device__ __forceinline__ void gemm_build_sched(const GemmArgs& a, GemmSched& sched) {
+  sched.nt = (a.N + BN - 1) / BN;
+  if (a.num_groups == 0) {
+    int rows = a.M;
+    if (a.m_dev != nullptr) rows = min(rows, *a.m_dev);
+    rows = max(rows, 0);
+    sched.rows = rows;
+    sched.mt = (rows + kBM - 1) / kBM;
+    sched.units = sched.mt * sched.nt;
+  } else {
+    int u = 0;
+    for (int g = 0; g < a.num_groups; ++g) {
+      const int rs = a.seg[g] * a.rows_per_sample;
+      const int re = a.seg[g + 1] * a.rows_per_sample;
+      sched.rstart[g] = rs;
+      sched.rend[g] = re;
+      sched.uprefix[g] = u;
+      u += ((re - rs + kBM - 1) / kBM) * sched.nt;
+    }
+    sched.uprefix[a.num_groups] = u;
+    sched.units = u;
+  }
+}
+
 __device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
 __device__ __forceinline__ float swish_f(float x) { return x / (1.0f + __expf(-x)); }
 
@@ -137,10 +165,17 @@ __device__ __forceinline__ void gemm_epilogue32(const GemmArgs& a, int g, int m,
   const long long orow = (long long)gi * a.out_group + (ri - a.in_skip) + a.out_off;
   long long col = n;
   long long blk_off = 0;
+  long long ldo = a.ldo;
   if (a.nblk > 0) {
     const int blk = n / a.nblk;
     col = n - (long long)blk * a.nblk;
     blk_off = (long long)blk * a.blk_stride;
+    if (a.head_cols > 0) {   // head-major: 32 columns never straddle a sub-matrix (head_cols % 32 == 0)
+      const long long hh = col / a.head_cols;
+      blk_off += hh * a.head_stride;
+      col -= hh * a.head_cols;
+      ldo = a.head_cols;
+    }
   }
   const int epi = a.epi;
   if (epi == EPI_SWISH_VEC_BF16) {
@@ -172,7 +207,7 @@ __device__ __forceinline__ void gemm_epilogue32(const GemmArgs& a, int g, int m,
     for (int j = 0; j < 32; ++j) v[j] = fmaxf(v[j], 0.0f);
   }
   if (epi <= EPI_SWISH_VEC_BF16) {
-    __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) + blk_off + orow * a.ldo + col;
+    __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) + blk_off + orow * ldo + col;
     uint4* o4 = reinterpret_cast<uint4*>(o);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -185,7 +220,7 @@ __device__ __forceinline__ void gemm_epilogue32(const GemmArgs& a, int g, int m,
     }
     return;
   }
-  float* o = reinterpret_cast<float*>(a.out) + blk_off + orow * a.ldo + col;
+  float* o = reinterpret_cast<float*>(a.out) + blk_off + orow * ldo + col;
   float4* o4 = reinterpret_cast<float4*>(o);
   if (epi == EPI_F32) {
 #pragma unroll
@@ -272,31 +307,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tmem_relinquish();
     tc_fence_before();
   }
-  // Inputs (A, seg, m_dev, residuals) come from earlier kernels on the stream.
-  pdl_wait();
+  // The schedule of a dense GEMM with a fixed row count depends on nothing an
+  // earlier kernel writes, and neither do the weights (operand B): their first
+  // stages are requested before waiting for the previous kernel, so weight
+  // streaming overlaps its tail.  A, seg, m_dev and residuals are read after.
+  const bool early = a.num_groups == 0 && a.m_dev == nullptr;
+  int pre = 0;   // stages whose B tile was issued before the wait (first tile only)
   if (threadIdx.x == 0) {
-    sched.nt = (a.N + BN - 1) / BN;
-    if (a.num_groups == 0) {
-      int rows = a.M;
-      if (a.m_dev != nullptr) rows = min(rows, *a.m_dev);
-      rows = max(rows, 0);
-      sched.rows = rows;
-      sched.mt = (rows + kBM - 1) / kBM;
-      sched.units = sched.mt * sched.nt;
-    } else {
-      int u = 0;
-      for (int g = 0; g < a.num_groups; ++g) {
-        const int rs = a.seg[g] * a.rows_per_sample;
-        const int re = a.seg[g + 1] * a.rows_per_sample;
-        sched.rstart[g] = rs;
-        sched.rend[g] = re;
-        sched.uprefix[g] = u;
-        u += ((re - rs + kBM - 1) / kBM) * sched.nt;
+    if (early) gemm_build_sched<BN>(a, sched);
+    if (early && (int)blockIdx.x < sched.units * a.splits) {
+      TileInfo ti;
+      gemm_decode(a, sched, blockIdx.x, ti);
+      pre = min(ti.kb1 - ti.kb0, STAGES);
+      const int brow = ti.g * a.b_group_rows + ti.n_idx * BN;
+      for (int i = 0; i < pre; ++i) {
+        mbar_arrive_expect_tx(&full[i], Cfg::STAGE_BYTES);
+        tma_load_2d(sB + i * Cfg::B_BYTES, &tmB, &full[i], (ti.kb0 + i) * kBK, brow);
       }
-      sched.uprefix[a.num_groups] = u;
-      sched.units = u;
     }
   }
+  pdl_wait();
+  pdl_launch_dependents();
+  if (threadIdx.x == 0 && !early) gemm_build_sched<BN>(a, sched);
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = tmem_holder;
@@ -314,11 +346,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         gemm_decode(a, sched, t, ti);
         const int brow = ti.g * a.b_group_rows + ti.n_idx * BN;
         for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, a.err)) { ok = false; s_abort = 1; break; }
-          if (s_abort) { ok = false; break; }
-          mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
-          tma_load_2d(sA + stage * Cfg::A_BYTES, &tmA, &full[stage], kb * kBK, ti.m0);
-          tma_load_2d(sB + stage * Cfg::B_BYTES, &tmB, &full[stage], kb * kBK, brow);
+          if (pre > 0) {
+            // stage armed and its B tile requested before the dependency wait
+            tma_load_2d(sA + stage * Cfg::A_BYTES, &tmA, &full[stage], kb * kBK, ti.m0);
+            --pre;
+          } else {
+            if (!mbar_wait(&empty[stage], phase ^ 1u, a.err)) { ok = false; s_abort = 1; break; }
+            if (s_abort) { ok = false; break; }
+            mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
+            tma_load_2d(sA + stage * Cfg::A_BYTES, &tmA, &full[stage], kb * kBK, ti.m0);
+            tma_load_2d(sB + stage * Cfg::B_BYTES, &tmB, &full[stage], kb * kBK, brow);
+          }
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }

@@ -42,6 +42,7 @@ __global__ void __launch_bounds__(kRouteThreads)
   __shared__ int s_cat[kMaxBatch];
   __shared__ int s_pos[65];
   pdl_wait();
+  pdl_launch_dependents();
   const int32_t* ids = io->ids;
   const uint8_t* mask = io->mask;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -96,6 +97,7 @@ __global__ void __launch_bounds__(kPackThreads)
   __shared__ int s_n;
   __shared__ int s_before;
   pdl_wait();
+  pdl_launch_dependents();
   const int i = blockIdx.x;
   const int j0 = blockIdx.y * 32;
   const int b = perm[i];
@@ -147,6 +149,7 @@ __global__ void __launch_bounds__(kPackThreads)
 __global__ void gather_inputs_kernel(const IoPtrs* io, int B, int HA, int Sd, const int* perm, float* x,
                                      __nv_bfloat16* xb, __nv_bfloat16* sb) {
   pdl_wait();
+  pdl_launch_dependents();
   const int i = blockIdx.x;
   const int b = perm[i];
   for (int e = threadIdx.x; e < HA; e += blockDim.x) {
@@ -161,6 +164,7 @@ __global__ void gather_inputs_kernel(const IoPtrs* io, int B, int HA, int Sd, co
 // out_actions[perm[i]] = x[i]; NaN for a sample whose embodiment id was invalid.
 __global__ void scatter_out_kernel(const IoPtrs* io, int HA, const int* perm, const uint8_t* bad, const float* x) {
   pdl_wait();
+  pdl_launch_dependents();
   const int i = blockIdx.x;
   const int b = perm[i];
   const bool nan_out = bad[b] != 0;
@@ -184,6 +188,7 @@ __global__ void __launch_bounds__(256)
                      __nv_bfloat16* u, const float* restore, int period) {
   constexpr int D = 128 * VEC;
   pdl_wait();
+  pdl_launch_dependents();
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
