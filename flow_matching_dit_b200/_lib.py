@@ -25,6 +25,7 @@ GDIT_F32 = 0
 GDIT_BF16 = 1
 GDIT_FLAG_STRICT_PROFILES = 1
 GDIT_FLAG_NO_GRAPH = 2
+GDIT_FLAG_NO_SMALL = 4
 
 
 class gdit_config(ctypes.Structure):

@@ -101,7 +101,8 @@ __device__ __forceinline__ void attn_load_q(const AttnArgs& a, int b, int h, __n
   for (int i = t; i < MT * 16 * PIECES; i += nthreads) {
     const int r = i / PIECES, c = (i % PIECES) * 8;
     uint4 val = make_uint4(0, 0, 0, 0);
-    if (r < a.n_tok) val = *reinterpret_cast<const uint4*>(qbase + (long long)r * a.q_ld + c);
+    // L2 load: queries are rewritten every layer by other CTAs of a persistent loop
+    if (r < a.n_tok) val = __ldcg(reinterpret_cast<const uint4*>(qbase + (long long)r * a.q_ld + c));
     *reinterpret_cast<uint4*>(sQ + r * ROW + c) = val;
   }
 }

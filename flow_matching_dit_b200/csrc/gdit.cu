@@ -31,6 +31,7 @@
 #include "gemm_tc.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
+#include "small_loop.cuh"
 
 using namespace gdit;
 
@@ -191,6 +192,7 @@ GemmArgs default_args() {
 }
 
 constexpr long long kWsFloats = 16ll << 20;   // split-K partials (64 MB)
+constexpr int kSmallMaxPhases = 64 * (5 * kSmallMaxLayers + 6);
 constexpr int kCounters = 1 << 16;
 
 // Picks the tile width and split-K factor.  Large row counts use wide tiles;
@@ -250,6 +252,10 @@ struct Profile {
   GemmOp kv, st1, st2, a1, a2, a3, proj, d1, d2;
   std::vector<GemmOp> q, o, ff1, ff2;
   cudaGraphExec_t exec = nullptr;
+  // single-sample profiles run the K-step loop as one persistent kernel
+  bool small = false;
+  SmallPlan* small_plan = nullptr;   // device copy
+  int small_phases = 0;
 };
 
 struct KStat {
@@ -292,6 +298,8 @@ struct gdit_handle {
   __nv_bfloat16 *xp, *kv, *u, *qkv, *o, *f, *xb, *abf, *zbf, *ybf, *rbf, *sb, *s1;
   float *h, *x, *sfeat, *ws;
   int *perm, *seg, *vofs, *counters;
+  int* phase_counters;      // per-phase arrival counters of the single-sample loop
+  SmallPhase* phase_table;  // per-phase descriptors of the single-sample loop
   uint8_t* bad;
   unsigned* status;
   IoPtrs* io;
@@ -596,6 +604,8 @@ void alloc_workspace(gdit_handle* h) {
   h->io = h->dalloc<IoPtrs>(1);
   h->ws = h->dalloc<float>((size_t)kWsFloats);
   h->counters = h->dalloc<int>((size_t)kCounters);
+  h->phase_counters = h->dalloc<int>((size_t)kSmallMaxPhases);
+  h->phase_table = h->dalloc<SmallPhase>((size_t)kSmallMaxPhases);
   CUDA_TRY(cudaMemset(h->counters, 0, sizeof(int) * kCounters));
   CUDA_TRY(cudaMemset(h->status, 0, sizeof(unsigned)));
   CUDA_TRY(cudaMemset(h->h, 0, sizeof(float) * (size_t)Bm * N * D));
@@ -640,6 +650,13 @@ void set_kernel_attrs() {
   set_gemm_attr<64>();
   set_gemm_attr<128>();
   set_gemm_attr<256>();
+  CUDA_TRY(cudaFuncSetAttribute(small_loop_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                SmallSmem<64>::TOTAL));
+  CUDA_TRY(cudaFuncSetAttribute(small_loop_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                SmallSmem<32>::TOTAL));
+  max_shared_carveout(small_loop_kernel<64>);
+  max_shared_carveout(small_describe_kernel);
+  max_shared_carveout(small_loop_kernel<32>);
   set_attn_attrs<2, 64>();
   set_attn_attrs<4, 64>();
   set_attn_attrs<2, 32>();
@@ -837,6 +854,39 @@ std::unique_ptr<Profile> build_profile(gdit_handle* h, int B, int S, int K, int 
   p->d2.rows_kind = 2;
   for (GemmOp* g : {&p->st1, &p->st2, &p->a1, &p->a2, &p->a3, &p->d1, &p->d2})
     g->weight_bytes = (long long)g->args.N * g->args.K * 2;   // per category used
+
+  // one sample: the K-step loop as one persistent kernel
+  p->small = B == 1 && N <= kSmallMaxTok && D <= kSmallMaxD && L <= kSmallMaxLayers &&
+             h->cfg.num_heads <= h->num_sms && N * D * 4 <= kSmHStageBytes && (h->cfg.flags & GDIT_FLAG_NO_SMALL) == 0;
+  if (p->small) {
+    const Tables& t = h->tables.at(K);
+    SmallPlan sp;
+    std::memset(&sp, 0, sizeof(sp));
+    sp.D = D; sp.F = F; sp.A = A; sp.H = H; sp.N = N; sp.nh = h->cfg.num_heads; sp.dh = h->cfg.head_dim;
+    sp.L = L; sp.K = K; sp.C = C;
+    sp.eps = h->cfg.ln_eps;
+    sp.scale_log2 = 1.4426950408889634f / std::sqrt((float)h->cfg.head_dim);
+    sp.max_tok = h->max_tok;
+    sp.h = h->h; sp.x = h->x; sp.xb = h->xb;
+    sp.abf = h->abf; sp.zbf = h->zbf; sp.qkv = h->qkv; sp.o = h->o; sp.f = h->f; sp.ybf = h->ybf; sp.rbf = h->rbf;
+    sp.sfeat = h->sfeat; sp.seg = h->seg; sp.vofs = h->vofs;
+    sp.ada = t.ada; sp.tw2 = t.tw2;
+    sp.wa1t = m.wa1t; sp.wa2at = m.wa2at; sp.wa3t = m.wa3t; sp.wd1t = m.wd1t; sp.wd2t = m.wd2t; sp.proj_w = m.proj_w;
+    sp.ba1 = m.ba1; sp.ba3 = m.ba3; sp.bd1 = m.bd1; sp.bd2 = m.bd2; sp.proj_b = m.proj_b;
+    for (int l = 0; l < L; ++l) {
+      SmallLayer& y = sp.layers[l];
+      y.wq = m.wq[l]; y.bq = m.bq[l]; y.wo = m.wo[l]; y.bo = m.bo[l]; y.ln3g = m.ln3g[l]; y.ln3b = m.ln3b[l];
+      y.wff1 = m.wff1[l]; y.bff1 = m.bff1[l]; y.wff2 = m.wff2[l]; y.bff2 = m.bff2[l];
+      y.kv = (l % 2 == 0) ? h->kv + (size_t)(l / 2) * h->max_tok * 2 * D : nullptr;
+    }
+    sp.counters = h->phase_counters;
+    sp.phases = h->phase_table;
+    sp.err = h->status;
+    p->small_phases = (5 * L + 6) * K;
+    if (p->small_phases > kSmallMaxPhases) throw GditError(GDIT_EINVAL, "too many phases for the single-sample loop");
+    p->small_plan = h->dalloc<SmallPlan>(1);
+    CUDA_TRY(cudaMemcpy(p->small_plan, &sp, sizeof(sp), cudaMemcpyHostToDevice));
+  }
   return p;
 }
 
@@ -932,6 +982,36 @@ void enqueue_forward(gdit_handle* h, Profile& p, cudaStream_t s, Recorder* rec) 
   lx.gemm("gemm_kv_proj", p.kv);
   lx.gemm("gemm_embodiment", p.st1);
   lx.gemm("gemm_embodiment", p.st2);
+
+  if (p.small) {
+    lx.timed("small_loop", 0, 0, nullptr, [&] {
+      launch_k(s, pdl, small_describe_kernel, dim3((p.small_phases + 127) / 128), dim3(128), 0,
+               (const SmallPlan*)p.small_plan);
+      CUDA_TRY(cudaMemsetAsync(h->phase_counters, 0, sizeof(int) * (size_t)p.small_phases, s));
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(h->num_sms);
+      cfg.blockDim = dim3(kSmallThreads);
+      cfg.stream = s;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeCooperative;   // all CTAs co-resident: they wait on one another
+      attr[0].val.cooperative = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      const SmallPlan* sp = p.small_plan;
+      if (h->cfg.head_dim == 64) {
+        cfg.dynamicSmemBytes = SmallSmem<64>::TOTAL;
+        CUDA_TRY(cudaLaunchKernelEx(&cfg, small_loop_kernel<64>, sp));
+      } else {
+        cfg.dynamicSmemBytes = SmallSmem<32>::TOTAL;
+        CUDA_TRY(cudaLaunchKernelEx(&cfg, small_loop_kernel<32>, sp));
+      }
+    });
+    lx.timed("route_pack", 0, 0, nullptr, [&] {
+      launch_k(s, pdl, scatter_out_kernel, dim3(B), dim3(128), 0, (const IoPtrs*)h->io, H * A, (const int*)h->perm,
+               (const uint8_t*)h->bad, (const float*)h->x);
+    });
+    return;
+  }
 
   const float scale_log2 = 1.4426950408889634f / std::sqrt((float)h->cfg.head_dim);
   for (int k = 0; k < K; ++k) {

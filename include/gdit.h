@@ -65,6 +65,8 @@ extern "C" {
 /* flags for gdit_config.flags */
 #define GDIT_FLAG_STRICT_PROFILES 1u  /* unprepared (batch, seq, steps) -> GDIT_EPROFILE, never a capture */
 #define GDIT_FLAG_NO_GRAPH 2u         /* run eagerly (no CUDA graph); same kernels, for debugging */
+#define GDIT_FLAG_NO_SMALL 4u         /* never use the single-sample persistent loop (batch 1 then runs the
+                                         same per-layer kernels as larger batches) */
 
 /* ------------------------------------------------------------------ config
  * Model geometry and capacity.  Every size is explicit.  Defaults of the

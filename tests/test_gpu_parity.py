@@ -251,3 +251,57 @@ def test_long_chunk_workload_sampled(full_weights):
     rows = [5]
     ref = run_oracle(full_weights, w.geom, inp, w.num_steps, samples=rows)
     assert_parity(gpu[rows], ref, inp["init_noise"][rows], "long chunk B=8 H=50 K=8 (row 5)")
+
+
+# ---------------------------------------------------------------- single-sample persistent loop
+
+def test_single_sample_loop_matches_general_path_and_oracle(full_weights, full_model, head_full):
+    """B = 1 runs the whole K-step loop as one persistent kernel; the general
+    per-layer path (GDIT_FLAG_NO_SMALL) and the oracle must agree with it."""
+    from flow_matching_dit_b200 import GDIT_FLAG_NO_SMALL, ActionHead
+    w = synth.WORKLOADS["latency"]
+    inp = synth.make_inputs(w, seed=13)
+    small, st = run_gpu(head_full, inp, w.num_steps)
+    assert st == 0
+    with ActionHead(w.geom, full_weights, max_batch=1, max_seq=w.seq, flags=GDIT_FLAG_NO_SMALL) as general:
+        gen, st2 = run_gpu(general, inp, w.num_steps)
+    assert st2 == 0
+    ref = run_oracle(full_weights, w.geom, inp, w.num_steps, model=full_model)
+    assert_parity(small, ref, inp["init_noise"], "single-sample loop vs oracle")
+    assert_parity(gen, ref, inp["init_noise"], "general path B=1 vs oracle")
+    assert_parity(small, gen, inp["init_noise"], "single-sample loop vs general path")
+
+
+def test_single_sample_loop_eager_equals_graph(tiny_weights):
+    require_gpu()
+    from flow_matching_dit_b200 import GDIT_FLAG_NO_GRAPH, ActionHead
+    w = synth.workload("tiny", fixed_ids=(1,))
+    inp = synth.make_inputs(w, seed=17)
+    with ActionHead(synth.GEOM_TINY, tiny_weights, max_batch=1, max_seq=64, flags=GDIT_FLAG_NO_GRAPH) as eager:
+        a, _ = run_gpu(eager, inp, 4)
+    with ActionHead(synth.GEOM_TINY, tiny_weights, max_batch=1, max_seq=64) as graph:
+        b, _ = run_gpu(graph, inp, 4)
+        c, _ = run_gpu(graph, inp, 4)
+    np.testing.assert_array_equal(a, b)
+    np.testing.assert_array_equal(b, c)
+
+
+@pytest.mark.parametrize("case", ["empty", "one_token", "bad_id"])
+def test_single_sample_loop_edge_cases(head_tiny, tiny_weights, case):
+    from flow_matching_dit_b200._lib import GDIT_EDEVICE
+    w = synth.workload("tiny", fixed_ids=(1,))
+    inp = synth.make_inputs(w, seed=19)
+    if case == "empty":
+        inp["vl_mask"][:] = 0
+    elif case == "one_token":
+        inp["vl_mask"][:] = 0
+        inp["vl_mask"][0, 33] = 1
+    else:
+        inp["embodiment_id"][:] = 5
+    gpu, st = run_gpu(head_tiny, inp, 4)
+    if case == "bad_id":
+        assert st == GDIT_EDEVICE and np.isnan(gpu).all()
+        return
+    assert st == 0
+    ref = run_oracle(tiny_weights, w.geom, inp, 4)
+    assert_parity(gpu, ref, inp["init_noise"], f"single-sample loop, {case}")
