@@ -154,7 +154,21 @@ __device__ __forceinline__ void gemm_build_sched(const GemmArgs& a, GemmSched& s
   }
 }
 
-__device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
+// erf by the rational approximation 7.1.26 of Abramowitz & Stegun, Handbook of
+// Mathematical Functions (1964): |error| < 1.5e-7, far below bf16 resolution.
+__device__ __forceinline__ float erf_as(float x) {
+  const float ax = fabsf(x);
+  const float t = __fdividef(1.0f, fmaf(0.3275911f, ax, 1.0f));
+  float y = fmaf(1.061405429f, t, -1.453152027f);
+  y = fmaf(y, t, 1.421413741f);
+  y = fmaf(y, t, -0.284496736f);
+  y = fmaf(y, t, 0.254829592f);
+  y *= t;
+  return copysignf(1.0f - y * __expf(-ax * ax), x);
+}
+
+// exact (erf) GELU: x * Phi(x)
+__device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.0f + erf_as(x * 0.70710678118654752f)); }
 __device__ __forceinline__ float swish_f(float x) { return x / (1.0f + __expf(-x)); }
 
 // Epilogue of 32 consecutive columns [n, n + 32) of row m (group g).
