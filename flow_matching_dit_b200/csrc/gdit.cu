@@ -123,6 +123,25 @@ CUtensorMap make_tmap(const void* ptr, long long rows, long long cols, long long
   return m;
 }
 
+// Output map for the TMA-store epilogue: [rows, cols] with row pitch `pitch`
+// elements, 32-row boxes of 128 bytes (bf16: 64 columns, f32: 32), 128-byte swizzle.
+CUtensorMap make_out_tmap(const void* ptr, bool f32, long long rows, long long cols, long long pitch) {
+  const int esz = f32 ? 4 : 2;
+  REQUIRE(((uintptr_t)ptr & 15u) == 0, "TMA base pointer not 16-byte aligned");
+  REQUIRE((pitch * esz) % 16 == 0, "output row pitch not a multiple of 16 bytes");
+  CUtensorMap m;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)std::max<long long>(rows, 1)};
+  cuuint64_t strides[1] = {(cuuint64_t)(pitch * esz)};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / esz), 32u};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = encode_fn()(&m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                           const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) throw GditError(GDIT_ECUDA, fmt("cuTensorMapEncodeTiled (output) failed (%d)", (int)r));
+  return m;
+}
+
 // ------------------------------------------------------------------ launch helper
 
 bool g_pdl_default = true;
@@ -146,7 +165,7 @@ void launch_k(cudaStream_t s, bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 
 // ------------------------------------------------------------------ GEMM ops
 
 struct GemmOp {
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, to;
   GemmArgs args;
   int bn = 64;
   int grid = 1;
@@ -156,6 +175,20 @@ struct GemmOp {
   int out_bytes = 2;
 };
 
+// Switch a planned dense GEMM to the TMA-store epilogue when its output is a
+// plain [M, N] matrix (no split-K, no row remap, no column blocking).
+void enable_tma_out(GemmOp& op) {
+  GemmArgs& a = op.args;
+  const bool plain_epi = a.epi == EPI_BF16 || a.epi == EPI_GELU_BF16 || a.epi == EPI_RELU_BF16 ||
+                         a.epi == EPI_F32 || a.epi == EPI_RESID_F32;
+  if (a.splits != 1 || a.num_groups != 0 || a.m_dev != nullptr || a.nblk != 0 || a.in_group != 0x7fffffff ||
+      a.out_off != 0 || !plain_epi || op.bn < 64)
+    return;
+  const bool f32 = a.epi == EPI_F32 || a.epi == EPI_RESID_F32;
+  op.to = make_out_tmap(a.out, f32, a.M, a.N, a.ldo);
+  a.tma_out = 1;
+}
+
 template <int BN>
 void set_gemm_attr() {
   CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmCfg<BN>::SMEM));
@@ -164,16 +197,16 @@ void set_gemm_attr() {
 void launch_gemm(const GemmOp& op, const GemmArgs& a, cudaStream_t s, bool pdl) {
   switch (op.bn) {
     case 32:
-      launch_k(s, pdl, gemm_tc_kernel<32>, dim3(op.grid), dim3(kGemmThreads), GemmCfg<32>::SMEM, op.ta, op.tb, a);
+      launch_k(s, pdl, gemm_tc_kernel<32>, dim3(op.grid), dim3(kGemmThreads), GemmCfg<32>::SMEM, op.ta, op.tb, op.to, a);
       break;
     case 64:
-      launch_k(s, pdl, gemm_tc_kernel<64>, dim3(op.grid), dim3(kGemmThreads), GemmCfg<64>::SMEM, op.ta, op.tb, a);
+      launch_k(s, pdl, gemm_tc_kernel<64>, dim3(op.grid), dim3(kGemmThreads), GemmCfg<64>::SMEM, op.ta, op.tb, op.to, a);
       break;
     case 128:
-      launch_k(s, pdl, gemm_tc_kernel<128>, dim3(op.grid), dim3(kGemmThreads), GemmCfg<128>::SMEM, op.ta, op.tb, a);
+      launch_k(s, pdl, gemm_tc_kernel<128>, dim3(op.grid), dim3(kGemmThreads), GemmCfg<128>::SMEM, op.ta, op.tb, op.to, a);
       break;
     case 256:
-      launch_k(s, pdl, gemm_tc_kernel<256>, dim3(op.grid), dim3(kGemmThreads), GemmCfg<256>::SMEM, op.ta, op.tb, a);
+      launch_k(s, pdl, gemm_tc_kernel<256>, dim3(op.grid), dim3(kGemmThreads), GemmCfg<256>::SMEM, op.ta, op.tb, op.to, a);
       break;
     default:
       throw GditError(GDIT_EINVAL, fmt("bad GEMM tile width %d", op.bn));
@@ -726,6 +759,7 @@ GemmOp plan_gemm(gdit_handle* h, const void* A, long long a_rows, int K, const v
   a.splits = splits;
   op.ta = make_tmap(A, a_rows, K, K, kBM);
   op.tb = make_tmap(Bw, b_rows, K, K, bn);
+  op.to = op.ta;   // placeholder unless the TMA-store epilogue is enabled
   const long long nt = (N + bn - 1) / bn;
   long long max_units = ((a_rows + kBM - 1) / kBM + (groups ? std::min<long long>(groups, a_rows) : 0)) * nt;
   if (splits > 1 && max_units > kCounters) throw GditError(GDIT_EINVAL, "too many split-K tiles");
@@ -826,6 +860,8 @@ std::unique_ptr<Profile> build_profile(gdit_handle* h, int B, int S, int K, int 
     p->ff2[l].args.out = h->h;
     p->ff2[l].args.ldo = D;
     p->ff2[l].weight_bytes = (long long)D * F * 2;
+    if ((h->cfg.flags & GDIT_FLAG_NO_TMA_STORE) == 0)
+      for (GemmOp* g : {&p->q[l], &p->o[l], &p->ff1[l], &p->ff2[l]}) enable_tma_out(*g);
   }
   // norm_out + proj_out on every token; only the H action rows are kept (compact)
   p->proj = plan_gemm(h, h->u, rows, D, m.proj_w, D, D, EPI_BF16, rows, 0, 0, 1);
@@ -1437,6 +1473,7 @@ int gdit_profile_get_action(gdit_handle* h, const void* backbone_features, int b
 
 int gdit_test_gemm(const void* A, const void* B, const float* bias, float* C, int M, int N, int K, int bn, int splits,
                    void* cuda_stream) {
+  const bool tma_out = getenv("GDIT_TEST_TMA_OUT") != nullptr;   // unit-test knob: exercise the TMA-store epilogue
   g_create_error.clear();
   return guarded(nullptr, [&] {
     REQUIRE(A && B && C, "NULL matrix");
@@ -1477,6 +1514,11 @@ int gdit_test_gemm(const void* A, const void* B, const float* bias, float* C, in
     op.bn = bn;
     op.ta = make_tmap(A, M, K, K, kBM);
     op.tb = make_tmap(B, N, K, K, bn);
+    op.to = op.ta;
+    if (tma_out && splits == 1) {
+      op.to = make_out_tmap(C, true, M, N, N);
+      op.args.tma_out = 1;
+    }
     op.grid = (int)std::min<long long>(mt * nt * splits, sms);
     launch_gemm(op, op.args, s, false);
     CUDA_TRY(cudaStreamSynchronize(s));
@@ -1573,6 +1615,7 @@ extern "C" int gdit_gemm_static_scratch(const void* A, const void* B, const floa
     op.bn = bn;
     op.ta = make_tmap(A, M, K, K, kBM);
     op.tb = make_tmap(B, N, K, K, bn);
+    op.to = op.ta;
     op.grid = (int)std::min<long long>(mt * nt * splits, sms);
     launch_gemm(op, op.args, s, false);
     unsigned e = 0;

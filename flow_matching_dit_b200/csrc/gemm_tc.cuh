@@ -18,7 +18,11 @@
 // 128 x BN (BN in {32, 64, 128, 256}) with 64-wide K blocks in the 128-byte
 // swizzled layout.  Split-K is deterministic: every split writes an f32
 // partial, and the last split to finish (per-tile counter) sums the partials
-// in split order and runs the epilogue.
+// in split order and runs the epilogue.  Dense GEMMs with a plain output
+// store through TMA: each epilogue warp stages 32 rows x 128 bytes in a
+// 128-byte-swizzled shared buffer (conflict-free 16-byte stores) and one lane
+// issues a bulk tensor store, or a bulk reduce-add (f32) for the residual
+// adds, so the residual is never read back.
 #pragma once
 
 #include "ptx.cuh"
@@ -67,6 +71,7 @@ struct GemmArgs {
   int head_cols;            // > 0 (with nblk): inside a block, column c goes to sub-matrix c / head_cols,
   long long head_stride;    //   stored [rows][head_cols] at block + (c / head_cols) * head_stride
 
+  int tma_out;              // 1: output through the TMA map (dense, one split, plain [M, N] layout)
   unsigned* err;
 };
 
@@ -77,7 +82,8 @@ struct GemmCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
   static constexpr int TMEM_COLS = 2 * BN;
-  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 256;
+  static constexpr int STG_BYTES = 4 * 2 * 4096;   // per epilogue warp: two 32 x 128-byte staging boxes
+  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + STG_BYTES + 256;
   static constexpr uint32_t IDESC = idesc_bf16_f32(kBM, BN);
 };
 
@@ -279,7 +285,7 @@ __device__ __forceinline__ void gemm_epilogue32(const GemmArgs& a, int g, int m,
 template <int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const GemmArgs a) {
+                   const __grid_constant__ CUtensorMap tmO, const GemmArgs a) {
   using Cfg = GemmCfg<BN>;
   constexpr int STAGES = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -292,7 +298,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * Cfg::A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);
+  uint8_t* stg = smem + STAGES * Cfg::STAGE_BYTES;   // 1024-aligned staging boxes
+  uint64_t* full = reinterpret_cast<uint64_t*>(stg + Cfg::STG_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -315,6 +322,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (a.tma_out) tma_prefetch_desc(&tmO);
   }
   if (warp == 1) {
     tmem_alloc(&tmem_holder, Cfg::TMEM_COLS);
@@ -427,6 +435,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ epilogue (warps 2..5)
     const int q = warp & 3;             // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;
+    int ebuf = 0;                       // staging box of the next TMA store
     int it = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
       TileInfo ti;
@@ -442,7 +451,85 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const bool row_ok = m < ti.m_end;
       const int n0 = ti.n_idx * BN;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
-      if (a.splits == 1) {
+      if (a.tma_out) {
+        // rows [m0 + 32q, +32) of the tile; f32 boxes hold 32 columns, bf16 boxes 64
+        const bool f32out = a.epi == EPI_RESID_F32 || a.epi == EPI_F32;
+        const int ccols = f32out ? 32 : 64;
+        const int ym = ti.m0 + q * 32;
+        const int rs = lane & 7;   // swizzle phase of this thread's row
+#pragma unroll 1
+        for (int cs = 0; cs < BN / ccols; ++cs) {
+          const int n = n0 + cs * ccols;
+          float v[64];
+          {
+            uint32_t r[32];
+            tmem_ld32(taddr + cs * ccols, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+            if (!f32out) {
+              tmem_ld32(taddr + cs * ccols + 32, r);
+              tmem_ld_wait();
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[32 + j] = __uint_as_float(r[j]);
+            }
+          }
+          uint8_t* box = stg + (warp - 2) * 8192 + ebuf * 4096;
+          if (lane == 0) bulk_wait_read<1>();   // this buffer's previous store has read it
+          __syncwarp();
+          if (f32out) {
+            if (a.bias != nullptr) {
+              const float4* bp = reinterpret_cast<const float4*>(a.bias + n);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const float4 b = bp[j];
+                v[4 * j] += b.x; v[4 * j + 1] += b.y; v[4 * j + 2] += b.z; v[4 * j + 3] += b.w;
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<float4*>(box + lane * 128 + ((j ^ rs) << 4)) =
+                  make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+          } else {
+            if (a.bias != nullptr) {
+              const float4* bp = reinterpret_cast<const float4*>(a.bias + n);
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const float4 b = bp[j];
+                v[4 * j] += b.x; v[4 * j + 1] += b.y; v[4 * j + 2] += b.z; v[4 * j + 3] += b.w;
+              }
+            }
+            if (a.epi == EPI_GELU_BF16) {
+#pragma unroll
+              for (int j = 0; j < 64; ++j) v[j] = gelu_erf(v[j]);
+            } else if (a.epi == EPI_RELU_BF16) {
+#pragma unroll
+              for (int j = 0; j < 64; ++j) v[j] = fmaxf(v[j], 0.0f);
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              uint4 w;
+              w.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
+              w.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+              w.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+              w.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+              *reinterpret_cast<uint4*>(box + lane * 128 + ((j ^ rs) << 4)) = w;
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (a.epi == EPI_RESID_F32)
+              tma_reduce_add_2d(&tmO, box, n, ym);
+            else
+              tma_store_2d(&tmO, box, n, ym);
+            bulk_commit();
+          }
+          ebuf ^= 1;
+        }
+        tc_fence_before();
+        mbar_arrive(&tempty[buf]);
+      } else if (a.splits == 1) {
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t r[32];
@@ -513,6 +600,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         named_bar_sync(1, 128);   // s_last is reused by the next tile
       }
     }
+    if (a.tma_out && lane == 0) bulk_wait<0>();   // stores complete before the CTA exits
   }
   __syncthreads();
   if (warp == 1) {

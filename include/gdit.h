@@ -67,6 +67,7 @@ extern "C" {
 #define GDIT_FLAG_NO_GRAPH 2u         /* run eagerly (no CUDA graph); same kernels, for debugging */
 #define GDIT_FLAG_NO_SMALL 4u         /* never use the single-sample persistent loop (batch 1 then runs the
                                          same per-layer kernels as larger batches) */
+#define GDIT_FLAG_NO_TMA_STORE 8u     /* DiT GEMMs store their outputs thread by thread instead of by TMA */
 
 /* ------------------------------------------------------------------ config
  * Model geometry and capacity.  Every size is explicit.  Defaults of the

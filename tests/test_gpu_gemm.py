@@ -18,8 +18,14 @@ pytestmark = pytest.mark.gpu
     (4352, 1024, 1024, 256, 1),    # persistent: more tiles than SMs
     (65, 4096, 512, 128, 3),       # split-K with a ragged row tile
 ])
-def test_gemm_matches_float64(M, N, K, bn, splits):
+@pytest.mark.parametrize("tma_out", [False, True])
+def test_gemm_matches_float64(M, N, K, bn, splits, tma_out, monkeypatch):
+    """tma_out: the epilogue stages 32-row boxes in shared memory and stores them by TMA."""
     require_gpu()
+    if tma_out:
+        if splits > 1 or bn < 64:
+            pytest.skip("the TMA-store epilogue serves single-split tiles of width >= 64")
+        monkeypatch.setenv("GDIT_TEST_TMA_OUT", "1")
     import torch
     from flow_matching_dit_b200 import test_gemm
     g = torch.Generator().manual_seed(M * 7 + N + K)

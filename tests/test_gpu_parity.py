@@ -305,3 +305,17 @@ def test_single_sample_loop_edge_cases(head_tiny, tiny_weights, case):
     assert st == 0
     ref = run_oracle(tiny_weights, w.geom, inp, 4)
     assert_parity(gpu, ref, inp["init_noise"], f"single-sample loop, {case}")
+
+
+def test_tma_store_epilogue_is_bitwise_equal_to_thread_stores(full_weights):
+    """The DiT GEMMs' TMA store / reduce-add epilogue computes the same f32
+    values as the per-thread stores (same adds, same roundings)."""
+    require_gpu()
+    from flow_matching_dit_b200 import GDIT_FLAG_NO_TMA_STORE, ActionHead
+    w = synth.WORKLOADS["batched"]
+    inp = synth.make_inputs(w, seed=23)
+    with ActionHead(w.geom, full_weights, max_batch=32, max_seq=600) as a:
+        x, _ = run_gpu(a, inp, w.num_steps)
+    with ActionHead(w.geom, full_weights, max_batch=32, max_seq=600, flags=GDIT_FLAG_NO_TMA_STORE) as b:
+        y, _ = run_gpu(b, inp, w.num_steps)
+    np.testing.assert_array_equal(x, y)
