@@ -11,10 +11,12 @@
 // projectors"), which run grouped: rows are sorted by embodiment and each
 // group multiplies by its own category's weights.
 //
-// CTA = 6 warps: warp 0 issues TMA loads into a STAGES-deep shared-memory
+// CTA = 10 warps: warp 0 issues TMA loads into a STAGES-deep shared-memory
 // ring, warp 1 allocates TMEM and one thread issues tcgen05.mma (128 x BN x 16
-// per instruction) into one of two TMEM accumulators, warps 2-5 drain the
-// other accumulator through tcgen05.ld and run the epilogue.  Tiles are
+// per instruction) into one of two TMEM accumulators, warps 2-9 drain the
+// other accumulator through tcgen05.ld and run the epilogue: two warps per
+// 32-lane TMEM quarter, taking alternate column chunks, so that on each SM
+// sub-partition one epilogue warp computes while the other waits on memory.  Tiles are
 // 128 x BN (BN in {32, 64, 128, 256}) with 64-wide K blocks in the 128-byte
 // swizzled layout.  Split-K is deterministic: every split writes an f32
 // partial, and the last split to finish (per-tile counter) sums the partials
@@ -41,7 +43,9 @@ enum Epi : int {
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;
-constexpr int kGemmThreads = 192;
+constexpr int kEpiWarps = 8;
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kGemmThreads = 64 + kEpiThreads;
 constexpr int kMaxGroups = 64;
 
 struct GemmArgs {
@@ -82,7 +86,7 @@ struct GemmCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
   static constexpr int TMEM_COLS = 2 * BN;
-  static constexpr int STG_BYTES = 4 * 2 * 4096;   // per epilogue warp: two 32 x 128-byte staging boxes
+  static constexpr int STG_BYTES = kEpiWarps * 4096;   // per epilogue warp: one 32 x 128-byte staging box
   static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + STG_BYTES + 256;
   static constexpr uint32_t IDESC = idesc_bf16_f32(kBM, BN);
 };
@@ -314,7 +318,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 128);
+      mbar_init(&tempty[b], kEpiThreads);
     }
     fence_mbar_init();
     s_abort = 0;
@@ -432,10 +436,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2..5)
+    // ------------------------------------------------------------ epilogue (warps 2..9)
     const int q = warp & 3;             // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;   // column chunks half, half + 2, ... of the tile
     const int row = q * 32 + lane;
-    int ebuf = 0;                       // staging box of the next TMA store
     int it = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
       TileInfo ti;
@@ -458,7 +462,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int ym = ti.m0 + q * 32;
         const int rs = lane & 7;   // swizzle phase of this thread's row
 #pragma unroll 1
-        for (int cs = 0; cs < BN / ccols; ++cs) {
+        for (int cs = half; cs < BN / ccols; cs += 2) {
           const int n = n0 + cs * ccols;
           float v[64];
           {
@@ -474,8 +478,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               for (int j = 0; j < 32; ++j) v[32 + j] = __uint_as_float(r[j]);
             }
           }
-          uint8_t* box = stg + (warp - 2) * 8192 + ebuf * 4096;
-          if (lane == 0) bulk_wait_read<1>();   // this buffer's previous store has read it
+          uint8_t* box = stg + (warp - 2) * 4096;
+          if (lane == 0) bulk_wait_read<0>();   // this warp's previous store has read its box
           __syncwarp();
           if (f32out) {
             if (a.bias != nullptr) {
@@ -525,13 +529,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               tma_store_2d(&tmO, box, n, ym);
             bulk_commit();
           }
-          ebuf ^= 1;
         }
         tc_fence_before();
         mbar_arrive(&tempty[buf]);
       } else if (a.splits == 1) {
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = half; c < BN / 32; c += 2) {
           uint32_t r[32];
           tmem_ld32(taddr + c * 32, r);
           tmem_ld_wait();
@@ -549,7 +552,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // write this split's partial, then the last split reduces in split order
         float* wsp = a.ws + ((long long)ti.split * a.M + m) * a.N;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = half; c < BN / 32; c += 2) {
           uint32_t r[32];
           tmem_ld32(taddr + c * 32, r);
           tmem_ld_wait();
@@ -565,18 +568,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tc_fence_before();
         mbar_arrive(&tempty[buf]);
         __threadfence();
-        named_bar_sync(1, 128);
+        named_bar_sync(1, kEpiThreads);
         if (threadIdx.x == 64) {
           const int old = atomicAdd(&a.counters[ti.unit], 1);
           s_last = (old == a.splits - 1);
           if (s_last) a.counters[ti.unit] = 0;
         }
-        named_bar_sync(1, 128);
+        named_bar_sync(1, kEpiThreads);
         if (s_last) {
           __threadfence();
           if (row_ok) {
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
+            for (int c = half; c < BN / 32; c += 2) {
               const int n = n0 + c * 32;
               if (n >= a.N) break;
               float v[32];
@@ -597,7 +600,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
           }
         }
-        named_bar_sync(1, 128);   // s_last is reused by the next tile
+        named_bar_sync(1, kEpiThreads);   // s_last is reused by the next tile
       }
     }
     if (a.tma_out && lane == 0) bulk_wait<0>();   // stores complete before the CTA exits
