@@ -768,6 +768,24 @@ GemmOp plan_gemm(gdit_handle* h, const void* A, long long a_rows, int K, const v
   return op;
 }
 
+// Whether one sample of N tokens fits the single-sample loop: its shared
+// buffers, its weight chunking (K <= 1024 or a multiple of 1024) and at most
+// kSmallMaxUnits units of 8 features per CTA in every linear.
+bool small_loop_fits(const gdit_config& c, int N, int num_sms) {
+  const long long D = c.hidden, F = c.mlp_hidden, A = c.action_dim;
+  if (N > kSmallMaxTok || D > kSmallMaxD || c.num_layers > kSmallMaxLayers || c.num_heads > num_sms) return false;
+  if ((long long)N * D * 4 > kSmLnStageBytes || (long long)N * (D + 8) * 2 > kSmLnStage) return false;
+  for (long long K : {A, D, F}) {
+    if (K % 16 != 0 || (K > kSmallKC && K % kSmallKC != 0)) return false;
+    if ((long long)N * (K + 8) * 2 > kSmXBytes) return false;
+  }
+  for (long long n_out : {A, D, 3 * D, F}) {
+    if (n_out % kSmallUF != 0) return false;
+    if ((n_out / kSmallUF + num_sms - 1) / num_sms > kSmallMaxUnits) return false;
+  }
+  return true;
+}
+
 std::unique_ptr<Profile> build_profile(gdit_handle* h, int B, int S, int K, int bf16) {
   auto p = std::make_unique<Profile>();
   p->B = B;
@@ -892,8 +910,7 @@ std::unique_ptr<Profile> build_profile(gdit_handle* h, int B, int S, int K, int 
     g->weight_bytes = (long long)g->args.N * g->args.K * 2;   // per category used
 
   // one sample: the K-step loop as one persistent kernel
-  p->small = B == 1 && N <= kSmallMaxTok && D <= kSmallMaxD && L <= kSmallMaxLayers &&
-             h->cfg.num_heads <= h->num_sms && N * D * 4 <= kSmHStageBytes && (h->cfg.flags & GDIT_FLAG_NO_SMALL) == 0;
+  p->small = B == 1 && small_loop_fits(h->cfg, N, h->num_sms) && (h->cfg.flags & GDIT_FLAG_NO_SMALL) == 0;
   if (p->small) {
     const Tables& t = h->tables.at(K);
     SmallPlan sp;
