@@ -62,18 +62,27 @@ __device__ __forceinline__ uint32_t mbar_try_wait(uint64_t* bar, uint32_t parity
   return ok;
 }
 
+// A waiter looks at the shared status word (another wait's timeout) only
+// after it has itself waited this long: thousands of threads polling one
+// global word on every iteration would queue at its L2 slice and delay every
+// wakeup by the length of that queue.
+constexpr unsigned long long kWaitPeekNs = 50000ull;
+
 // Waits for the phase with the given parity to complete.  Returns false (and
 // sets DEV_ERR_TIMEOUT in *err) if it has not completed within kWaitTimeoutNs,
-// or at once if another wait has already recorded a timeout in *err.
+// or soon after another wait has recorded a timeout in *err.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* err) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
-    // once any wait of the call has timed out, every other wait gives up at once
-    if (*reinterpret_cast<volatile unsigned*>(err) & DEV_ERR_TIMEOUT) return false;
-    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
-      atomicOr(err, DEV_ERR_TIMEOUT);
-      return false;
+    const unsigned long long dt = globaltimer_ns() - t0;
+    if (dt > kWaitPeekNs) {
+      // once any wait of the call has timed out, every other wait gives up
+      if (*reinterpret_cast<volatile unsigned*>(err) & DEV_ERR_TIMEOUT) return false;
+      if (dt > kWaitTimeoutNs) {
+        atomicOr(err, DEV_ERR_TIMEOUT);
+        return false;
+      }
     }
   }
   return true;

@@ -55,12 +55,14 @@ constexpr int kSlotBytes = kSmallUF * kSlotRow * 2;
 constexpr int kSmXBytes = 139776;                        // X rows / LN staging / attention / reduction
 constexpr int kSmLnStage = kSmXBytes / 2;                // f32 h rows staged for LN (upper half)
 constexpr int kSmLnStageBytes = kSmXBytes - kSmLnStage;
+constexpr int kSmLnParams = kSmLnStage - 2 * kSmallMaxD * 4;   // LN modulation vectors p0, p1 (f32)
 constexpr int kSmRing = kSmXBytes;                       // weight slots
 constexpr int kSmHold = kSmRing + kSmallSlots * kSlotBytes;                       // [unit][tok][8] f32 old values
 constexpr int kSmBias = kSmHold + kSmallMaxUnits * kSmallMaxTok * kSmallUF * 4;  // [unit][8] f32
 constexpr int kSmallSmem = kSmBias + kSmallMaxUnits * kSmallUF * 4;
 constexpr int kSmRedBytes = kSmallWarps * kSmallMaxUnits * kSmallMaxTok * kSmallUF * 4;   // over X
 static_assert(kSmRedBytes <= kSmXBytes, "reduction buffer fits the X area");
+static_assert(kSmallMaxUnits <= kSmallSlots, "one K-chunk of every unit of a phase is resident at once");
 static_assert(kSmallSmem <= 227 * 1024 - 1024, "shared memory budget");
 
 struct SmallLayer {
@@ -96,7 +98,7 @@ struct SmallPlan {
   const __nv_bfloat16 *wa1t, *wa2at, *wa3t, *wd1t, *wd2t, *proj_w;
   const float *ba1, *ba3, *bd1, *bd2, *proj_b;
   SmallLayer layers[kSmallMaxLayers];
-  int* counters;             // one per phase, zero at launch
+  int* counters;             // one arrival counter per phase, zero at launch
   struct SmallPhase* phases; // descriptor of every phase, written by small_describe_kernel
   unsigned* err;
 };
@@ -154,7 +156,11 @@ __device__ __forceinline__ void red_release_add(int* p, int v) {
   asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-struct SmallPhase {
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+struct alignas(16) SmallPhase {
   int kind;          // 0 GEMM, 1 attention
   SmallGemm g;
   AttnArgs a;
@@ -241,9 +247,25 @@ __device__ __forceinline__ void small_describe(const SmallPlan& P, int c, int k,
   }
 }
 
+// The plan's scalars that the loop reads in every phase, copied into registers
+// once: a field read through the plan pointer would be reloaded from global
+// memory after every barrier or fence (they clobber memory), and with nearly
+// all of L1 given to shared memory each reload is an L2 round trip.
+struct SmallCtx {
+  unsigned* err;
+  int* counters;
+  const float* h;
+  float eps;
+  const SmallPhase* phases;
+  const int* vofs;
+  int dh;
+};
+
 // Thread 0 waits (acquire) until `target` CTAs have arrived on `phase`; the
-// compute warps then continue together.
-__device__ __forceinline__ bool small_wait(const SmallPlan& P, int phase, int target, int* s_ok) {
+// compute warps then continue together.  One counter per phase: a waiter
+// polls a single word.  (One flag per CTA, polled as 37 16-byte words by a
+// warp, measured 0.85 ms slower per call: the polls flood L2.)
+__device__ __forceinline__ bool small_wait(const SmallCtx& P, int phase, int target, int* s_ok) {
   if (threadIdx.x == 0) {
     int ok = 1;
     if (phase >= 0 && target > 0) {
@@ -251,11 +273,14 @@ __device__ __forceinline__ bool small_wait(const SmallPlan& P, int phase, int ta
       if (ld_acquire(c) < target) {
         const unsigned long long t0 = globaltimer_ns();
         while (ld_acquire(c) < target) {
-          if (*reinterpret_cast<volatile unsigned*>(P.err) & DEV_ERR_TIMEOUT) { ok = 0; break; }
-          if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
-            atomicOr(P.err, DEV_ERR_TIMEOUT);
-            ok = 0;
-            break;
+          const unsigned long long dt = globaltimer_ns() - t0;
+          if (dt > kWaitPeekNs) {
+            if (*reinterpret_cast<volatile unsigned*>(P.err) & DEV_ERR_TIMEOUT) { ok = 0; break; }
+            if (dt > kWaitTimeoutNs) {
+              atomicOr(P.err, DEV_ERR_TIMEOUT);
+              ok = 0;
+              break;
+            }
           }
         }
       }
@@ -267,7 +292,7 @@ __device__ __forceinline__ bool small_wait(const SmallPlan& P, int phase, int ta
 }
 
 // All compute threads' writes of the phase, then one release increment.
-__device__ __forceinline__ void small_arrive(const SmallPlan& P, int phase) {
+__device__ __forceinline__ void small_arrive(const SmallCtx& P, int phase) {
   csync();
   if (threadIdx.x == 0) red_release_add(P.counters + phase, 1);
 }
@@ -298,7 +323,7 @@ struct SmallRing {
 // Streams this CTA's weight chunks of every GEMM phase, in the order the
 // compute warps consume them, into the slot ring; runs ahead as far as free
 // slots allow.  Lanes 0..7 each copy one weight row per chunk.
-__device__ __forceinline__ void small_producer(const SmallPlan& P, int total, uint8_t* smem, SmallRing& R) {
+__device__ __forceinline__ void small_producer(const SmallCtx& P, int total, uint8_t* smem, SmallRing& R) {
   const int lane = threadIdx.x & 31;
   uint32_t item = 0;
   bool ok = true;
@@ -327,8 +352,8 @@ __device__ __forceinline__ void small_producer(const SmallPlan& P, int total, ui
     if (ph.kind != 0) continue;
     const SmallGemm& g = ph.g;
     const int nu = small_my_units(g), nch = small_nchunks(g), kc = small_kc(g);
-    for (int j = 0; j < nu && ok; ++j) {
-      for (int c = 0; c < nch; ++c, ++item) {
+    for (int c = 0; c < nch && ok; ++c) {
+      for (int j = 0; j < nu; ++j, ++item) {
         const int slot = (int)(item % kSmallSlots);
         const uint32_t use = item / kSmallSlots;
         int good = 1;
@@ -362,19 +387,28 @@ __device__ __forceinline__ void small_producer(const SmallPlan& P, int total, ui
 
 // ---------------------------------------------------------------- GEMM phase (compute warps)
 
-// bf16 rows of X (row stride ldx) -> shared rows of K + 8 elements; bias and,
-// for the residual and Euler epilogues, the old output values of this CTA's
-// units.  One cp.async group.
-__device__ __forceinline__ void small_issue_inputs(const SmallGemm& g, const SmallPlan& P, int nu, uint8_t* smem) {
-  const int tid = threadIdx.x;
-  if (g.x_mode == 0) {
-    const int pieces = g.K / 8, xrow = g.K + 8;
-    __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(smem);
-    for (int i = tid; i < g.rows * pieces; i += kSmallCompute) {
-      const int r = i / pieces, q = i - r * pieces;
-      cp_async16(xs + r * xrow + q * 8, g.X + (size_t)r * g.ldx + q * 8, true);
-    }
+// Warp 0: the phase's bf16 activation rows (row stride ldx) by bulk copies on
+// `xbar`, into shared rows of K + 8 elements.  The proxy fences order the
+// other CTAs' stores (seen through the acquire) and this CTA's earlier reads
+// of the area before the async-proxy copies.
+__device__ __forceinline__ void small_issue_x(const SmallGemm& g, uint8_t* smem, uint64_t* xbar) {
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x >= 32) return;
+  if (lane == 0) {
+    fence_proxy_async_global();
+    fence_proxy_async_smem();
+    mbar_arrive_expect_tx(xbar, (uint32_t)(g.rows * g.K * 2));
   }
+  __syncwarp();
+  const int xrow = g.K + 8;
+  for (int r = lane; r < g.rows; r += 32)
+    bulk_g2s(smem + (size_t)r * xrow * 2, g.X + (size_t)r * g.ldx, (uint32_t)g.K * 2u, xbar);
+}
+
+// Bias and, for the residual and Euler epilogues, the old output values of
+// this CTA's units: one cp.async group, waited for before the epilogue.
+__device__ __forceinline__ void small_issue_side(const SmallGemm& g, int nu, uint8_t* smem) {
+  const int tid = threadIdx.x;
   const float* bsrc = g.epi == EPI_SWISH_VEC_BF16 ? g.vec : g.bias;
   if (bsrc != nullptr && tid < 2 * nu) {
     const int j = tid >> 1, q = tid & 1;
@@ -391,62 +425,82 @@ __device__ __forceinline__ void small_issue_inputs(const SmallGemm& g, const Sma
                  true);
     }
   }
-  if (g.x_mode == 1) {
-    // f32 h rows for LN, staged in the upper half of the X area
-    const int D = g.K, d4 = D / 4;
-    float* hs = reinterpret_cast<float*>(smem + kSmLnStage);
-    for (int i = tid; i < g.rows * d4; i += kSmallCompute) {
-      const int r = i / d4, q = i - r * d4;
-      cp_async16(hs + (size_t)r * D + q * 4, P.h + (size_t)(g.h_row_off + r) * D + q * 4, true);
-    }
-  }
   cp_async_commit();
 }
 
-// LN(h rows) -> bf16 X rows (after the staging group has landed): per-row
-// mean and E[x^2] in one pass, then the AdaLN (1 + p0, p1) or affine (p0, p1)
-// modulation.
-__device__ __forceinline__ void small_ln_rows(const SmallGemm& g, float eps, uint8_t* smem, float* stat) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+// LN(h rows) -> bf16 X rows.  Thread t owns columns [4t, 4t + 4) of every
+// row: it loads them from L2 into registers, the CTA reduces each row's sum
+// and sum of squares (warp shuffles, then the 8 warps' totals through shared
+// memory), and the thread writes its columns of every normalised row with the
+// AdaLN ((1 + p0), p1) or affine (p0, p1) modulation, loaded once.
+__device__ __forceinline__ void small_ln_rows(const SmallGemm& g, const SmallCtx& P, uint8_t* smem) {
+  constexpr int G = 17;   // rows per round (N = H + 1 = 17 in one)
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int D = g.K, d4 = D / 4, xrow = D + 8;
-  const float* hs = reinterpret_cast<const float*>(smem + kSmLnStage);
-  for (int r = warp; r < g.rows; r += kSmallWarps) {
-    const float4* row = reinterpret_cast<const float4*>(hs + (size_t)r * D);
-    float s0 = 0.0f, s1 = 0.0f, q0 = 0.0f, q1 = 0.0f;
-    for (int c = lane; c < d4; c += 32) {
-      const float4 v = row[c];
-      s0 += v.x + v.y;
-      s1 += v.z + v.w;
-      q0 += v.x * v.x + v.y * v.y;
-      q1 += v.z * v.z + v.w * v.w;
-    }
-    float sum = s0 + s1, sq = q0 + q1;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      sq += __shfl_xor_sync(0xffffffffu, sq, o);
-    }
-    if (lane == 0) {
-      const float mean = sum / (float)D;
-      stat[r * 2] = mean;
-      stat[r * 2 + 1] = rsqrtf(fmaxf(sq / (float)D - mean * mean, 0.0f) + eps);
-    }
-  }
-  csync();
+  const bool has = tid < d4;
+  float* part = reinterpret_cast<float*>(smem + kSmLnStage);   // [warp][row][2]
+  float* stat = part + kSmallWarps * G * 2;                     // [row][2]
   __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(smem);
-  for (int c4 = threadIdx.x; c4 < d4; c4 += kSmallCompute) {
-    const float4 a = reinterpret_cast<const float4*>(g.p0)[c4];
-    const float4 b = reinterpret_cast<const float4*>(g.p1)[c4];
-    const float a0 = g.ln_mode == 0 ? 1.0f + a.x : a.x, a1 = g.ln_mode == 0 ? 1.0f + a.y : a.y;
-    const float a2 = g.ln_mode == 0 ? 1.0f + a.z : a.z, a3 = g.ln_mode == 0 ? 1.0f + a.w : a.w;
-    for (int r = 0; r < g.rows; ++r) {
-      const float4 v = reinterpret_cast<const float4*>(hs + (size_t)r * D)[c4];
-      const float mean = stat[r * 2], rstd = stat[r * 2 + 1];
-      uint2 w;
-      w.x = pack_bf16x2((v.x - mean) * rstd * a0 + b.x, (v.y - mean) * rstd * a1 + b.y);
-      w.y = pack_bf16x2((v.z - mean) * rstd * a2 + b.z, (v.w - mean) * rstd * a3 + b.w);
-      *reinterpret_cast<uint2*>(xs + (size_t)r * xrow + 4 * c4) = w;
+  const float4 zero = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  float4 a = zero, b = zero;
+  if (has) {
+    a = __ldg(reinterpret_cast<const float4*>(g.p0) + tid);
+    b = __ldg(reinterpret_cast<const float4*>(g.p1) + tid);
+  }
+  if (g.ln_mode == 0) {
+    a.x += 1.0f; a.y += 1.0f; a.z += 1.0f; a.w += 1.0f;
+  }
+  const float4* hcol = reinterpret_cast<const float4*>(P.h + (size_t)g.h_row_off * D) + tid;
+  for (int r0 = 0; r0 < g.rows; r0 += G) {
+    const int nr = min(G, g.rows - r0);
+    float4 v[G];
+#pragma unroll
+    for (int i = 0; i < G; ++i) v[i] = (has && i < nr) ? __ldcg(hcol + (size_t)(r0 + i) * d4) : zero;
+    float sm[G], sq[G];
+#pragma unroll
+    for (int i = 0; i < G; ++i) {
+      sm[i] = (v[i].x + v[i].y) + (v[i].z + v[i].w);
+      sq[i] = fmaf(v[i].x, v[i].x, fmaf(v[i].y, v[i].y, fmaf(v[i].z, v[i].z, v[i].w * v[i].w)));
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+      for (int i = 0; i < G; ++i) {
+        sm[i] += __shfl_xor_sync(0xffffffffu, sm[i], o);
+        sq[i] += __shfl_xor_sync(0xffffffffu, sq[i], o);
+      }
+    if (lane == 0)
+#pragma unroll
+      for (int i = 0; i < G; ++i) {
+        part[(warp * G + i) * 2] = sm[i];
+        part[(warp * G + i) * 2 + 1] = sq[i];
+      }
+    csync();
+    if (tid < nr) {
+      float S = 0.0f, Q = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kSmallWarps; ++w) {
+        S += part[(w * G + tid) * 2];
+        Q += part[(w * G + tid) * 2 + 1];
+      }
+      const float mean = S / (float)D;
+      stat[tid * 2] = mean;
+      stat[tid * 2 + 1] = rsqrtf(fmaxf(Q / (float)D - mean * mean, 0.0f) + P.eps);
+    }
+    csync();
+    if (has) {
+#pragma unroll
+      for (int i = 0; i < G; ++i) {
+        if (i < nr) {
+          const float mean = stat[i * 2], rstd = stat[i * 2 + 1];
+          uint2 w;
+          w.x = pack_bf16x2((v[i].x - mean) * rstd * a.x + b.x, (v[i].y - mean) * rstd * a.y + b.y);
+          w.y = pack_bf16x2((v[i].z - mean) * rstd * a.z + b.z, (v[i].w - mean) * rstd * a.w + b.w);
+          *reinterpret_cast<uint2*>(xs + (size_t)(r0 + i) * xrow + 4 * tid) = w;
+        }
+      }
+    }
+    csync();   // part / stat are reused by the next round
   }
 }
 
@@ -485,17 +539,23 @@ __device__ __forceinline__ void small_epilogue(const SmallGemm& g, int n, int to
 
 // One GEMM phase on the compute warps.  Chunk `item` of the CTA's running
 // count sits in slot item % kSmallSlots, filled for the (item / kSmallSlots)-th
-// time; every warp releases a slot after its last read of it.
-__device__ __forceinline__ bool small_gemm_phase(const SmallGemm& g, const SmallPlan& P, uint8_t* smem,
-                                                 SmallRing& R, uint32_t& item, float* stat) {
+// time; a phase's items go chunk by chunk (every unit's K-chunk 0, then 1 ...)
+// and every warp releases a slot after its last read of it.
+__device__ __forceinline__ bool small_gemm_phase(const SmallGemm& g, const SmallCtx& P, uint8_t* smem,
+                                                 SmallRing& R, uint32_t& item, uint64_t* xbar,
+                                                 uint32_t& xuse) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gr = lane >> 2, tig = lane & 3;
   const int nu = small_my_units(g), nch = small_nchunks(g), kc = small_kc(g);
-  small_issue_inputs(g, P, nu, smem);
-  cp_async_wait<0>();
-  csync();
-  if (g.x_mode == 1) {
-    small_ln_rows(g, P.eps, smem, stat);
+  small_issue_side(g, nu, smem);
+  bool ok = true;
+  if (g.x_mode == 0) {
+    small_issue_x(g, smem, xbar);
+    // every thread waits for the activations itself: no barrier before the MMAs
+    ok = mbar_wait(xbar, xuse & 1u, P.err);
+    ++xuse;
+  } else {
+    small_ln_rows(g, P, smem);
     csync();
   }
   const int xrow = g.K + 8;
@@ -503,48 +563,108 @@ __device__ __forceinline__ bool small_gemm_phase(const SmallGemm& g, const Small
   const int ks = kc / 16;
   const int ks0 = warp * ks / kSmallWarps, ks1 = (warp + 1) * ks / kSmallWarps;
   const bool two = g.rows > 16;
-  // A rows supplied by this lane (rows past the last token repeat it: their
-  // products land in accumulator rows that are never stored)
-  const int ar0 = min(lane & 15, g.rows - 1), ar1 = min(16 + (lane & 15), g.rows - 1);
+  // tile 0 (tokens 0-15): ldmatrix rows (rows past the last token repeat it:
+  // their products land in accumulator rows that are never stored)
+  const int ar0 = min(lane & 15, g.rows - 1);
   const __nv_bfloat16* xa0 = xs + (size_t)ar0 * xrow + (lane >> 4) * 8;
-  const __nv_bfloat16* xa1 = xs + (size_t)ar1 * xrow + (lane >> 4) * 8;
-  const int wrow = (lane & 7) * kSlotRow + ((lane >> 3) & 1) * 8;
-  float acc[kSmallMaxUnits][2][4];
+  // tile 1 (tokens 16-31) usually holds one real token: each lane reads only
+  // the 32-bit words of its fragment rows that exist (16 + gr, 24 + gr)
+  const bool lo1 = 16 + gr < g.rows, hi1 = 24 + gr < g.rows;
+  const __nv_bfloat16* xb_lo = xs + (size_t)(lo1 ? 16 + gr : 0) * xrow + 2 * tig;
+  const __nv_bfloat16* xb_hi = xs + (size_t)(hi1 ? 24 + gr : 0) * xrow + 2 * tig;
+  auto tile1 = [&](int kk, uint32_t (&f)[4]) {
+    f[0] = lo1 ? *reinterpret_cast<const uint32_t*>(xb_lo + kk) : 0u;
+    f[1] = hi1 ? *reinterpret_cast<const uint32_t*>(xb_hi + kk) : 0u;
+    f[2] = lo1 ? *reinterpret_cast<const uint32_t*>(xb_lo + kk + 8) : 0u;
+    f[3] = hi1 ? *reinterpret_cast<const uint32_t*>(xb_hi + kk + 8) : 0u;
+  };
+  // weight fragments: ldmatrix.x4 over k, k + 8, k + 16, k + 24 (two k-steps)
+  const int wrow = (lane & 7) * kSlotRow + (lane >> 3) * 8;
+  // accumulators per (unit, token tile); unit 0 keeps a second chain for the
+  // odd k-steps, so that single-unit phases still have independent MMAs
+  float acc[kSmallMaxUnits][2][4], acc2[2][4];
 #pragma unroll
   for (int j = 0; j < kSmallMaxUnits; ++j)
 #pragma unroll
     for (int t = 0; t < 2; ++t)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[j][t][e] = 0.0f;
-  bool ok = true;
 #pragma unroll
-  for (int j = 0; j < kSmallMaxUnits; ++j) {
-    if (j < nu && ok) {
-      for (int c = 0; c < nch; ++c, ++item) {
-        const int slot = (int)(item % kSmallSlots);
-        if (!mbar_wait(&R.full[slot], (item / kSmallSlots) & 1u, P.err)) { ok = false; break; }
-        const __nv_bfloat16* ws =
-            reinterpret_cast<const __nv_bfloat16*>(smem + kSmRing + slot * kSlotBytes) + wrow;
-        const int kx = c * kc;
-        for (int s = ks0; s < ks1; ++s) {
-          const int k = s * 16;
-          uint32_t b0, b1, a0, a1, a2, a3;
-          ldmatrix_x2(b0, b1, ws + k);
-          ldmatrix_x4(a0, a1, a2, a3, xa0 + kx + k);
-          mma_bf16_16816(acc[j][0], a0, a1, a2, a3, b0, b1);
-          if (two) {
-            ldmatrix_x4(a0, a1, a2, a3, xa1 + kx + k);
-            mma_bf16_16816(acc[j][1], a0, a1, a2, a3, b0, b1);
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&R.empty[slot]);
+  for (int t = 0; t < 2; ++t)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc2[t][e] = 0.0f;
+  // chunk c of every unit (items base + c * nu + j): wait for all, then each
+  // k-step loads the token fragments once and runs them against every unit
+  const uint32_t base = item;
+  for (int c = 0; c < nch; ++c) {
+    const __nv_bfloat16* wsj[kSmallMaxUnits];
+#pragma unroll
+    for (int j = 0; j < kSmallMaxUnits; ++j) {
+      wsj[j] = nullptr;
+      if (j < nu) {
+        const uint32_t it = base + (uint32_t)(c * nu + j);
+        const int slot = (int)(it % kSmallSlots);
+        if (ok && !mbar_wait(&R.full[slot], (it / kSmallSlots) & 1u, P.err)) ok = false;
+        wsj[j] = reinterpret_cast<const __nv_bfloat16*>(smem + kSmRing + slot * kSlotBytes) + wrow;
       }
     }
+    if (ok) {
+      const int kx = c * kc;
+      int s = ks0;
+      for (; s + 1 < ks1; s += 2) {
+        const int k = s * 16;
+        uint32_t a[4], e[4], a1[4], e1[4];
+        ldmatrix_x4(a[0], a[1], a[2], a[3], xa0 + kx + k);
+        ldmatrix_x4(e[0], e[1], e[2], e[3], xa0 + kx + k + 16);
+        if (two) {
+          tile1(kx + k, a1);
+          tile1(kx + k + 16, e1);
+        }
+#pragma unroll
+        for (int j = 0; j < kSmallMaxUnits; ++j) {
+          if (j < nu) {
+            uint32_t b[4];
+            ldmatrix_x4(b[0], b[1], b[2], b[3], wsj[j] + k);
+            float(&o0)[4] = j == 0 ? acc2[0] : acc[j][0];
+            float(&o1)[4] = j == 0 ? acc2[1] : acc[j][1];
+            mma_bf16_16816(acc[j][0], a[0], a[1], a[2], a[3], b[0], b[1]);
+            mma_bf16_16816(o0, e[0], e[1], e[2], e[3], b[2], b[3]);
+            if (two) {
+              mma_bf16_16816(acc[j][1], a1[0], a1[1], a1[2], a1[3], b[0], b[1]);
+              mma_bf16_16816(o1, e1[0], e1[1], e1[2], e1[3], b[2], b[3]);
+            }
+          }
+        }
+      }
+      if (s < ks1) {   // odd step count (narrow K)
+        const int k = s * 16;
+        uint32_t a[4], a1[4];
+        ldmatrix_x4(a[0], a[1], a[2], a[3], xa0 + kx + k);
+        if (two) tile1(kx + k, a1);
+#pragma unroll
+        for (int j = 0; j < kSmallMaxUnits; ++j) {
+          if (j < nu) {
+            uint32_t b0, b1;
+            ldmatrix_x2(b0, b1, wsj[j] + k);
+            mma_bf16_16816(acc[j][0], a[0], a[1], a[2], a[3], b0, b1);
+            if (two) mma_bf16_16816(acc[j][1], a1[0], a1[1], a1[2], a1[3], b0, b1);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0)
+        for (int j = 0; j < nu; ++j) mbar_arrive(&R.empty[(base + (uint32_t)(c * nu + j)) % kSmallSlots]);
+    }
   }
+  item = base + (uint32_t)(nch * nu);
   // all warps stay together from here on, also on a timeout
+  cp_async_wait<0>();   // bias / old values
   csync();
   float* red = reinterpret_cast<float*>(smem);   // over the X area, no longer read
+#pragma unroll
+  for (int t = 0; t < 2; ++t)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[0][t][e] += acc2[t][e];
 #pragma unroll
   for (int j = 0; j < kSmallMaxUnits; ++j) {
     if (j < nu) {
@@ -690,31 +810,36 @@ __global__ void small_describe_kernel(const SmallPlan* __restrict__ plan) {
   small_describe(P, small_category(P), gp / per_step, gp % per_step, P.phases[gp]);
 }
 
-// compute threads: descriptor gp -> shared slot
-__device__ __forceinline__ void small_load_phase(const SmallPlan& P, int gp, SmallPhase* dst) {
-  static_assert(sizeof(SmallPhase) % 4 == 0, "descriptor copied as words");
-  const uint32_t* src = reinterpret_cast<const uint32_t*>(P.phases + gp);
-  uint32_t* d = reinterpret_cast<uint32_t*>(dst);
-  for (int i = threadIdx.x; i < (int)(sizeof(SmallPhase) / 4); i += kSmallCompute) d[i] = src[i];
+// compute threads: descriptor gp -> shared slot, as one cp.async group (no
+// stall; complete by the next wait_group 0)
+__device__ __forceinline__ void small_fetch_phase(const SmallPhase* phases, int gp, SmallPhase* dst) {
+  static_assert(sizeof(SmallPhase) % 16 == 0, "descriptor copied in 16-byte pieces");
+  constexpr int kPieces = (int)(sizeof(SmallPhase) / 16);
+  static_assert(kPieces <= kSmallCompute, "one piece per thread");
+  if (threadIdx.x < kPieces)
+    cp_async16(reinterpret_cast<uint8_t*>(dst) + threadIdx.x * 16,
+               reinterpret_cast<const uint8_t*>(phases + gp) + threadIdx.x * 16, true);
+  cp_async_commit();
 }
 
 template <int DH>
 __global__ void __launch_bounds__(kSmallThreads, 1) small_loop_kernel(const SmallPlan* __restrict__ plan) {
   extern __shared__ __align__(16) uint8_t smem[];
-  // phase descriptors: slot gp & 1 holds the current phase, the other the next
-  __shared__ __align__(16) SmallPhase s_ph[2];
+  // phase descriptors: slot gp % 3 holds the current phase; the one two ahead
+  // is fetched while the current one runs
+  __shared__ __align__(16) SmallPhase s_ph[3];
   __shared__ __align__(8) SmallRing s_ring;
-  __shared__ float s_stat[kSmallMaxTok * 2];
+  __shared__ __align__(8) uint64_t s_xbar;
   __shared__ int s_ok;
   __shared__ int s_fail;
-  const SmallPlan& P = *plan;
-  const int per_step = 5 * P.L + 6;
-  const int total = per_step * P.K;
+  const SmallCtx P = {plan->err, plan->counters, plan->h, plan->eps, plan->phases, plan->vofs, plan->dh};
+  const int total = (5 * plan->L + 6) * plan->K;
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSmallSlots; ++i) {
       mbar_init(&s_ring.full[i], 1);
       mbar_init(&s_ring.empty[i], kSmallWarps);
     }
+    mbar_init(&s_xbar, 1);
     fence_mbar_init();
     s_fail = 0;
   }
@@ -723,20 +848,24 @@ __global__ void __launch_bounds__(kSmallThreads, 1) small_loop_kernel(const Smal
     small_producer(P, total, smem, s_ring);
     return;
   }
-  small_load_phase(P, 0, &s_ph[0]);
+  small_fetch_phase(P.phases, 0, &s_ph[0]);
+  if (total > 1) small_fetch_phase(P.phases, 1, &s_ph[1]);
+  cp_async_wait<0>();
   csync();
   uint32_t item = 0;   // weight chunks consumed so far (same count in every compute thread)
+  uint32_t xuse = 0;   // activation loads on s_xbar so far
   int prev_workers = 0;
+  int slot = 0;        // gp % 3
   for (int gp = 0; gp < total; ++gp) {
-    const SmallPhase& cur = s_ph[gp & 1];
-    if (gp + 1 < total) small_load_phase(P, gp + 1, &s_ph[(gp + 1) & 1]);
+    const SmallPhase& cur = s_ph[slot];
+    if (gp + 2 < total) small_fetch_phase(P.phases, gp + 2, &s_ph[slot == 0 ? 2 : slot - 1]);
     const int w = small_phase_workers(cur);
     bool ok = true;
     if ((int)blockIdx.x < w) {
       ok = small_wait(P, gp - 1, prev_workers, &s_ok);
       if (ok) {
         if (cur.kind == 0) {
-          if (!small_gemm_phase(cur.g, P, smem, s_ring, item, s_stat)) s_fail = 1;
+          if (!small_gemm_phase(cur.g, P, smem, s_ring, item, &s_xbar, xuse)) s_fail = 1;
           csync();
           ok = s_fail == 0;
         } else {
@@ -747,10 +876,20 @@ __global__ void __launch_bounds__(kSmallThreads, 1) small_loop_kernel(const Smal
     }
     if (!ok) {
       cp_async_wait<0>();   // requested rows land before the CTA exits
+      if (threadIdx.x == 0) {
+        // the last activation load (if any) lands too
+        const unsigned long long t0 = globaltimer_ns();
+        while (xuse > 0u && !mbar_try_wait(&s_xbar, (xuse - 1u) & 1u) && globaltimer_ns() - t0 < 10000000ull) {
+        }
+      }
       return;
     }
     prev_workers = w;
-    csync();   // every compute thread is done with s_ph[gp & 1] before it is rewritten
+    // the next descriptor has landed, and every compute thread is done with
+    // this one before its slot is refilled
+    cp_async_wait<0>();
+    csync();
+    slot = slot == 2 ? 0 : slot + 1;
   }
 }
 
