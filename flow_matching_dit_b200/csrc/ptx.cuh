@@ -50,6 +50,20 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// As mbar_try_wait, but a waiting thread may be suspended (not spinning) for
+// up to `ns` nanoseconds; it resumes as soon as the phase completes.
+__device__ __forceinline__ uint32_t mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok;
+}
+
 __device__ __forceinline__ uint32_t mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -67,6 +81,9 @@ __device__ __forceinline__ uint32_t mbar_try_wait(uint64_t* bar, uint32_t parity
 // global word on every iteration would queue at its L2 slice and delay every
 // wakeup by the length of that queue.
 constexpr unsigned long long kWaitPeekNs = 50000ull;
+// Longest suspension of one try_wait (the thread resumes earlier when the
+// phase completes); bounds how late a timeout is noticed.
+constexpr uint32_t kWaitSleepNs = 1000000u;
 
 // Waits for the phase with the given parity to complete.  Returns false (and
 // sets DEV_ERR_TIMEOUT in *err) if it has not completed within kWaitTimeoutNs,
@@ -74,7 +91,9 @@ constexpr unsigned long long kWaitPeekNs = 50000ull;
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* err) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
+  // suspended rather than spinning, so that waiting warps leave the issue
+  // slots to the warps that do the work
+  while (!mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) {
     const unsigned long long dt = globaltimer_ns() - t0;
     if (dt > kWaitPeekNs) {
       // once any wait of the call has timed out, every other wait gives up
