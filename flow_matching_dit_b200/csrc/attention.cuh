@@ -42,12 +42,12 @@ struct AttnArgs {
 
 // MT: 16-row query tiles (queries padded to 16 * MT); DH: head dim (32 or 64).
 // Shared-memory rows hold DH + 8 bf16 so fragment loads are bank-conflict free.
-template <int MT, int DH>
+template <int MT, int DH, int RING_ = 3>
 struct AttnSmem {
   static constexpr int ROW = DH + 8;
   static constexpr int Q_ELEMS = MT * 16 * ROW;
   static constexpr int CHUNK_ELEMS = 16 * ROW;                    // 16 keys x DH dims (padded)
-  static constexpr int RING = 3;                                  // chunks in flight per warp
+  static constexpr int RING = RING_;                              // chunks in flight per warp
   static constexpr int RING_ELEMS = RING * 2 * CHUNK_ELEMS;       // (K, V) per slot
   // split schedule: one Q tile, 4 rings, per-warp partials
   static constexpr int SPLIT_O_BYTES = 4 * MT * 16 * DH * 4;
@@ -122,12 +122,12 @@ __device__ __forceinline__ void attn_init(float (&o)[MT][DH / 8][4], float (&mro
 
 // One warp: chunks c0, c0 + cstep, ... of the keys [k_begin, k_begin + n_keys)
 // of head h, folded into (o, mrow, lrow) with an online softmax.
-template <int MT, int DH>
+template <int MT, int DH, int RING_ = 3>
 __device__ __forceinline__ void attn_stream_chunks(const AttnArgs& a, int h, int k_begin, int n_keys, int c0,
                                                    int cstep, const __nv_bfloat16* sQ, __nv_bfloat16* ring,
                                                    float (&o)[MT][DH / 8][4], float (&mrow)[MT][2],
                                                    float (&lrow)[MT][2]) {
-  using SM = AttnSmem<MT, DH>;
+  using SM = AttnSmem<MT, DH, RING_>;
   constexpr int ROW = SM::ROW;
   constexpr int PIECES = DH / 8;
   const int lane = threadIdx.x & 31;
@@ -346,9 +346,15 @@ __global__ void __launch_bounds__(kAttnThreads) attention_split_kernel(const Att
 }
 
 // ---------------------------------------------------------------- warp schedule
+// Ring depth of the warp schedule: two chunks in flight per warp keep a warp's
+// shared memory at 13.8 KB (DH 64), so 16 warps fit an SM.
+constexpr int kWarpRing = 2;
+
+// Persistent: warp w of CTA c takes items c * 4 + w, + 4 * gridDim.x, ...; the
+// host sizes the grid so that every warp gets the same number of items.
 template <int MT, int DH>
-__global__ void __launch_bounds__(kAttnThreads) attention_warp_kernel(const AttnArgs a) {
-  using SM = AttnSmem<MT, DH>;
+__global__ void __launch_bounds__(kAttnThreads, MT == 2 ? 4 : 2) attention_warp_kernel(const AttnArgs a) {
+  using SM = AttnSmem<MT, DH, kWarpRing>;
   extern __shared__ __align__(16) uint8_t smem[];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -359,36 +365,37 @@ __global__ void __launch_bounds__(kAttnThreads) attention_warp_kernel(const Attn
 
   pdl_wait();
   pdl_launch_dependents();
-  const int item = blockIdx.x * 4 + warp;
-  if (item >= a.num_items) return;
-  const int b = item / a.num_heads;
-  const int h = item - b * a.num_heads;
-  int k_begin, n_keys;
-  attn_key_range(a, b, k_begin, n_keys);
-  attn_load_q<MT, DH>(a, b, h, sQ, lane, 32);
-  __syncwarp();
+  for (int item = blockIdx.x * 4 + warp; item < a.num_items; item += gridDim.x * 4) {
+    const int b = item / a.num_heads;
+    const int h = item - b * a.num_heads;
+    int k_begin, n_keys;
+    attn_key_range(a, b, k_begin, n_keys);
+    attn_load_q<MT, DH>(a, b, h, sQ, lane, 32);
+    __syncwarp();
 
-  float o[MT][DH / 8][4];
-  float mrow[MT][2], lrow[MT][2];
-  attn_init<MT, DH>(o, mrow, lrow);
-  attn_stream_chunks<MT, DH>(a, h, k_begin, n_keys, 0, 1, sQ, ring, o, mrow, lrow);
+    float o[MT][DH / 8][4];
+    float mrow[MT][2], lrow[MT][2];
+    attn_init<MT, DH>(o, mrow, lrow);
+    attn_stream_chunks<MT, DH, kWarpRing>(a, h, k_begin, n_keys, 0, 1, sQ, ring, o, mrow, lrow);
 
-  __nv_bfloat16* obase = a.out + (long long)b * a.n_tok * a.out_ld + h * DH;
+    __nv_bfloat16* obase = a.out + (long long)b * a.n_tok * a.out_ld + h * DH;
 #pragma unroll
-  for (int mt = 0; mt < MT; ++mt) {
+    for (int mt = 0; mt < MT; ++mt) {
 #pragma unroll
-    for (int hr = 0; hr < 2; ++hr) {
-      float l = lrow[mt][hr];
-      l += __shfl_xor_sync(0xffffffffu, l, 1);
-      l += __shfl_xor_sync(0xffffffffu, l, 2);
-      const int row = mt * 16 + g + hr * 8;
-      if (row >= a.n_tok) continue;
-      const float inv = l > 0.0f ? 1.0f / l : 0.0f;   // no key: zero output
+      for (int hr = 0; hr < 2; ++hr) {
+        float l = lrow[mt][hr];
+        l += __shfl_xor_sync(0xffffffffu, l, 1);
+        l += __shfl_xor_sync(0xffffffffu, l, 2);
+        const int row = mt * 16 + g + hr * 8;
+        if (row >= a.n_tok) continue;
+        const float inv = l > 0.0f ? 1.0f / l : 0.0f;   // no key: zero output
 #pragma unroll
-      for (int nd = 0; nd < DH / 8; ++nd)
-        *reinterpret_cast<uint32_t*>(obase + (long long)row * a.out_ld + nd * 8 + tig * 2) =
-            pack_bf16x2(o[mt][nd][hr * 2 + 0] * inv, o[mt][nd][hr * 2 + 1] * inv);
+        for (int nd = 0; nd < DH / 8; ++nd)
+          *reinterpret_cast<uint32_t*>(obase + (long long)row * a.out_ld + nd * 8 + tig * 2) =
+              pack_bf16x2(o[mt][nd][hr * 2 + 0] * inv, o[mt][nd][hr * 2 + 1] * inv);
+      }
     }
+    __syncwarp();   // the Q tile is rewritten by the next item
   }
 }
 

@@ -650,14 +650,21 @@ void max_shared_carveout(K* kern) {
                                 (int)cudaSharedmemCarveoutMaxShared));
 }
 
+// CTAs of the warp-schedule attention kernel resident per SM, by (MT == 4, DH == 64)
+int g_attn_warp_ctas[2][2];
+
 template <int MT, int DH>
 void set_attn_attrs() {
   CUDA_TRY(cudaFuncSetAttribute(attention_split_kernel<MT, DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 AttnSmem<MT, DH>::SPLIT_TOTAL));
   CUDA_TRY(cudaFuncSetAttribute(attention_warp_kernel<MT, DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                AttnSmem<MT, DH>::WARP_TOTAL));
+                                AttnSmem<MT, DH, kWarpRing>::WARP_TOTAL));
   max_shared_carveout(attention_split_kernel<MT, DH>);
   max_shared_carveout(attention_warp_kernel<MT, DH>);
+  int n = 0;
+  CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, attention_warp_kernel<MT, DH>, kAttnThreads,
+                                                         AttnSmem<MT, DH, kWarpRing>::WARP_TOTAL));
+  g_attn_warp_ctas[MT == 4][DH == 64] = n > 0 ? n : 1;
 }
 
 void set_kernel_attrs() {
@@ -1003,11 +1010,18 @@ void enqueue_forward(gdit_handle* h, Profile& p, cudaStream_t s, Recorder* rec) 
     const int DH = h->cfg.head_dim;
     lx.timed(name, 0, 0, nullptr, [&] {
       if (warp_sched) {
-        const dim3 grid((aa.num_items + 3) / 4);
-        if (DH == 64 && MT == 2) launch_k(s, pdl, attention_warp_kernel<2, 64>, grid, block, AttnSmem<2, 64>::WARP_TOTAL, aa);
-        else if (DH == 64) launch_k(s, pdl, attention_warp_kernel<4, 64>, grid, block, AttnSmem<4, 64>::WARP_TOTAL, aa);
-        else if (MT == 2) launch_k(s, pdl, attention_warp_kernel<2, 32>, grid, block, AttnSmem<2, 32>::WARP_TOTAL, aa);
-        else launch_k(s, pdl, attention_warp_kernel<4, 32>, grid, block, AttnSmem<4, 32>::WARP_TOTAL, aa);
+        // persistent warps, every one with the same number of items: as many
+        // rounds as a full GPU of resident warps needs, then as few CTAs as
+        // still finish in that many rounds
+        const long long resident = 4LL * g_attn_warp_ctas[MT == 4][DH == 64] * h->num_sms;
+        const long long rounds = (aa.num_items + resident - 1) / resident;
+        const long long warps = (aa.num_items + rounds - 1) / rounds;
+        const dim3 grid((unsigned)((warps + 3) / 4));
+        constexpr int R = kWarpRing;
+        if (DH == 64 && MT == 2) launch_k(s, pdl, attention_warp_kernel<2, 64>, grid, block, AttnSmem<2, 64, R>::WARP_TOTAL, aa);
+        else if (DH == 64) launch_k(s, pdl, attention_warp_kernel<4, 64>, grid, block, AttnSmem<4, 64, R>::WARP_TOTAL, aa);
+        else if (MT == 2) launch_k(s, pdl, attention_warp_kernel<2, 32>, grid, block, AttnSmem<2, 32, R>::WARP_TOTAL, aa);
+        else launch_k(s, pdl, attention_warp_kernel<4, 32>, grid, block, AttnSmem<4, 32, R>::WARP_TOTAL, aa);
       } else {
         const dim3 grid(aa.num_items);
         if (DH == 64 && MT == 2) launch_k(s, pdl, attention_split_kernel<2, 64>, grid, block, AttnSmem<2, 64>::SPLIT_TOTAL, aa);

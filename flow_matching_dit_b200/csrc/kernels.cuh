@@ -187,10 +187,22 @@ __global__ void __launch_bounds__(256)
     layernorm_kernel(float* h, int rows, const float* p0, const float* p1, int mode, float eps,
                      __nv_bfloat16* u, const float* restore, int period) {
   constexpr int D = 128 * VEC;
-  pdl_wait();
-  pdl_launch_dependents();
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
+  // the modulation vectors are tables no earlier kernel writes: fetched
+  // before waiting for the previous kernel, so their latency overlaps its tail
+  // (up to D = 1024; wider rows would not fit the registers)
+  constexpr bool kEarly = VEC <= 8;
+  float4 pa[kEarly ? VEC : 1], pb[kEarly ? VEC : 1];
+  if constexpr (kEarly) {
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) {
+      pa[i] = __ldg(reinterpret_cast<const float4*>(p0) + lane + 32 * i);
+      pb[i] = __ldg(reinterpret_cast<const float4*>(p1) + lane + 32 * i);
+    }
+  }
+  pdl_wait();
+  pdl_launch_dependents();
   if (row >= rows) return;
   float4 x[VEC];
   float* hr = h + (long long)row * D;
@@ -221,8 +233,14 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
   for (int i = 0; i < VEC; ++i) {
     const int c4 = lane + 32 * i;
-    const float4 a = reinterpret_cast<const float4*>(p0)[c4];
-    const float4 b = reinterpret_cast<const float4*>(p1)[c4];
+    float4 a, b;
+    if constexpr (kEarly) {
+      a = pa[i];
+      b = pb[i];
+    } else {
+      a = __ldg(reinterpret_cast<const float4*>(p0) + c4);
+      b = __ldg(reinterpret_cast<const float4*>(p1) + c4);
+    }
     float4 y;
     y.x = (x[i].x - mean) * rstd;
     y.y = (x[i].y - mean) * rstd;
