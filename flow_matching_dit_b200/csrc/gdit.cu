@@ -786,6 +786,8 @@ bool small_loop_fits(const gdit_config& c, int N, int num_sms) {
     if (K % 16 != 0 || (K > kSmallKC && K % kSmallKC != 0)) return false;
     if ((long long)N * (K + 8) * 2 > kSmXBytes) return false;
   }
+  // self layers: the attention output rows and the QKV rows share the X area
+  if ((((long long)N * (D + 8) * 2 + 127) & ~127LL) + (long long)N * (3 * D + 8) * 2 > kSmXBytes) return false;
   for (long long n_out : {A, D, 3 * D, F}) {
     if (n_out % kSmallUF != 0) return false;
     if ((n_out / kSmallUF + num_sms - 1) / num_sms > kSmallMaxUnits) return false;
@@ -942,7 +944,7 @@ std::unique_ptr<Profile> build_profile(gdit_handle* h, int B, int S, int K, int 
     sp.counters = h->phase_counters;
     sp.phases = h->phase_table;
     sp.err = h->status;
-    p->small_phases = (5 * L + 6) * K;
+    p->small_phases = small_phases_per_step(L) * K;
     if (p->small_phases > kSmallMaxPhases) throw GditError(GDIT_EINVAL, "too many phases for the single-sample loop");
     p->small_plan = h->dalloc<SmallPlan>(1);
     CUDA_TRY(cudaMemcpy(p->small_plan, &sp, sizeof(sp), cudaMemcpyHostToDevice));

@@ -48,11 +48,12 @@ constexpr int kSmallKC = 1024;                           // widest weight chunk 
 constexpr int kSmallUF = 8;                              // output features per unit
 constexpr int kSmallMaxUnits = 4;                        // units of one CTA in one phase
 constexpr int kSmallSlots = 5;                           // weight chunks resident at once
+constexpr int kSmallPairPhases = 9;                      // phases of a (cross, self) layer pair
 constexpr int kSlotRow = kSmallKC + 8;                   // padded slot row (elements): conflict-free ldmatrix
 constexpr int kSlotBytes = kSmallUF * kSlotRow * 2;
 
 // dynamic shared memory (bytes)
-constexpr int kSmXBytes = 139776;                        // X rows / LN staging / attention / reduction
+constexpr int kSmXBytes = 140800;                        // X rows / LN / attention / QKV rows / reduction
 constexpr int kSmLnStage = kSmXBytes / 2;                // f32 h rows staged for LN (upper half)
 constexpr int kSmLnStageBytes = kSmXBytes - kSmLnStage;
 constexpr int kSmLnParams = kSmLnStage - 2 * kSmallMaxD * 4;   // LN modulation vectors p0, p1 (f32)
@@ -64,6 +65,10 @@ constexpr int kSmRedBytes = kSmallWarps * kSmallMaxUnits * kSmallMaxTok * kSmall
 static_assert(kSmRedBytes <= kSmXBytes, "reduction buffer fits the X area");
 static_assert(kSmallMaxUnits <= kSmallSlots, "one K-chunk of every unit of a phase is resident at once");
 static_assert(kSmallSmem <= 227 * 1024 - 1024, "shared memory budget");
+
+// 3 encoder GEMMs, 9 phases per (cross, self) layer pair, norm_out + proj_out
+// and the 2 decoder GEMMs (the layer count is even)
+__host__ __device__ constexpr int small_phases_per_step(int L) { return kSmallPairPhases * (L / 2) + 6; }
 
 struct SmallLayer {
   const __nv_bfloat16* wq;   // [nq, D]: Q (cross) or Q|K|V (self)
@@ -109,7 +114,7 @@ struct SmallGemm {
   const float* bias;         // [N] or nullptr
   const float* vec;          // swish: additive term [N] (bias included)
   int epi;
-  int x_mode;                // 0: X from global bf16; 1: LN(h) into shared memory
+  int x_mode;                // 0: X from global bf16; 1: LN(h) into shared memory; 2: self-attention of the QKV rows
   const __nv_bfloat16* X;
   int ldx;
   int ln_mode;               // 0: AdaLN (1 + p0) and p1; 1: affine p0, p1
@@ -190,8 +195,12 @@ __device__ __forceinline__ void small_describe(const SmallPlan& P, int c, int k,
     return;
   }
   const int j = idx - 3;
-  if (j < 5 * L) {
-    const int l = j / 5, part = j % 5;
+  if (j < kSmallPairPhases * (L / 2)) {
+    // a (cross, self) layer pair: Q, attention, O, FF1, FF2 of the cross layer,
+    // then QKV, attention fused into O, FF1, FF2 of the self layer
+    const int r = j % kSmallPairPhases;
+    const int l = 2 * (j / kSmallPairPhases) + (r >= 5 ? 1 : 0);
+    const int part = r < 5 ? r : (r == 5 ? 0 : r - 4);
     const SmallLayer& Ly = P.layers[l];
     const bool self = (l % 2) == 1;
     switch (part) {
@@ -219,9 +228,15 @@ __device__ __forceinline__ void small_describe(const SmallPlan& P, int c, int k,
         }
         break;
       }
-      case 2:                // h += O(attn) + b
+      case 2:                // h += O(attn) + b; self layers compute attn here, from the QKV rows
         g.W = Ly.wo; g.N = D; g.K = D; g.bias = Ly.bo; g.epi = EPI_RESID_F32; g.X = P.o; g.ldx = D;
         g.out = P.h; g.ldo = D;
+        if (self) {
+          g.x_mode = 2;
+          AttnArgs& a = ph.a;
+          a.q = P.qkv; a.q_ld = 3 * D; a.k = P.qkv + D; a.v = P.qkv + 2 * D; a.kv_ld = 3 * D;
+          a.n_tok = N; a.num_heads = P.nh; a.num_items = P.nh; a.scale_log2 = P.scale_log2;
+        }
         break;
       case 3:                // f = GELU(LN3(h) W1^T + b1)
         g.W = Ly.wff1; g.N = P.F; g.K = D; g.bias = Ly.bff1; g.epi = EPI_GELU_BF16; g.x_mode = 1; g.ln_mode = 1;
@@ -233,7 +248,7 @@ __device__ __forceinline__ void small_describe(const SmallPlan& P, int c, int k,
     }
     return;
   }
-  const int t = j - 5 * L;
+  const int t = j - kSmallPairPhases * (L / 2);
   g.rows = H;
   if (t == 0) {              // y = AdaLN_out(h[1..H]) W_out^T + b  (the state row is not decoded)
     g.W = P.proj_w; g.N = D; g.K = D; g.bias = P.proj_b; g.epi = EPI_BF16; g.x_mode = 1; g.ln_mode = 0;
@@ -504,6 +519,135 @@ __device__ __forceinline__ void small_ln_rows(const SmallGemm& g, const SmallCtx
   }
 }
 
+// Self-attention of all heads from the phase's own copy of the QKV rows, for
+// the O projection that follows in the same phase.  The QKV rows (N tokens,
+// 3D wide) sit after the X rows in the X area; the output goes to the X rows.
+__device__ __forceinline__ int small_qkv_offset(int rows, int D) { return (rows * (D + 8) * 2 + 127) & ~127; }
+
+__device__ __forceinline__ void small_issue_qkv(const AttnArgs& a, int D, uint8_t* smem, uint64_t* xbar) {
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x >= 32) return;
+  const int rows = a.n_tok, qrow = 3 * D + 8;
+  if (lane == 0) {
+    fence_proxy_async_global();
+    fence_proxy_async_smem();
+    mbar_arrive_expect_tx(xbar, (uint32_t)(rows * 3 * D * 2));
+  }
+  __syncwarp();
+  uint8_t* dst = smem + small_qkv_offset(rows, D);
+  for (int r = lane; r < rows; r += 32)
+    bulk_g2s(dst + (size_t)r * qrow * 2, a.q + (size_t)r * a.q_ld, (uint32_t)(3 * D * 2), xbar);
+}
+
+// One warp per head (heads warp, warp + 8, ...), all N <= 32 keys at once, one
+// 16-query tile after the other: S = Q K^T (four 8-key tiles), softmax over
+// the valid keys (base 2), O = P V, rows divided by their sums.  Rows and keys
+// past N read the last token (finite values) and are masked or never stored.
+template <int DH>
+__device__ __forceinline__ void small_self_attention_dh(const AttnArgs& a, int D, uint8_t* smem) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, tig = lane & 3;
+  const int N = a.n_tok, qrow = 3 * D + 8, xrow = D + 8;
+  const __nv_bfloat16* qkv = reinterpret_cast<const __nv_bfloat16*>(smem + small_qkv_offset(N, D));
+  __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(smem);
+  for (int h = warp; h < a.num_heads; h += kSmallWarps) {
+    const __nv_bfloat16* Qh = qkv + h * DH;
+    const __nv_bfloat16* Kh = qkv + D + h * DH;
+    const __nv_bfloat16* Vh = qkv + 2 * D + h * DH;
+#pragma unroll 1
+    for (int mt = 0; mt * 16 < N; ++mt) {
+      float s[4][4];
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s[nt][e] = 0.0f;
+      const int qr = min(mt * 16 + (lane & 15), N - 1);
+#pragma unroll
+      for (int ks = 0; ks < DH / 16; ++ks) {
+        uint32_t a0, a1, a2, a3;
+        ldmatrix_x4(a0, a1, a2, a3, Qh + (size_t)qr * qrow + ks * 16 + (lane >> 4) * 8);
+        // K fragments: keys (lane & 7) + 8 (lane >> 4) of each 16-key pair, k half (lane >> 3) & 1
+#pragma unroll
+        for (int kp = 0; kp < 2; ++kp) {
+          const int key = min(kp * 16 + (lane & 7) + ((lane >> 4) << 3), N - 1);
+          uint32_t k0, k1, k2, k3;
+          ldmatrix_x4(k0, k1, k2, k3, Kh + (size_t)key * qrow + ks * 16 + ((lane >> 3) & 1) * 8);
+          mma_bf16_16816(s[2 * kp], a0, a1, a2, a3, k0, k1);
+          mma_bf16_16816(s[2 * kp + 1], a0, a1, a2, a3, k2, k3);
+        }
+      }
+      // softmax over keys 0..N-1 of each query row (a row's 32 keys: 4 tiles x 4 lanes x 2)
+      float inv[2];
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        float m = -INFINITY;
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int key = nt * 8 + tig * 2 + e;
+            const float x = key < N ? s[nt][hr * 2 + e] * a.scale_log2 : -INFINITY;
+            s[nt][hr * 2 + e] = x;
+            m = fmaxf(m, x);
+          }
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        float l = 0.0f;
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float p = exp2f(s[nt][hr * 2 + e] - m);
+            s[nt][hr * 2 + e] = p;
+            l += p;
+          }
+        l += __shfl_xor_sync(0xffffffffu, l, 1);
+        l += __shfl_xor_sync(0xffffffffu, l, 2);
+        inv[hr] = 1.0f / l;
+      }
+      // O = P V over the two 16-key chunks; V fragments by ldmatrix.trans
+      float o[DH / 8][4];
+#pragma unroll
+      for (int nd = 0; nd < DH / 8; ++nd)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[nd][e] = 0.0f;
+#pragma unroll
+      for (int kc = 0; kc < 2; ++kc) {
+        const uint32_t p0 = pack_bf16x2(s[2 * kc][0], s[2 * kc][1]);
+        const uint32_t p1 = pack_bf16x2(s[2 * kc][2], s[2 * kc][3]);
+        const uint32_t p2 = pack_bf16x2(s[2 * kc + 1][0], s[2 * kc + 1][1]);
+        const uint32_t p3 = pack_bf16x2(s[2 * kc + 1][2], s[2 * kc + 1][3]);
+        const int r = lane & 7, mtx = lane >> 3;   // matrices: (keys 0-7 | 8-15) x (dims nd | nd + 8)
+        const int key = min(kc * 16 + (mtx & 1) * 8 + r, N - 1);
+#pragma unroll
+        for (int nd2 = 0; nd2 < DH / 16; ++nd2) {
+          uint32_t vb0, vb1, vb2, vb3;
+          ldmatrix_x4_trans(vb0, vb1, vb2, vb3, Vh + (size_t)key * qrow + (nd2 * 2 + (mtx >> 1)) * 8);
+          mma_bf16_16816(o[nd2 * 2 + 0], p0, p1, p2, p3, vb0, vb1);
+          mma_bf16_16816(o[nd2 * 2 + 1], p0, p1, p2, p3, vb2, vb3);
+        }
+      }
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        const int row = mt * 16 + g + hr * 8;
+        if (row < N) {
+#pragma unroll
+          for (int nd = 0; nd < DH / 8; ++nd)
+            *reinterpret_cast<uint32_t*>(xs + (size_t)row * xrow + h * DH + nd * 8 + tig * 2) =
+                pack_bf16x2(o[nd][hr * 2] * inv[hr], o[nd][hr * 2 + 1] * inv[hr]);
+        }
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void small_self_attention(const AttnArgs& a, int D, uint8_t* smem) {
+  if (D / a.num_heads == 64)
+    small_self_attention_dh<64>(a, D, smem);
+  else
+    small_self_attention_dh<32>(a, D, smem);
+}
+
 __device__ __forceinline__ void small_epilogue(const SmallGemm& g, int n, int tok, float v, float bias,
                                                float hold) {
   if (g.epi == EPI_SWISH_VEC_BF16) {
@@ -541,8 +685,8 @@ __device__ __forceinline__ void small_epilogue(const SmallGemm& g, int n, int to
 // count sits in slot item % kSmallSlots, filled for the (item / kSmallSlots)-th
 // time; a phase's items go chunk by chunk (every unit's K-chunk 0, then 1 ...)
 // and every warp releases a slot after its last read of it.
-__device__ __forceinline__ bool small_gemm_phase(const SmallGemm& g, const SmallCtx& P, uint8_t* smem,
-                                                 SmallRing& R, uint32_t& item, uint64_t* xbar,
+__device__ __forceinline__ bool small_gemm_phase(const SmallGemm& g, const AttnArgs& att, const SmallCtx& P,
+                                                 uint8_t* smem, SmallRing& R, uint32_t& item, uint64_t* xbar,
                                                  uint32_t& xuse) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gr = lane >> 2, tig = lane & 3;
@@ -554,8 +698,14 @@ __device__ __forceinline__ bool small_gemm_phase(const SmallGemm& g, const Small
     // every thread waits for the activations itself: no barrier before the MMAs
     ok = mbar_wait(xbar, xuse & 1u, P.err);
     ++xuse;
-  } else {
+  } else if (g.x_mode == 1) {
     small_ln_rows(g, P, smem);
+    csync();
+  } else {
+    small_issue_qkv(att, g.K, smem, xbar);
+    ok = mbar_wait(xbar, xuse & 1u, P.err);
+    ++xuse;
+    if (ok) small_self_attention(att, g.K, smem);
     csync();
   }
   const int xrow = g.K + 8;
@@ -803,7 +953,7 @@ __global__ void small_describe_kernel(const SmallPlan* __restrict__ plan) {
   const SmallPlan& P = *plan;
   pdl_wait();
   pdl_launch_dependents();
-  const int per_step = 5 * P.L + 6;
+  const int per_step = small_phases_per_step(P.L);
   const int total = per_step * P.K;
   const int gp = blockIdx.x * blockDim.x + threadIdx.x;
   if (gp >= total) return;
@@ -833,7 +983,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1) small_loop_kernel(const Smal
   __shared__ int s_ok;
   __shared__ int s_fail;
   const SmallCtx P = {plan->err, plan->counters, plan->h, plan->eps, plan->phases, plan->vofs, plan->dh};
-  const int total = (5 * plan->L + 6) * plan->K;
+  const int total = small_phases_per_step(plan->L) * plan->K;
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSmallSlots; ++i) {
       mbar_init(&s_ring.full[i], 1);
@@ -865,7 +1015,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1) small_loop_kernel(const Smal
       ok = small_wait(P, gp - 1, prev_workers, &s_ok);
       if (ok) {
         if (cur.kind == 0) {
-          if (!small_gemm_phase(cur.g, P, smem, s_ring, item, &s_xbar, xuse)) s_fail = 1;
+          if (!small_gemm_phase(cur.g, cur.a, P, smem, s_ring, item, &s_xbar, xuse)) s_fail = 1;
           csync();
           ok = s_fail == 0;
         } else {
