@@ -139,6 +139,33 @@ def time_oracle(W, w, samples: int):
     return samples / dt, cores, dt
 
 
+# ------------------------------------------------------------------ replicas (one per GPU, no data-path collective)
+
+def ranks_from_env():
+    """(rank, world, local rank) as torchrun sets them; (0, 1, 0) without it."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest value of x over all ranks (every rank gets it).  Timings of
+    the replicas are reported as their maximum: the job is as slow as its
+    slowest replica."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, units_per_rank_step: int, steps: int, seconds: float) -> float:
+    """Units per second of the whole job: every rank processed
+    units_per_rank_step units in each of `steps` steps, within `seconds`."""
+    return world * units_per_rank_step * steps / seconds
+
+
 # ------------------------------------------------------------------ reference arm
 
 def run_reference(args, rank):
@@ -182,9 +209,7 @@ def run_reference(args, rank):
 
 def main():
     args = parse()
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = ranks_from_env()
     if args.impl == "reference":
         return run_reference(args, rank)
 
@@ -236,14 +261,10 @@ def main():
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     assert head.sync_status() == 0
     ms_per_step = ms / args.steps
-    value = world * w.batch * args.steps / (ms / 1e3)
+    value = whole_job_rate(world, w.batch, args.steps, ms / 1e3)
 
     # ---- B = 1 latency (device inputs, one call at a time)
     lat = None
@@ -284,13 +305,9 @@ def main():
         n_e2e = max(3, args.steps // 2)
         for _ in range(n_e2e):
             head.get_action_host(*hargs, num_steps=K, out=hout, stream=st)
-        sec = time.perf_counter() - t0
-        if world > 1:
-            t = torch.tensor([sec], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            sec = float(t.item())
+        sec = max_over_ranks(time.perf_counter() - t0, world, dev)
         h2d = sum(int(v.nbytes) for v in hargs)
-        e2e = {"value": world * w.batch * n_e2e / sec, "unit": UNIT, "h2d_bytes_per_step": h2d,
+        e2e = {"value": whole_job_rate(world, w.batch, n_e2e, sec), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": int(hout.nbytes), "steps": n_e2e,
                "api": "gdit_get_action_host (pinned host buffers, copies and sync inside)"}
 
