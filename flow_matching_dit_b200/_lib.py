@@ -65,6 +65,7 @@ _SIGS = {
                                      ctypes.POINTER(gdit_kernel_stat), _I]),
     "gdit_test_gemm": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "gdit_gemm_static_scratch": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "gdit_debug_wait_expiry": (_I, [_I, ctypes.c_ulonglong]),
 }
 
 _lock = threading.Lock()

@@ -1398,6 +1398,39 @@ int gdit_debug_routing(gdit_handle* h, int32_t* perm, int32_t* seg, int32_t* vof
   });
 }
 
+// One thread waits on an mbarrier that nothing arrives at, through the same
+// bounded wait every kernel uses, with a short limit.
+__global__ void wait_expiry_kernel(unsigned* status, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  mbar_wait(&bar, 0, status, limit_ns);
+}
+
+int gdit_debug_wait_expiry(int device, unsigned long long limit_ns) {
+  return guarded(nullptr, [&] {
+    REQUIRE(limit_ns >= 1000ull && limit_ns <= 1000000000ull, "limit_ns %llu outside [1 us, 1 s]", limit_ns);
+    int n = 0;
+    if (cudaGetDeviceCount(&n) != cudaSuccess || n == 0) throw GditError(GDIT_ENODEV, "no CUDA device");
+    REQUIRE(device >= 0 && device < n, "device %d of %d", device, n);
+    CUDA_TRY(cudaSetDevice(device));
+    unsigned* st = nullptr;
+    CUDA_TRY(cudaMalloc(&st, sizeof(unsigned)));
+    unsigned host = 0;
+    cudaError_t e = cudaMemset(st, 0, sizeof(unsigned));
+    if (e == cudaSuccess) {
+      wait_expiry_kernel<<<1, 32>>>(st, limit_ns);
+      e = cudaGetLastError();
+    }
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e == cudaSuccess) e = cudaMemcpy(&host, st, sizeof(unsigned), cudaMemcpyDeviceToHost);
+    cudaFree(st);
+    CUDA_TRY(e);
+    if (host & DEV_ERR_TIMEOUT) throw GditError(GDIT_ETIMEOUT, "the bounded wait expired and reported it");
+  });
+}
+
 int gdit_debug_kv(gdit_handle* h, int layer, float* k_out, float* v_out, int* total_valid) {
   if (!h) return GDIT_EINVAL;
   return guarded(h, [&] {

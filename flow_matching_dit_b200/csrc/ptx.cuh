@@ -86,9 +86,10 @@ constexpr unsigned long long kWaitPeekNs = 50000ull;
 constexpr uint32_t kWaitSleepNs = 1000000u;
 
 // Waits for the phase with the given parity to complete.  Returns false (and
-// sets DEV_ERR_TIMEOUT in *err) if it has not completed within kWaitTimeoutNs,
-// or soon after another wait has recorded a timeout in *err.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* err) {
+// sets DEV_ERR_TIMEOUT in *err) if it has not completed within limit_ns, or
+// soon after another wait has recorded a timeout in *err.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* err,
+                                          unsigned long long limit_ns = kWaitTimeoutNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   // suspended rather than spinning, so that waiting warps leave the issue
@@ -98,7 +99,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
     if (dt > kWaitPeekNs) {
       // once any wait of the call has timed out, every other wait gives up
       if (*reinterpret_cast<volatile unsigned*>(err) & DEV_ERR_TIMEOUT) return false;
-      if (dt > kWaitTimeoutNs) {
+      if (dt > limit_ns) {
         atomicOr(err, DEV_ERR_TIMEOUT);
         return false;
       }

@@ -197,6 +197,16 @@ int gdit_debug_routing(gdit_handle* h, int32_t* perm, int32_t* seg, int32_t* vof
  * order.  *total_valid receives the row count; pass NULL buffers to query it. */
 int gdit_debug_kv(gdit_handle* h, int layer, float* k_out, float* v_out, int* total_valid);
 
+/* Failure detection check: launches one thread on `device` that waits, through
+ * the bounded mbarrier wait every kernel of the library uses, on an mbarrier
+ * that nothing ever arrives at, with a limit of limit_ns nanoseconds (1 us to
+ * 1 s) instead of the kernels' 2 s.  No GPU fault or hang: the wait gives up,
+ * records the timeout in a status word, and the thread exits.  Returns
+ * GDIT_ETIMEOUT when the expiry was detected and reported (the expected
+ * outcome), GDIT_EINVAL for a bad limit or device, GDIT_ENODEV without a GPU.
+ * Allocates and frees one status word on the device; synchronous. */
+int gdit_debug_wait_expiry(int device, unsigned long long limit_ns);
+
 /* Per-kernel-class timing of one eager (graph-free) run of gdit_get_action
  * with the given device inputs, each launch bracketed by CUDA events on
  * cuda_stream.  Fills up to max_stats entries; returns the count (>= 0) or an

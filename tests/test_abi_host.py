@@ -132,3 +132,12 @@ def test_null_handle_calls_are_rejected(L):
     assert L.gdit_get_action(None, None, 0, None, None, None, None, 4, None, 1, 1, None) == _lib.GDIT_EINVAL
     assert L.gdit_sync_status(None) == _lib.GDIT_EINVAL
     L.gdit_destroy(None)
+
+
+def test_wait_expiry_check_validates_on_host(L):
+    from flow_matching_dit_b200._lib import GDIT_EINVAL, GDIT_ENODEV
+    assert L.gdit_debug_wait_expiry(0, 10) == GDIT_EINVAL              # below 1 us
+    assert L.gdit_debug_wait_expiry(0, 5_000_000_000) == GDIT_EINVAL   # above 1 s
+    import torch
+    if not torch.cuda.is_available():
+        assert L.gdit_debug_wait_expiry(0, 1_000_000) == GDIT_ENODEV

@@ -319,3 +319,20 @@ def test_tma_store_epilogue_is_bitwise_equal_to_thread_stores(full_weights):
     with ActionHead(w.geom, full_weights, max_batch=32, max_seq=600, flags=GDIT_FLAG_NO_TMA_STORE) as b:
         y, _ = run_gpu(b, inp, w.num_steps)
     np.testing.assert_array_equal(x, y)
+
+
+def test_bounded_wait_expiry_is_reported_and_the_device_stays_usable(head_tiny, tiny_weights):
+    """A wait on an mbarrier that nothing arrives at, through the library's
+    bounded wait with a 1 ms limit: it gives up, reports GDIT_ETIMEOUT, and the
+    next call on the same device runs normally."""
+    import time
+    from flow_matching_dit_b200 import debug_wait_expiry
+    from flow_matching_dit_b200._lib import GDIT_ETIMEOUT
+    t0 = time.perf_counter()
+    assert debug_wait_expiry(0, 1_000_000) == GDIT_ETIMEOUT
+    assert time.perf_counter() - t0 >= 1e-3
+    w = synth.workload("tiny", fixed_ids=(1,))
+    inp = synth.make_inputs(w, seed=29)
+    gpu, st = run_gpu(head_tiny, inp, 4)
+    assert st == 0
+    assert_parity(gpu, run_oracle(tiny_weights, w.geom, inp, 4), inp["init_noise"], "after a wait expiry")
