@@ -202,11 +202,13 @@ __device__ __forceinline__ void attn_stream_chunks(const AttnArgs& a, int h, int
       }
     }
 
-    // online softmax (base 2); masked keys get -inf
+    // online softmax (base 2); masked keys get -inf.  Row groups of 8 with no
+    // query (past n_tok: zero Q rows, never stored) are skipped.
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
 #pragma unroll
       for (int hr = 0; hr < 2; ++hr) {   // hr 0: row g, hr 1: row g + 8
+        if (mt * 16 + hr * 8 >= a.n_tok) continue;
         float x[4];
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
