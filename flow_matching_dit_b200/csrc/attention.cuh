@@ -74,6 +74,12 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ void ldmatrix_x4(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3, const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(smem_u32(p)));
+}
+
 __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3,
                                                   const void* p) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
@@ -183,20 +189,16 @@ __device__ __forceinline__ void attn_stream_chunks(const AttnArgs& a, int h, int
         for (int j = 0; j < 4; ++j) s[mt][nt][j] = 0.0f;
 #pragma unroll
     for (int ks = 0; ks < DH / 16; ++ks) {
+      // K fragments of both 8-key tiles in one ldmatrix: lanes 0-7 keys 0-7
+      // (k 0-7), 8-15 keys 0-7 (k 8-15), 16-23 keys 8-15 (k 0-7), 24-31 keys 8-15 (k 8-15)
       uint32_t kb[2][2];
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const __nv_bfloat16* kr = sk + (nt * 8 + g) * ROW + ks * 16 + tig * 2;
-        kb[nt][0] = *reinterpret_cast<const uint32_t*>(kr);
-        kb[nt][1] = *reinterpret_cast<const uint32_t*>(kr + 8);
-      }
+      ldmatrix_x4(kb[0][0], kb[0][1], kb[1][0], kb[1][1],
+                  sk + ((lane & 7) + ((lane >> 4) << 3)) * ROW + ks * 16 + ((lane >> 3) & 1) * 8);
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
-        const __nv_bfloat16* qr = sQ + (mt * 16 + g) * ROW + ks * 16 + tig * 2;
-        const uint32_t a0 = *reinterpret_cast<const uint32_t*>(qr);
-        const uint32_t a1 = *reinterpret_cast<const uint32_t*>(qr + 8 * ROW);
-        const uint32_t a2 = *reinterpret_cast<const uint32_t*>(qr + 8);
-        const uint32_t a3 = *reinterpret_cast<const uint32_t*>(qr + 8 * ROW + 8);
+        // Q fragments: lane supplies row (lane & 15) of the tile, k half (lane >> 4)
+        uint32_t a0, a1, a2, a3;
+        ldmatrix_x4(a0, a1, a2, a3, sQ + (mt * 16 + (lane & 15)) * ROW + ks * 16 + (lane >> 4) * 8);
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) mma_bf16_16816(s[mt][nt], a0, a1, a2, a3, kb[nt][0], kb[nt][1]);
       }
