@@ -65,6 +65,15 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
+// 2^x by the PTX ex2.approx instruction (one special-function op; relative
+// error of a few ulp, far below bf16 resolution).  Arguments here are <= 0
+// (scores minus their running maximum); -inf gives 0.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -143,19 +152,32 @@ __device__ __forceinline__ void attn_stream_chunks(const AttnArgs& a, int h, int
   const __nv_bfloat16* kbase = a.k + h * a.kv_head_stride;
   const __nv_bfloat16* vbase = a.v + h * a.kv_head_stride;
 
-  // each lane copies DH/16 x 16 bytes of K and of V per chunk
+  // each lane copies DH/16 x 16 bytes of K and of V per chunk: piece i is row
+  // r0 + i * RSTEP, column c (fixed per lane); full chunks skip the per-row
+  // validity test
+  constexpr int RSTEP = 32 / PIECES;
+  const int r0 = lane / PIECES, c = (lane % PIECES) * 8;
   auto issue = [&](int chunk, int slot) {
     __nv_bfloat16* dk = ring + slot * 2 * SM::CHUNK_ELEMS;
     __nv_bfloat16* dv = dk + SM::CHUNK_ELEMS;
+    if (chunk * 16 + 16 <= n_keys) {
+      const long long off = (long long)(k_begin + chunk * 16 + r0) * a.kv_ld + c;
+      const long long step = (long long)RSTEP * a.kv_ld;
 #pragma unroll
-    for (int i = 0; i < DH / 16; ++i) {
-      const int idx = lane + 32 * i;      // 16 rows x PIECES pieces
-      const int r = idx / PIECES, c = (idx % PIECES) * 8;
-      const int key = chunk * 16 + r;
-      const bool valid = key < n_keys;
-      const long long row = (long long)(k_begin + (valid ? key : 0));
-      cp_async16(dk + r * ROW + c, kbase + row * a.kv_ld + c, valid);
-      cp_async16(dv + r * ROW + c, vbase + row * a.kv_ld + c, valid);
+      for (int i = 0; i < DH / 16; ++i) {
+        cp_async16(dk + (r0 + i * RSTEP) * ROW + c, kbase + off + i * step, true);
+        cp_async16(dv + (r0 + i * RSTEP) * ROW + c, vbase + off + i * step, true);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < DH / 16; ++i) {
+        const int r = r0 + i * RSTEP;
+        const int key = chunk * 16 + r;
+        const bool valid = key < n_keys;
+        const long long row = (long long)(k_begin + (valid ? key : 0));
+        cp_async16(dk + r * ROW + c, kbase + row * a.kv_ld + c, valid);
+        cp_async16(dv + r * ROW + c, vbase + row * a.kv_ld + c, valid);
+      }
     }
   };
 
@@ -224,11 +246,11 @@ __device__ __forceinline__ void attn_stream_chunks(const AttnArgs& a, int h, int
         cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 2));
         const float m_old = mrow[mt][hr];
         const float m_new = fmaxf(m_old, cm);
-        const float alpha = (m_new == -INFINITY) ? 1.0f : exp2f(m_old - m_new);
+        const float alpha = (m_new == -INFINITY) ? 1.0f : ex2_approx(m_old - m_new);
         float psum = 0.0f;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const float p = (m_new == -INFINITY) ? 0.0f : exp2f(x[j] - m_new);
+          const float p = (m_new == -INFINITY) ? 0.0f : ex2_approx(x[j] - m_new);
           x[j] = p;
           psum += p;
         }
