@@ -781,7 +781,7 @@ GemmOp plan_gemm(gdit_handle* h, const void* A, long long a_rows, int K, const v
 bool small_loop_fits(const gdit_config& c, int N, int num_sms) {
   const long long D = c.hidden, F = c.mlp_hidden, A = c.action_dim;
   if (N > kSmallMaxTok || D > kSmallMaxD || c.num_layers > kSmallMaxLayers || c.num_heads > num_sms) return false;
-  if ((long long)N * D * 4 > kSmLnStageBytes || (long long)N * (D + 8) * 2 > kSmLnParams) return false;
+  if ((long long)N * (D + 8) * 2 > kSmLnScratch) return false;   // LN output rows below the LN scratch
   for (long long K : {A, D, F}) {
     if (K % 16 != 0 || (K > kSmallKC && K % kSmallKC != 0)) return false;
     if ((long long)N * (K + 8) * 2 > kSmXBytes) return false;

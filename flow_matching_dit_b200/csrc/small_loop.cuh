@@ -22,8 +22,10 @@
 //     among themselves (bf16 mma.sync m16n8k16: tokens as the A operand,
 //     weight rows as B), reduce through shared memory and run the epilogue
 //     (bias, GELU / ReLU / swish, residual add, Euler update);
-//   * an attention phase runs one head per CTA (the streaming routine of the
-//     attention kernels, keys split over the 8 warps).
+//   * a cross-attention phase runs one head per CTA (the streaming routine of
+//     the attention kernels, keys split over the 8 warps); self-attention (17
+//     keys) is computed inside the self layer's O phase by every CTA of it,
+//     from its own copy of the QKV rows, so that phase needs no X load.
 //
 // Phases are ordered by arrival counters in global memory: the CTAs that work
 // in phase p wait until every CTA that worked in phase p-1 has arrived (each
@@ -54,9 +56,8 @@ constexpr int kSlotBytes = kSmallUF * kSlotRow * 2;
 
 // dynamic shared memory (bytes)
 constexpr int kSmXBytes = 140800;                        // X rows / LN / attention / QKV rows / reduction
-constexpr int kSmLnStage = kSmXBytes / 2;                // f32 h rows staged for LN (upper half)
-constexpr int kSmLnStageBytes = kSmXBytes - kSmLnStage;
-constexpr int kSmLnParams = kSmLnStage - 2 * kSmallMaxD * 4;   // LN modulation vectors p0, p1 (f32)
+constexpr int kSmLnScratchBytes = 4096;                  // LN row sums across warps, at the end of the X area
+constexpr int kSmLnScratch = kSmXBytes - kSmLnScratchBytes;
 constexpr int kSmRing = kSmXBytes;                       // weight slots
 constexpr int kSmHold = kSmRing + kSmallSlots * kSlotBytes;                       // [unit][tok][8] f32 old values
 constexpr int kSmBias = kSmHold + kSmallMaxUnits * kSmallMaxTok * kSmallUF * 4;  // [unit][8] f32
@@ -165,8 +166,8 @@ struct alignas(16) SmallPhase {
   AttnArgs a;
 };
 
-// Phase `idx` of Euler step k (per step: 3 action-encoder GEMMs, 5 phases per
-// DiT block, norm_out + proj_out, 2 decoder GEMMs).
+// Phase `idx` of Euler step k (per step: 3 action-encoder GEMMs, 9 phases per
+// (cross, self) block pair, norm_out + proj_out, 2 decoder GEMMs).
 __device__ __forceinline__ void small_describe(const SmallPlan& P, int c, int k, int idx, SmallPhase& ph) {
   const int D = P.D, H = P.H, N = P.N, A = P.A, C = P.C, L = P.L;
   memset(&ph, 0, sizeof(ph));
@@ -447,7 +448,8 @@ __device__ __forceinline__ void small_ln_rows(const SmallGemm& g, const SmallCtx
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int D = g.K, d4 = D / 4, xrow = D + 8;
   const bool has = tid < d4;
-  float* part = reinterpret_cast<float*>(smem + kSmLnStage);   // [warp][row][2]
+  static_assert((kSmallWarps * G * 2 + G * 2) * 4 <= kSmLnScratchBytes, "LN scratch");
+  float* part = reinterpret_cast<float*>(smem + kSmLnScratch);   // [warp][row][2]
   float* stat = part + kSmallWarps * G * 2;                     // [row][2]
   __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(smem);
   const float4 zero = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
