@@ -189,18 +189,15 @@ __global__ void __launch_bounds__(256)
   constexpr int D = 128 * VEC;
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  // the modulation vectors are tables no earlier kernel writes: fetched
-  // before waiting for the previous kernel, so their latency overlaps its tail
-  // (up to D = 1024; wider rows would not fit the registers)
-  constexpr bool kEarly = VEC <= 8;
-  float4 pa[kEarly ? VEC : 1], pb[kEarly ? VEC : 1];
-  if constexpr (kEarly) {
-#pragma unroll
-    for (int i = 0; i < VEC; ++i) {
-      pa[i] = __ldg(reinterpret_cast<const float4*>(p0) + lane + 32 * i);
-      pb[i] = __ldg(reinterpret_cast<const float4*>(p1) + lane + 32 * i);
-    }
+  // The modulation vectors are tables no earlier kernel writes: staged once
+  // per CTA in shared memory before waiting for the previous kernel, so their
+  // latency overlaps its tail (and they cost no registers: more CTAs per SM).
+  __shared__ float4 sp[2][D / 4];
+  for (int i = threadIdx.x; i < D / 4; i += blockDim.x) {
+    sp[0][i] = __ldg(reinterpret_cast<const float4*>(p0) + i);
+    sp[1][i] = __ldg(reinterpret_cast<const float4*>(p1) + i);
   }
+  __syncthreads();
   pdl_wait();
   pdl_launch_dependents();
   if (row >= rows) return;
@@ -233,14 +230,7 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
   for (int i = 0; i < VEC; ++i) {
     const int c4 = lane + 32 * i;
-    float4 a, b;
-    if constexpr (kEarly) {
-      a = pa[i];
-      b = pb[i];
-    } else {
-      a = __ldg(reinterpret_cast<const float4*>(p0) + c4);
-      b = __ldg(reinterpret_cast<const float4*>(p1) + c4);
-    }
+    const float4 a = sp[0][c4], b = sp[1][c4];
     float4 y;
     y.x = (x[i].x - mean) * rstd;
     y.y = (x[i].y - mean) * rstd;
