@@ -312,12 +312,30 @@ def velocity(m: Model, x: np.ndarray, td: float, state_feat: np.ndarray,
     return v[state_feat.shape[0]:]
 
 
-def prepare_sample(m: Model, feats: np.ndarray, mask: np.ndarray, state: np.ndarray, c: int):
+def cross_key_mask(layer: int, mask: np.ndarray, image_mask, n: int) -> np.ndarray:
+    """The backbone tokens cross layer `layer` attends to ([ARCH] "AlternateVLDiT
+    variant").  Without the image/text split (n == 0, the task's workloads) it
+    is every valid token (mask == 1).  With it, the page builds
+    image = image_mask & mask and text = ~image_mask & mask once, and a cross
+    block with index idx uses text when idx % (2 n) == 0, else image.
+    READING: image_mask None means no token is an image token."""
+    valid = np.asarray(mask).astype(bool)
+    if n == 0:
+        return valid
+    img = np.zeros_like(valid) if image_mask is None else np.asarray(image_mask).astype(bool)
+    if layer % (2 * n) == 0:
+        return (~img) & valid
+    return img & valid
+
+
+def prepare_sample(m: Model, feats: np.ndarray, mask: np.ndarray, state: np.ndarray, c: int,
+                   image_mask=None, n: int = 0):
     """Per-sample quantities that do not change across Euler steps: the state
-    features and every cross layer's K/V over the valid tokens (mask == 1,
-    [ARCH] backbone forward: attention_mask == 1)."""
-    valid = to_f64(feats)[np.asarray(mask).astype(bool)]
-    kvs = {layer: cross_kv(m, layer, valid) for layer in range(0, m.g.num_layers, 2)}
+    features and every cross layer's K/V over the tokens it attends to
+    (``cross_key_mask``; [ARCH] backbone forward: attention_mask == 1)."""
+    f = to_f64(feats)
+    kvs = {layer: cross_kv(m, layer, f[cross_key_mask(layer, mask, image_mask, n)])
+           for layer in range(0, m.g.num_layers, 2)}
     s = state_encoder(m, to_f64(state).reshape(-1, m.g.state_dim), c)
     return s, kvs
 
@@ -325,14 +343,16 @@ def prepare_sample(m: Model, feats: np.ndarray, mask: np.ndarray, state: np.ndar
 def get_action(weights: Dict[str, np.ndarray], geom, backbone_features, vl_mask, state,
                embodiment_id, init_noise, num_steps: int,
                samples: Optional[Sequence[int]] = None,
-               model: Optional[Model] = None) -> np.ndarray:
+               model: Optional[Model] = None, image_mask=None) -> np.ndarray:
     """Flow-matching Euler inference ([ARCH] "Inference (denoising)").
 
     x = init_noise; for k = 0..K-1: x = x + dt * v(x, t_k); returns x [B, H, A]
     (float64).  ``samples`` restricts the run to those batch rows (samples are
     independent), returned in that order.  ``init_noise`` is an input, as in the
     request's optional noise field ([WS1] "Prepare a request": a fixed tensor
-    gives deterministic regression checks).
+    gives deterministic regression checks).  ``image_mask`` [B, S] marks image
+    tokens for the image/text split of the cross layers, which is on when
+    ``geom.attend_text_every_n_blocks`` > 0 (``cross_key_mask``).
     """
     m = model if model is not None else Model(weights, geom)
     ids = np.asarray(embodiment_id).reshape(-1)
@@ -343,7 +363,9 @@ def get_action(weights: Dict[str, np.ndarray], geom, backbone_features, vl_mask,
         c = int(ids[b])
         if not 0 <= c < geom.num_embodiments:
             raise ValueError(f"embodiment_id {c} out of range")
-        s, kvs = prepare_sample(m, backbone_features[b], vl_mask[b], state[b], c)
+        n = int(getattr(geom, "attend_text_every_n_blocks", 0))
+        s, kvs = prepare_sample(m, backbone_features[b], vl_mask[b], state[b], c,
+                                None if image_mask is None else image_mask[b], n)
         x = to_f64(init_noise[b]).copy()
         for td in tds:
             x = x + dt * velocity(m, x, td, s, kvs, c)

@@ -33,7 +33,7 @@ from typing import Dict, List, Optional, Tuple
 import numpy as np
 
 __all__ = [
-    "Geometry", "Workload", "GEOM_FULL", "GEOM_TINY", "WORKLOADS", "workload",
+    "Geometry", "Workload", "GEOM_FULL", "GEOM_TINY", "WORKLOADS", "workload", "make_image_mask",
     "splitmix64_stream", "uniform53", "normal", "randint", "tensor_seed",
     "f32_to_bf16_bits", "bf16_bits_to_f32", "weight_shapes", "make_weights",
     "make_inputs",
@@ -169,6 +169,7 @@ class Geometry:
     num_timestep_buckets: int = 1000
     ln_eps: float = 1e-5
     weight_dtype: str = "bf16"      # "bf16" -> uint16 bit patterns, "f32" -> float32
+    attend_text_every_n_blocks: int = 0   # 0: every cross layer attends to all valid tokens
 
 
 GEOM_FULL = Geometry()
@@ -286,6 +287,19 @@ def make_weights(g: Geometry, seed: int = 0) -> Dict[str, np.ndarray]:
 # --------------------------------------------------------------------------
 # per-call inputs
 # --------------------------------------------------------------------------
+
+def make_image_mask(w: Workload, seed: int = 1, batch: Optional[int] = None) -> np.ndarray:
+    """image_mask [B,S] uint8 (1 = image token) for the image/text split of the
+    cross layers: sample b's first n_b backbone tokens are image tokens, n_b
+    uniform in 0..S (image tokens lead a VLM prompt; padding positions may be
+    marked too and must not matter)."""
+    B = w.batch if batch is None else batch
+    n = randint(tensor_seed(seed, "image_len"), B, 0, w.seq)
+    m = np.zeros((B, w.seq), dtype=np.uint8)
+    for b in range(B):
+        m[b, : n[b]] = 1
+    return m
+
 
 def make_inputs(w: Workload, seed: int = 1, batch: Optional[int] = None) -> Dict[str, np.ndarray]:
     """Inputs of one get_action call.

@@ -353,3 +353,97 @@ def test_action_encoder_applies_swish_to_w2(W):
     expect = torch.nn.functional.silu(torch.from_numpy(tau)).numpy()
     out = oracle.action_encoder(m, x, 250.0, 0)
     np.testing.assert_allclose(out, np.broadcast_to(expect, out.shape), rtol=1e-13, atol=1e-15)
+
+
+# ---------------------------------------------------------------- image/text split of the cross layers
+
+G4 = dataclasses.replace(G, num_layers=4)
+
+
+@pytest.fixture(scope="module")
+def W4():
+    return synth.make_weights(G4)
+
+
+def _split_inputs(seed=3):
+    w = dataclasses.replace(TINY, geom=G4, batch=2, seq=64, valid_min=40, fixed_ids=(0, 1))
+    inp = synth.make_inputs(w, seed=seed)
+    img = np.zeros_like(inp["vl_mask"])
+    img[:, :20] = 1   # the first 20 tokens of every sample are image tokens
+    return inp, img
+
+
+def test_split_layer_kinds_follow_the_page_rule():
+    """Cross block idx attends to text when idx % (2 n) == 0, else to images
+    ([ARCH] "AlternateVLDiT variant"): for 8 layers, blocks 0, 2, 4, 6 are
+    text/text/text/text (n = 1), text/image/text/image (n = 2) and
+    text/image/image/text (n = 3)."""
+    mask = np.ones(6, dtype=np.uint8)
+    img = np.array([1, 1, 1, 0, 0, 0], dtype=np.uint8)
+    text_keys, image_keys = [False] * 3 + [True] * 3, [True] * 3 + [False] * 3
+    expect = {1: "TTTT", 2: "TITI", 3: "TIIT"}
+    for n, kinds in expect.items():
+        for idx, kind in zip((0, 2, 4, 6), kinds):
+            got = list(oracle.cross_key_mask(idx, mask, img, n))
+            assert got == (text_keys if kind == "T" else image_keys), (n, idx)
+    # n = 0: no split, every valid token
+    assert list(oracle.cross_key_mask(2, mask, img, 0)) == [True] * 6
+    # padding never enters, image or not
+    pad = np.array([1, 1, 0, 1, 0, 1], dtype=np.uint8)
+    assert list(oracle.cross_key_mask(2, pad, img, 2)) == [True, True, False, False, False, False]
+
+
+def test_split_off_is_the_plain_model(W4):
+    inp, img = _split_inputs()
+    a = _run(W4, inp, g=G4)
+    b = _run(W4, inp, g=G4, image_mask=img)
+    np.testing.assert_array_equal(a, b)
+
+
+def test_split_n1_image_tokens_have_no_influence(W4):
+    """n = 1: every cross block attends to text, so image-token features do not
+    matter; text-token features do."""
+    g1 = dataclasses.replace(G4, attend_text_every_n_blocks=1)
+    inp, img = _split_inputs()
+    base = _run(W4, inp, g=g1, image_mask=img)
+    pert = dict(inp)
+    f = inp["backbone_features"].copy()
+    f[:, :20] += np.float32(3.0)        # image tokens only
+    pert["backbone_features"] = f
+    np.testing.assert_array_equal(_run(W4, pert, g=g1, image_mask=img), base)
+    f2 = inp["backbone_features"].copy()
+    f2[:, 25] += np.float32(3.0)        # one valid text token
+    pert["backbone_features"] = f2
+    assert np.abs(_run(W4, pert, g=g1, image_mask=img) - base).max() > 1e-6
+
+
+def test_split_n2_alternates_text_and_image(W4):
+    """n = 2 with 4 layers: block 0 attends to text, block 2 to images; each
+    kind of token then changes the output, and each block's K/V holds exactly
+    its kind of valid token."""
+    g2 = dataclasses.replace(G4, attend_text_every_n_blocks=2)
+    inp, img = _split_inputs()
+    m = oracle.Model(W4, g2)
+    sv = int(inp["vl_mask"][0].sum())
+    _, kvs = oracle.prepare_sample(m, inp["backbone_features"][0], inp["vl_mask"][0], inp["state"][0], 0,
+                                   img[0], 2)
+    assert kvs[0][0].shape[0] == sv - 20 and kvs[2][0].shape[0] == 20
+    base = _run(W4, inp, g=g2, image_mask=img)
+    for cols in (slice(0, 20), slice(25, 26)):
+        pert = dict(inp)
+        f = inp["backbone_features"].copy()
+        f[:, cols] += np.float32(3.0)
+        pert["backbone_features"] = f
+        assert np.abs(_run(W4, pert, g=g2, image_mask=img) - base).max() > 1e-6
+    # with no image token, block 2 has no key: its attention output is zero and
+    # only its bias reaches the residual, whatever the features
+    none = np.zeros_like(img)
+    r0 = _run(W4, inp, g=g2, image_mask=none)
+    zero_k = _copy(W4)
+    zero_k["blk2.k.w"][:] = 0
+    zero_k["blk2.v.w"][:] = 0
+    zero_k["blk2.o.w"][:] = 0
+    zero_k["blk2.k.b"][:] = 0
+    zero_k["blk2.v.b"][:] = 0
+    g0 = dataclasses.replace(G4, attend_text_every_n_blocks=0)
+    np.testing.assert_allclose(r0, _run(zero_k, inp, g=g0), rtol=1e-12, atol=1e-12)
