@@ -46,6 +46,7 @@ class ActionHead:
         cfg.max_backbone_seq = int(max_seq)
         cfg.flags = int(flags)
         cfg.device = int(device)
+        cfg.attend_text_every_n_blocks = int(getattr(geom, "attend_text_every_n_blocks", 0))
         self.cfg = cfg
         keep = []
         arr = (_lib.gdit_tensor * len(weights))()
@@ -90,13 +91,23 @@ class ActionHead:
             out = torch.empty_like(noise)
         return bb, B, S, out
 
-    def get_action(self, feats, mask, state, ids, noise, num_steps: int = 4, out=None, stream=None):
-        """Asynchronous on ``stream`` (default: torch's current stream)."""
+    def get_action(self, feats, mask, state, ids, noise, num_steps: int = 4, out=None, stream=None,
+                   image_mask=None):
+        """Asynchronous on ``stream`` (default: torch's current stream).  ``image_mask``
+        (uint8 [B, S] CUDA tensor, 1 = image token) feeds the image/text split of the
+        cross layers when the geometry's attend_text_every_n_blocks > 0."""
         import torch
         bb, B, S, out = self._args(feats, mask, state, ids, noise, out)
         st = stream if stream is not None else torch.cuda.current_stream().cuda_stream
-        check(_lib.gdit_get_action(self.h, _ptr(feats), bb, _ptr(mask), _ptr(state), _ptr(ids), _ptr(noise),
-                                   int(num_steps), _ptr(out), B, S, st), self.h)
+        if image_mask is None:
+            check(_lib.gdit_get_action(self.h, _ptr(feats), bb, _ptr(mask), _ptr(state), _ptr(ids), _ptr(noise),
+                                       int(num_steps), _ptr(out), B, S, st), self.h)
+            return out
+        if image_mask.dtype != torch.uint8 or not image_mask.is_contiguous() or not image_mask.is_cuda \
+                or tuple(image_mask.shape) != (B, S):
+            raise TypeError("image_mask must be a contiguous CUDA uint8 tensor [batch, seq]")
+        check(_lib.gdit_get_action_vl(self.h, _ptr(feats), bb, _ptr(mask), _ptr(image_mask), _ptr(state), _ptr(ids),
+                                      _ptr(noise), int(num_steps), _ptr(out), B, S, st), self.h)
         return out
 
     def get_action_host(self, feats: np.ndarray, mask: np.ndarray, state: np.ndarray, ids: np.ndarray,

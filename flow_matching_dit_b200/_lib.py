@@ -34,7 +34,8 @@ class gdit_config(ctypes.Structure):
         "num_layers", "hidden", "num_heads", "head_dim", "mlp_hidden", "backbone_dim",
         "action_dim", "state_dim", "action_horizon", "num_embodiments",
         "max_batch", "max_backbone_seq", "time_freq_dim", "num_timestep_buckets")] + [
-        ("ln_eps", ctypes.c_float), ("flags", ctypes.c_uint), ("device", ctypes.c_int)]
+        ("ln_eps", ctypes.c_float), ("flags", ctypes.c_uint), ("device", ctypes.c_int),
+        ("attend_text_every_n_blocks", ctypes.c_int)]
 
 
 class gdit_tensor(ctypes.Structure):
@@ -66,6 +67,7 @@ _SIGS = {
     "gdit_test_gemm": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "gdit_gemm_static_scratch": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "gdit_debug_wait_expiry": (_I, [_I, ctypes.c_ulonglong]),
+    "gdit_get_action_vl": (_I, [_P, _P, _I, _P, _P, _P, _P, _P, _I, _P, _I, _I, _P]),
 }
 
 _lock = threading.Lock()
@@ -117,6 +119,10 @@ def gdit_destroy(h):
 
 def gdit_get_action(*a):
     return lib().gdit_get_action(*a)
+
+
+def gdit_get_action_vl(*a):
+    return lib().gdit_get_action_vl(*a)
 
 
 def gdit_get_action_host(*a):

@@ -38,6 +38,8 @@ struct AttnArgs {
   __nv_bfloat16* out;
   long long out_ld;
   float scale_log2;     // log2(e) / sqrt(head_dim)
+  const uint8_t* kflag; // cross: image flag of each packed key (used when ksel >= 0)
+  int ksel;             // -1: every key; 0: keys with flag 0 (text); 1: flag 1 (image)
 };
 
 // MT: 16-row query tiles (queries padded to 16 * MT); DH: head dim (32 or 64).
@@ -198,6 +200,18 @@ __device__ __forceinline__ void attn_stream_chunks(const AttnArgs& a, int h, int
     }
     cp_async_wait<SM::RING - 1>();
     __syncwarp();
+    // the keys of this lane's score columns that the layer keeps (bit nt * 2 + j)
+    uint32_t keep = 0xFu;
+    if (a.ksel >= 0) {
+      keep = 0u;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int key = chunk * 16 + nt * 8 + tig * 2 + j;
+          if (key < n_keys && (int)__ldg(a.kflag + k_begin + key) == a.ksel) keep |= 1u << (nt * 2 + j);
+        }
+    }
     const __nv_bfloat16* sk = ring + (it % SM::RING) * 2 * SM::CHUNK_ELEMS;
     const __nv_bfloat16* sv = sk + SM::CHUNK_ELEMS;
 
@@ -239,7 +253,8 @@ __device__ __forceinline__ void attn_stream_chunks(const AttnArgs& a, int h, int
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
             const int key = chunk * 16 + nt * 8 + tig * 2 + j;
-            x[nt * 2 + j] = key < n_keys ? s[mt][nt][hr * 2 + j] * a.scale_log2 : -INFINITY;
+            x[nt * 2 + j] = (key < n_keys && ((keep >> (nt * 2 + j)) & 1u)) ? s[mt][nt][hr * 2 + j] * a.scale_log2
+                                                                             : -INFINITY;
           }
         float cm = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
         cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 1));

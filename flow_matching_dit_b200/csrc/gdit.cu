@@ -329,6 +329,7 @@ struct gdit_handle {
   std::vector<void*> allocs;
   DevModel w;
   __nv_bfloat16 *xp, *kv, *u, *qkv, *o, *f, *xb, *abf, *zbf, *ybf, *rbf, *sb, *s1;
+  uint8_t* kflag;           // image flag of each packed backbone token
   float *h, *x, *sfeat, *ws;
   int *perm, *seg, *vofs, *counters;
   int* phase_counters;      // per-phase arrival counters of the single-sample loop
@@ -389,6 +390,15 @@ void validate_config(const gdit_config& c) {
   REQUIRE(c.time_freq_dim >= 2 && c.time_freq_dim % 2 == 0, "time_freq_dim must be even and >= 2");
   REQUIRE(c.num_timestep_buckets >= 1, "num_timestep_buckets must be >= 1");
   REQUIRE(c.ln_eps > 0.0f, "ln_eps must be > 0");
+  REQUIRE(c.attend_text_every_n_blocks >= 0, "attend_text_every_n_blocks must be >= 0");
+}
+
+// Which keys cross layer `layer` attends to (AlternateVLDiT image/text split):
+// -1 every valid key (no split), 0 the text keys, 1 the image keys.
+int cross_key_sel(const gdit_config& c, int layer) {
+  const int n = c.attend_text_every_n_blocks;
+  if (n <= 0) return -1;
+  return layer % (2 * n) == 0 ? 0 : 1;
 }
 
 std::vector<WeightSpec> weight_specs(const gdit_config& c) {
@@ -614,6 +624,7 @@ void alloc_workspace(gdit_handle* h) {
   const int D = h->D, F = h->F, N = h->N, H = h->H, A = h->A;
   h->max_tok = Bm * Sm;
   h->xp = h->dalloc<__nv_bfloat16>((size_t)h->max_tok * h->Dvl);
+  h->kflag = h->dalloc<uint8_t>((size_t)h->max_tok);
   h->kv = h->dalloc<__nv_bfloat16>((size_t)h->Lc * h->max_tok * 2 * D);
   h->h = h->dalloc<float>((size_t)Bm * N * D);
   h->u = h->dalloc<__nv_bfloat16>((size_t)Bm * N * D);
@@ -931,7 +942,8 @@ std::unique_ptr<Profile> build_profile(gdit_handle* h, int B, int S, int K, int 
     sp.max_tok = h->max_tok;
     sp.h = h->h; sp.x = h->x; sp.xb = h->xb;
     sp.abf = h->abf; sp.zbf = h->zbf; sp.qkv = h->qkv; sp.o = h->o; sp.f = h->f; sp.ybf = h->ybf; sp.rbf = h->rbf;
-    sp.sfeat = h->sfeat; sp.seg = h->seg; sp.vofs = h->vofs;
+    sp.sfeat = h->sfeat; sp.seg = h->seg; sp.vofs = h->vofs; sp.kflag = h->kflag;
+    sp.text_every = h->cfg.attend_text_every_n_blocks;
     sp.ada = t.ada; sp.tw2 = t.tw2;
     sp.wa1t = m.wa1t; sp.wa2at = m.wa2at; sp.wa3t = m.wa3t; sp.wd1t = m.wd1t; sp.wd2t = m.wd2t; sp.proj_w = m.proj_w;
     sp.ba1 = m.ba1; sp.ba3 = m.ba3; sp.bd1 = m.bd1; sp.bd2 = m.bd2; sp.proj_b = m.proj_b;
@@ -1042,7 +1054,7 @@ void enqueue_forward(gdit_handle* h, Profile& p, cudaStream_t s, Recorder* rec) 
   });
   lx.timed("route_pack", 0, (double)B * S * Dvl * (p.bf16 ? 4 : 6), nullptr, [&] {
     launch_k(s, pdl, pack_features_kernel, dim3(B, (S + 31) / 32), dim3(kPackThreads), 0, (const IoPtrs*)h->io,
-             p.bf16, S, Dvl, (const int*)h->perm, (const int*)h->vofs, h->xp);
+             p.bf16, S, Dvl, (const int*)h->perm, (const int*)h->vofs, h->xp, h->kflag);
   });
   lx.timed("route_pack", 0, 0, nullptr, [&] {
     launch_k(s, pdl, gather_inputs_kernel, dim3(B), dim3(128), 0, (const IoPtrs*)h->io, B, H * A, h->Sd,
@@ -1102,6 +1114,8 @@ void enqueue_forward(gdit_handle* h, Profile& p, cudaStream_t s, Recorder* rec) 
       aa.out = h->o;
       aa.out_ld = D;
       aa.scale_log2 = scale_log2;
+      aa.kflag = h->kflag;
+      aa.ksel = l % 2 == 1 ? -1 : cross_key_sel(h->cfg, l);
       if (l % 2 == 1) {
         aa.q_ld = 3 * D;
         aa.k = h->qkv + D;
@@ -1178,11 +1192,12 @@ void check_call(gdit_handle* h, const void* feats, int bb_dtype, const void* mas
 }
 
 void run_call(gdit_handle* h, const void* feats, int bb_dtype, const uint8_t* mask, const float* state,
-              const int32_t* ids, const float* noise, int K, float* out, int B, int S, cudaStream_t s) {
+              const int32_t* ids, const float* noise, int K, float* out, int B, int S, cudaStream_t s,
+              const uint8_t* image_mask = nullptr) {
   CUDA_TRY(cudaSetDevice(h->cfg.device));
   compute_tables(h, K, s);
   Profile& p = get_profile(h, B, S, K, bb_dtype == GDIT_BF16, !h->strict);
-  IoPtrs io{feats, mask, state, ids, noise, out};
+  IoPtrs io{feats, mask, state, ids, noise, out, image_mask};
   set_io_kernel<<<1, 1, 0, s>>>(h->io, io);
   CUDA_TRY(cudaGetLastError());
   if (p.exec != nullptr)
@@ -1309,6 +1324,19 @@ int gdit_get_action(gdit_handle* h, const void* backbone_features, int bb_dtype,
                batch, seq);
     run_call(h, backbone_features, bb_dtype, vl_mask, state, embodiment_id, init_noise, num_steps, out_actions, batch,
              seq, (cudaStream_t)cuda_stream);
+  });
+}
+
+int gdit_get_action_vl(gdit_handle* h, const void* backbone_features, int bb_dtype, const uint8_t* vl_mask,
+                       const uint8_t* image_mask, const float* state, const int32_t* embodiment_id,
+                       const float* init_noise, int num_steps, float* out_actions, int batch, int seq,
+                       void* cuda_stream) {
+  if (!h) return GDIT_EINVAL;
+  return guarded(h, [&] {
+    check_call(h, backbone_features, bb_dtype, vl_mask, state, embodiment_id, init_noise, num_steps, out_actions,
+               batch, seq);
+    run_call(h, backbone_features, bb_dtype, vl_mask, state, embodiment_id, init_noise, num_steps, out_actions, batch,
+             seq, (cudaStream_t)cuda_stream, image_mask);
   });
 }
 

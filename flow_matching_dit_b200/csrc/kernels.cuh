@@ -17,6 +17,7 @@ struct IoPtrs {
   const int32_t* ids;
   const float* noise;
   float* out;
+  const uint8_t* image_mask;   // [B, S] 1 = image token, or nullptr (none)
 };
 
 __global__ void set_io_kernel(IoPtrs* dst, IoPtrs src) { *dst = src; }
@@ -91,7 +92,7 @@ constexpr int kPackThreads = 256;
 
 __global__ void __launch_bounds__(kPackThreads)
     pack_features_kernel(const IoPtrs* io, int bb_bf16, int S, int Dvl, const int* perm, const int* vofs,
-                         __nv_bfloat16* xp) {
+                         __nv_bfloat16* xp, uint8_t* kflag) {
   __shared__ int s_red[kPackThreads / 32];
   __shared__ int s_rows[32];
   __shared__ int s_n;
@@ -125,6 +126,10 @@ __global__ void __launch_bounds__(kPackThreads)
   __syncthreads();
   const int n = s_n;
   const long long dst0 = (long long)vofs[i] + s_before;
+  // image flag of every packed token (the image/text split of the cross layers)
+  if ((int)threadIdx.x < n)
+    kflag[dst0 + threadIdx.x] =
+        io->image_mask != nullptr ? (uint8_t)(io->image_mask[(long long)b * S + s_rows[threadIdx.x]] != 0) : 0;
   const int vec_per_row = Dvl / 8;            // 8 bf16 = 16 bytes
   for (int idx = threadIdx.x; idx < n * vec_per_row; idx += kPackThreads) {
     const int r = idx / vec_per_row;

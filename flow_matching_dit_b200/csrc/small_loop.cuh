@@ -97,6 +97,8 @@ struct SmallPlan {
   const float* sfeat;
   const int* seg;
   const int* vofs;
+  const uint8_t* kflag;      // image flag of each packed backbone token
+  int text_every;            // attend_text_every_n_blocks (0: no image/text split)
   // per-K tables: AdaLN [K][L+1][2D], timestep term of the action encoder's W2 [K][C][D]
   const float* ada;
   const float* tw2;
@@ -214,6 +216,9 @@ __device__ __forceinline__ void small_describe(const SmallPlan& P, int c, int k,
         a.out = P.o;
         a.out_ld = D;
         a.scale_log2 = P.scale_log2;
+        a.kflag = P.kflag;
+        // keys of this cross layer: every valid key, or the text (0) / image (1) ones
+        a.ksel = (self || P.text_every <= 0) ? -1 : (l % (2 * P.text_every) == 0 ? 0 : 1);
         if (self) {
           a.q = P.qkv; a.q_ld = 3 * D; a.k = P.qkv + D; a.v = P.qkv + 2 * D; a.kv_ld = 3 * D;
           a.kv_head_stride = P.dh; a.kofs = nullptr;
@@ -230,7 +235,7 @@ __device__ __forceinline__ void small_describe(const SmallPlan& P, int c, int k,
           g.x_mode = 2;
           AttnArgs& a = ph.a;
           a.q = P.qkv; a.q_ld = 3 * D; a.k = P.qkv + D; a.v = P.qkv + 2 * D; a.kv_ld = 3 * D;
-          a.n_tok = N; a.num_heads = P.nh; a.num_items = P.nh; a.scale_log2 = P.scale_log2;
+          a.n_tok = N; a.num_heads = P.nh; a.num_items = P.nh; a.scale_log2 = P.scale_log2; a.ksel = -1;
         }
         break;
       case 3:                // f = GELU(LN3(h) W1^T + b1)

@@ -88,6 +88,12 @@ typedef struct {
   float ln_eps;
   unsigned flags;           /* GDIT_FLAG_* */
   int device;               /* CUDA device ordinal */
+  /* AlternateVLDiT image/text split (Isaac-GR00T architecture page,
+   * "AlternateVLDiT variant"): 0 = every cross layer attends to all valid
+   * tokens; n >= 1 = cross block idx attends to the valid text tokens when
+   * idx % (2n) == 0, else to the valid image tokens (image_mask of
+   * gdit_get_action_vl; without it no token is an image token). */
+  int attend_text_every_n_blocks;
 } gdit_config;
 
 /* One named host weight tensor.  Names and shapes (D hidden, F mlp_hidden,
@@ -156,6 +162,17 @@ int gdit_get_action(gdit_handle* h, const void* backbone_features, int bb_dtype,
                     const uint8_t* vl_mask, const float* state, const int32_t* embodiment_id,
                     const float* init_noise, int num_steps, float* out_actions,
                     int batch, int seq, void* cuda_stream);
+
+/* gdit_get_action with the image/text split's image_mask: device uint8
+ * [batch, seq], 1 = image token (input_ids == image_token_index), used when
+ * the handle's attend_text_every_n_blocks > 0; NULL = no image token.  The
+ * cross layers' K/V are computed once over all valid tokens; each cross
+ * layer's attention keeps the keys of its kind (a sample with no key of that
+ * kind gets a zero cross-attention output). */
+int gdit_get_action_vl(gdit_handle* h, const void* backbone_features, int bb_dtype,
+                       const uint8_t* vl_mask, const uint8_t* image_mask, const float* state,
+                       const int32_t* embodiment_id, const float* init_noise, int num_steps,
+                       float* out_actions, int batch, int seq, void* cuda_stream);
 
 /* Same computation with HOST buffers (same shapes and meanings as above).
  * Copies the inputs to handle-owned device buffers, runs, copies out_actions

@@ -91,6 +91,7 @@ def _create(L, cfg, W):
     ("action_horizon", 64, "action_horizon"),
     ("num_embodiments", 65, "num_embodiments"),
     ("max_batch", 0, "max_batch"),
+    ("attend_text_every_n_blocks", -1, "attend_text_every_n_blocks"),
 ])
 def test_bad_config_rejected_on_host(L, tinyW, field, value, msg):
     cfg = _cfg(synth.GEOM_TINY, **{field: value})

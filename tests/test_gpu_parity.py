@@ -336,3 +336,37 @@ def test_bounded_wait_expiry_is_reported_and_the_device_stays_usable(head_tiny, 
     gpu, st = run_gpu(head_tiny, inp, 4)
     assert st == 0
     assert_parity(gpu, run_oracle(tiny_weights, w.geom, inp, 4), inp["init_noise"], "after a wait expiry")
+
+
+# ---------------------------------------------------------------- image/text split of the cross layers
+
+@pytest.mark.parametrize("n", [1, 2])
+# 1: the persistent single-sample loop; 3: per-layer kernels, split attention schedule;
+# 160 (x 4 heads >= 4 x SMs): per-layer kernels, warp attention schedule (rows sampled)
+@pytest.mark.parametrize("batch", [1, 3, 160])
+def test_image_text_split_matches_oracle(n, batch):
+    """AlternateVLDiT with attend_text_every_n_blocks = n on a 4-layer tiny DiT
+    (cross blocks 0 and 2): ragged valid lengths and seeded image masks; the
+    cross layers keep only their kind of key, as the oracle's per-layer masks."""
+    require_gpu()
+    import torch
+    from flow_matching_dit_b200 import ActionHead
+    g = dataclasses.replace(synth.GEOM_TINY, num_layers=4, attend_text_every_n_blocks=n)
+    W = synth.make_weights(g)
+    w = dataclasses.replace(synth.WORKLOADS["tiny"], geom=g, batch=batch, seq=64, valid_min=30,
+                            fixed_ids=(1, 0, 1)[:min(batch, 3)])
+    inp = synth.make_inputs(w, seed=31 + n)
+    img = synth.make_image_mask(w, seed=41 + n)
+    with ActionHead(g, W, max_batch=batch, max_seq=64) as head:
+        out = head.get_action(*to_dev(inp), num_steps=4, image_mask=torch.from_numpy(img).cuda())
+        st = head.sync_status()
+        gpu = out.cpu().numpy()
+        plain = head.get_action(*to_dev(inp), num_steps=4).cpu().numpy()   # no image mask: no image token
+    assert st == 0
+    rows = list(range(batch)) if batch <= 3 else [0, 77, batch - 1]
+    ref = oracle.get_action(W, g, inp["backbone_features"], inp["vl_mask"], inp["state"], inp["embodiment_id"],
+                            inp["init_noise"], 4, image_mask=img, samples=rows)
+    assert_parity(gpu[rows], ref, inp["init_noise"][rows], f"image/text split n={n} B={batch}")
+    ref0 = oracle.get_action(W, g, inp["backbone_features"], inp["vl_mask"], inp["state"], inp["embodiment_id"],
+                             inp["init_noise"], 4, samples=rows)
+    assert_parity(plain[rows], ref0, inp["init_noise"][rows], f"split on, no image mask, n={n} B={batch}")
