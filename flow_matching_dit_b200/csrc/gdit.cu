@@ -264,6 +264,8 @@ struct WeightSpec {
 struct DevModel {
   // bf16 matrices
   __nv_bfloat16 *t1w, *t2w, *ada_w, *wkv, *proj_w;
+  float* vlln_g = nullptr;   // optional vision-language layer norm (f32 [Dvl])
+  float* vlln_b = nullptr;
   std::vector<__nv_bfloat16*> wq;     // per layer: [3D, D] (self) or [D, D] (cross)
   std::vector<__nv_bfloat16*> wo, wff1, wff2;
   __nv_bfloat16 *ws1t, *ws2t, *wa1t, *wa2at, *wa2taut, *wa3t, *wd1t, *wd2t;
@@ -490,8 +492,20 @@ std::unordered_map<std::string, HostW> check_weights(const gdit_config& c, const
                                        have.c_str(), want.c_str()));
     }
   }
-  REQUIRE(got.size() == specs.size(), "%zu unknown weight name(s) given (expected exactly %zu tensors)",
-          got.size() - specs.size(), specs.size());
+  // optional: the vision-language layer norm of the backbone features
+  size_t optional = 0;
+  if (got.count("vlln.g") || got.count("vlln.b")) {
+    REQUIRE(got.count("vlln.g") && got.count("vlln.b"), "vlln.g and vlln.b must be given together");
+    for (const char* n : {"vlln.g", "vlln.b"}) {
+      const gdit_tensor* t = got.at(n).t;
+      REQUIRE(t->ndim == 1 && t->shape[0] == c.backbone_dim, "weight '%s' must have shape [%d]", n, c.backbone_dim);
+    }
+    REQUIRE(c.backbone_dim % 256 == 0 && c.backbone_dim <= 4096,
+            "vlln needs backbone_dim a multiple of 256 and <= 4096 (got %d)", c.backbone_dim);
+    optional = 2;
+  }
+  REQUIRE(got.size() == specs.size() + optional, "%zu unknown weight name(s) given (expected exactly %zu tensors)",
+          got.size() - specs.size() - optional, specs.size() + optional);
   return got;
 }
 
@@ -545,6 +559,10 @@ void upload_model(gdit_handle* h, const std::unordered_map<std::string, HostW>& 
   const int D = h->D, F = h->F, L = h->L, C = h->C, Dvl = h->Dvl, A = h->A, Sd = h->Sd;
   DevModel& m = h->w;
   auto get = [&](const std::string& n) -> const HostW& { return W.at(n); };
+  if (W.count("vlln.g")) {
+    m.vlln_g = up.vec(get("vlln.g"));
+    m.vlln_b = up.vec(get("vlln.b"));
+  }
   m.t1w = up.matrix(get("t_enc.l1.w"));
   m.t1b = up.vec(get("t_enc.l1.b"));
   m.t2w = up.matrix(get("t_enc.l2.w"));
@@ -1056,6 +1074,20 @@ void enqueue_forward(gdit_handle* h, Profile& p, cudaStream_t s, Recorder* rec) 
     launch_k(s, pdl, pack_features_kernel, dim3(B, (S + 31) / 32), dim3(kPackThreads), 0, (const IoPtrs*)h->io,
              p.bf16, S, Dvl, (const int*)h->perm, (const int*)h->vofs, h->xp, h->kflag);
   });
+  if (h->w.vlln_g != nullptr) {
+    lx.timed("vlln", 0, (double)B * S * Dvl * 4, nullptr, [&] {
+      const dim3 grid((unsigned)(((long long)B * S + 7) / 8));
+      const int* tot = (const int*)h->vofs + B;
+      const float e = h->cfg.ln_eps;
+      switch (Dvl / 256) {
+        case 1: launch_k(s, pdl, vlln_kernel<1>, grid, dim3(256), 0, h->xp, tot, h->w.vlln_g, h->w.vlln_b, e); break;
+        case 2: launch_k(s, pdl, vlln_kernel<2>, grid, dim3(256), 0, h->xp, tot, h->w.vlln_g, h->w.vlln_b, e); break;
+        case 4: launch_k(s, pdl, vlln_kernel<4>, grid, dim3(256), 0, h->xp, tot, h->w.vlln_g, h->w.vlln_b, e); break;
+        case 8: launch_k(s, pdl, vlln_kernel<8>, grid, dim3(256), 0, h->xp, tot, h->w.vlln_g, h->w.vlln_b, e); break;
+        default: launch_k(s, pdl, vlln_kernel<16>, grid, dim3(256), 0, h->xp, tot, h->w.vlln_g, h->w.vlln_b, e); break;
+      }
+    });
+  }
   lx.timed("route_pack", 0, 0, nullptr, [&] {
     launch_k(s, pdl, gather_inputs_kernel, dim3(B), dim3(128), 0, (const IoPtrs*)h->io, B, H * A, h->Sd,
              (const int*)h->perm, h->x, h->xb, h->sb);

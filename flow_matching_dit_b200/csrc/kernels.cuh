@@ -187,6 +187,59 @@ __global__ void scatter_out_kernel(const IoPtrs* io, int HA, const int* perm, co
 // If restore != nullptr, rows r with r % period == 0 (the state token of each
 // sample) are first reset from restore[r / period] and written back to h: the
 // state features re-enter every Euler step.
+// Vision-language layer norm of the packed backbone tokens, in place: one warp
+// per packed row of Dvl = 256 * VEC bf16 features, f32 mean and (two-pass)
+// variance in registers, y = (x - mean) * rstd * g + b rounded to bf16.  Rows
+// past the call's valid-token count (vofs[B], on the device) are left alone.
+template <int VEC>
+__global__ void __launch_bounds__(256)
+    vlln_kernel(__nv_bfloat16* xp, const int* total, const float* g, const float* b, float eps) {
+  constexpr int Dvl = 256 * VEC;
+  pdl_wait();
+  pdl_launch_dependents();
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= *total) return;
+  uint4* xr = reinterpret_cast<uint4*>(xp + row * Dvl);
+  float v[8 * VEC];
+#pragma unroll
+  for (int i = 0; i < VEC; ++i) {
+    const uint4 u = xr[lane + 32 * i];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+      v[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+    }
+  }
+  float s = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8 * VEC; ++i) s += v[i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  const float mean = s * (1.0f / Dvl);
+  float q = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8 * VEC; ++i) q += (v[i] - mean) * (v[i] - mean);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+  const float rstd = rsqrtf(q * (1.0f / Dvl) + eps);
+#pragma unroll
+  for (int i = 0; i < VEC; ++i) {
+    const int c0 = (lane + 32 * i) * 8;
+    const float4 g0 = __ldg(reinterpret_cast<const float4*>(g + c0)), g1 = __ldg(reinterpret_cast<const float4*>(g + c0 + 4));
+    const float4 b0 = __ldg(reinterpret_cast<const float4*>(b + c0)), b1 = __ldg(reinterpret_cast<const float4*>(b + c0 + 4));
+    const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+    const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      w[j] = pack_bf16x2((v[8 * i + 2 * j] - mean) * rstd * gg[2 * j] + bb[2 * j],
+                         (v[8 * i + 2 * j + 1] - mean) * rstd * gg[2 * j + 1] + bb[2 * j + 1]);
+    xr[lane + 32 * i] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
 template <int VEC>
 __global__ void __launch_bounds__(256)
     layernorm_kernel(float* h, int rows, const float* p0, const float* p1, int mode, float eps,

@@ -334,6 +334,11 @@ def prepare_sample(m: Model, feats: np.ndarray, mask: np.ndarray, state: np.ndar
     features and every cross layer's K/V over the tokens it attends to
     (``cross_key_mask``; [ARCH] backbone forward: attention_mask == 1)."""
     f = to_f64(feats)
+    if "vlln.g" in m.w:
+        # READING: the vision-language layer norm ([ARCH] config "tune_vlln":
+        # a trainable LayerNorm of the action head) normalises every backbone
+        # token's features, with its gain and bias, before the cross layers
+        f = layer_norm(f, m.g.ln_eps, m["vlln.g"], m["vlln.b"])
     kvs = {layer: cross_kv(m, layer, f[cross_key_mask(layer, mask, image_mask, n)])
            for layer in range(0, m.g.num_layers, 2)}
     s = state_encoder(m, to_f64(state).reshape(-1, m.g.state_dim), c)

@@ -170,6 +170,7 @@ class Geometry:
     ln_eps: float = 1e-5
     weight_dtype: str = "bf16"      # "bf16" -> uint16 bit patterns, "f32" -> float32
     attend_text_every_n_blocks: int = 0   # 0: every cross layer attends to all valid tokens
+    vlln: bool = False              # vision-language LayerNorm (vlln.g, vlln.b) on the backbone features
 
 
 GEOM_FULL = Geometry()
@@ -258,6 +259,9 @@ def weight_shapes(g: Geometry) -> Dict[str, Tuple[int, ...]]:
         "act_dec.l1.W": (C, D, D), "act_dec.l1.b": (C, D),
         "act_dec.l2.W": (C, D, g.action_dim), "act_dec.l2.b": (C, g.action_dim),
     })
+    if g.vlln:
+        s["vlln.g"] = (g.backbone_dim,)
+        s["vlln.b"] = (g.backbone_dim,)
     return s
 
 
@@ -276,7 +280,7 @@ def make_weights(g: Geometry, seed: int = 0) -> Dict[str, np.ndarray]:
     shapes = weight_shapes(g)
 
     def work(name: str):
-        mean = 1.0 if name.endswith("ln3.g") else 0.0
+        mean = 1.0 if name.endswith("ln3.g") or name == "vlln.g" else 0.0
         return name, _draw(name, shapes[name], seed, g.weight_dtype, mean=mean)
 
     with ThreadPoolExecutor(_threads()) as ex:

@@ -142,3 +142,16 @@ def test_wait_expiry_check_validates_on_host(L):
     import torch
     if not torch.cuda.is_available():
         assert L.gdit_debug_wait_expiry(0, 1_000_000) == GDIT_ENODEV
+
+
+def test_vlln_weights_come_in_pairs_of_the_backbone_width(L, tinyW):
+    """The optional vision-language layer norm: vlln.g and vlln.b together, [Dvl] each."""
+    dvl = synth.GEOM_TINY.backbone_dim
+    only_g = dict(tinyW)
+    only_g["vlln.g"] = np.ones(dvl, np.float32)
+    rc, _, msg = _create(L, _cfg(synth.GEOM_TINY), only_g)
+    assert rc == _lib.GDIT_EINVAL and "together" in msg
+    bad = dict(only_g)
+    bad["vlln.b"] = np.zeros(dvl + 1, np.float32)
+    rc, _, msg = _create(L, _cfg(synth.GEOM_TINY), bad)
+    assert rc == _lib.GDIT_EINVAL and "vlln.b" in msg

@@ -370,3 +370,33 @@ def test_image_text_split_matches_oracle(n, batch):
     ref0 = oracle.get_action(W, g, inp["backbone_features"], inp["vl_mask"], inp["state"], inp["embodiment_id"],
                              inp["init_noise"], 4, samples=rows)
     assert_parity(plain[rows], ref0, inp["init_noise"][rows], f"split on, no image mask, n={n} B={batch}")
+
+
+# ---------------------------------------------------------------- vision-language layer norm (vlln)
+
+@pytest.mark.parametrize("batch", [1, 3])
+def test_vlln_matches_oracle_and_removes_token_scale(batch):
+    """With vlln weights the packed backbone tokens are layer-normalised before
+    the K/V projection.  Each token's features get a random scale in [0.5, 3]
+    and shift in [-2, 2] (which vlln removes and the parity would otherwise
+    show); the device must match the oracle and not see the transform."""
+    require_gpu()
+    from flow_matching_dit_b200 import ActionHead
+    g = dataclasses.replace(synth.GEOM_TINY, vlln=True)
+    W = synth.make_weights(g)
+    w = dataclasses.replace(synth.WORKLOADS["tiny"], geom=g, batch=batch, seq=64, valid_min=30,
+                            fixed_ids=(0, 1, 1)[:batch])
+    inp = synth.make_inputs(w, seed=51)
+    r = np.random.default_rng(52)
+    f = inp["backbone_features"].astype(np.float32)
+    a = r.uniform(0.5, 3.0, size=(batch, 64, 1)).astype(np.float32)
+    c = r.uniform(-2.0, 2.0, size=(batch, 64, 1)).astype(np.float32)
+    moved = dict(inp)
+    moved["backbone_features"] = (f * a + c).astype(np.float32)
+    with ActionHead(g, W, max_batch=batch, max_seq=64) as head:
+        got, st = run_gpu(head, moved, 4)
+        same, st2 = run_gpu(head, inp, 4)
+    assert st == 0 and st2 == 0
+    ref = run_oracle(W, g, moved, 4)
+    assert_parity(got, ref, inp["init_noise"], f"vlln B={batch}")
+    assert_parity(same, ref, inp["init_noise"], f"vlln B={batch}, untransformed features")

@@ -447,3 +447,46 @@ def test_split_n2_alternates_text_and_image(W4):
     zero_k["blk2.v.b"][:] = 0
     g0 = dataclasses.replace(G4, attend_text_every_n_blocks=0)
     np.testing.assert_allclose(r0, _run(zero_k, inp, g=g0), rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- vision-language layer norm (vlln)
+
+GV = dataclasses.replace(G, vlln=True)
+
+
+@pytest.fixture(scope="module")
+def WV():
+    return synth.make_weights(GV)
+
+
+def _token_affine(feats, seed=5):
+    """Each token's features scaled by a_t in [0.5, 3] and shifted by c_t in [-2, 2]."""
+    r = np.random.default_rng(seed)
+    B, S, _ = feats.shape
+    a = r.uniform(0.5, 3.0, size=(B, S, 1)).astype(np.float32)
+    c = r.uniform(-2.0, 2.0, size=(B, S, 1)).astype(np.float32)
+    return (feats * a + c).astype(np.float32)
+
+
+def test_vlln_makes_the_head_blind_to_each_tokens_scale_and_shift(WV):
+    """A LayerNorm over each token's features removes that token's mean and
+    scale: with vlln the actions do not change (up to the eps under the square
+    root, relative 1e-5, and the fp32 rounding of the moved features); without
+    it they change by more than 1e-3."""
+    inp = _inputs(seed=9)
+    base = _run(WV, inp, g=GV)
+    moved = dict(inp)
+    moved["backbone_features"] = _token_affine(inp["backbone_features"])
+    np.testing.assert_allclose(_run(WV, moved, g=GV), base, rtol=1e-4, atol=1e-5)
+    plain = {k: v for k, v in WV.items() if not k.startswith("vlln.")}
+    assert np.abs(_run(plain, moved, g=G) - _run(plain, inp, g=G)).max() > 1e-3
+
+
+def test_vlln_zero_gain_leaves_only_its_bias(WV):
+    """vlln.g = 0: every token becomes vlln.b, so the features do not matter."""
+    W0 = _copy(WV)
+    W0["vlln.g"][:] = 0
+    inp = _inputs(seed=9)
+    other = dict(inp)
+    other["backbone_features"] = -3.0 * inp["backbone_features"] + 1.0
+    np.testing.assert_allclose(_run(W0, other, g=GV), _run(W0, inp, g=GV), rtol=1e-12, atol=1e-12)
