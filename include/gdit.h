@@ -37,6 +37,10 @@
  *     call returns unless stated otherwise.
  *   - Row-major, densely packed tensors; shapes are given as [dim0, dim1, ...].
  *   - Calls on one handle must not run concurrently from several host threads.
+ *     The handle's workspace (activations, K/V cache, status word) is shared by
+ *     its calls: calls on different streams must be ordered by the caller (an
+ *     event or a synchronize), or use one handle per stream.  Handles are
+ *     independent of one another.
  */
 #ifndef GDIT_H
 #define GDIT_H
