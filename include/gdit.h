@@ -113,6 +113,9 @@ typedef struct {
  *   act_enc.W1.W [C,A,D] .b [C,D]    act_enc.W2.W [C,2D,D] .b [C,D]
  *   act_enc.W3.W [C,D,D] .b [C,D]    act_dec.l1.W [C,D,D] .b [C,D]
  *   act_dec.l2.W [C,D,A] .b [C,A]
+ * Optional, given together: vlln.g [Dvl] vlln.b [Dvl], the vision-language
+ * LayerNorm of each backbone token's features before the cross K/V (needs
+ * Dvl a multiple of 256, at most 4096).
  * Plain linears are PyTorch [out, in] (y = x W^T + b).  Category-specific
  * weights keep CategorySpecificLinear's [C, in, out] (y = x W[c] + b[c]).
  * dtype GDIT_F32 (float) or GDIT_BF16 (uint16 bit patterns); matrices are
