@@ -131,6 +131,8 @@ def test_valid_table_without_gpu_reports_no_device(L, tinyW):
 
 def test_null_handle_calls_are_rejected(L):
     assert L.gdit_get_action(None, None, 0, None, None, None, None, 4, None, 1, 1, None) == _lib.GDIT_EINVAL
+    assert L.gdit_get_action_vl(None, None, 0, None, None, None, None, None, 4, None, 1, 1, None) == _lib.GDIT_EINVAL
+    assert L.gdit_get_action_host(None, None, 0, None, None, None, None, 4, None, 1, 1, None) == _lib.GDIT_EINVAL
     assert L.gdit_sync_status(None) == _lib.GDIT_EINVAL
     L.gdit_destroy(None)
 
