@@ -306,9 +306,8 @@ __device__ __forceinline__ bool small_wait(const SmallCtx& P, int phase, int tar
   return *s_ok != 0;
 }
 
-// All compute threads' writes of the phase, then one release increment.
+// One release increment, after the barrier that ends the phase.
 __device__ __forceinline__ void small_arrive(const SmallCtx& P, int phase) {
-  csync();
   if (threadIdx.x == 0) red_release_add(P.counters + phase, 1);
 }
 
@@ -688,7 +687,7 @@ __device__ __forceinline__ void small_epilogue(const SmallGemm& g, int n, int to
 // and every warp releases a slot after its last read of it.
 __device__ __forceinline__ bool small_gemm_phase(const SmallGemm& g, const AttnArgs& att, const SmallCtx& P,
                                                  uint8_t* smem, SmallRing& R, uint32_t& item, uint64_t* xbar,
-                                                 uint32_t& xuse) {
+                                                 uint32_t& xuse, int* fail) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gr = lane >> 2, tig = lane & 3;
   const int nu = small_my_units(g), nch = small_nchunks(g), kc = small_kc(g);
@@ -848,8 +847,14 @@ __device__ __forceinline__ bool small_gemm_phase(const SmallGemm& g, const AttnA
     const int n = small_unit(threadIdx.x / kSmallUF) * kSmallUF + threadIdx.x % kSmallUF;
     reinterpret_cast<float*>(g.out)[n] = g.state_row[n];
   }
-  csync();   // the X area is rewritten by the next phase
-  return ok;
+  // One barrier ends the phase: every thread's epilogue stores precede the
+  // arrival (thread 0 releases right after it), the X area and the slot of
+  // this phase's descriptor may be rewritten after it (every thread waited
+  // for its descriptor copies first), and the failure flag is uniform.
+  if (!ok) *fail = 1;
+  cp_async_wait<0>();
+  csync();
+  return *fail == 0;
 }
 
 // ---------------------------------------------------------------- attention phase (one CTA per head)
@@ -933,7 +938,10 @@ __device__ __forceinline__ void small_attention_phase(const AttnArgs& a, int hea
     }
     *reinterpret_cast<uint32_t*>(obase + (size_t)row * a.out_ld + d) = pack_bf16x2(r0, r1);
   }
-  csync();   // shared memory is reused by the next phase
+  // one barrier ends the phase (as for a GEMM phase): stores before the
+  // arrival, shared memory and the descriptor slot free afterwards
+  cp_async_wait<0>();
+  csync();
 }
 
 template <int DH>
@@ -1015,13 +1023,10 @@ __global__ void __launch_bounds__(kSmallThreads, 1) small_loop_kernel(const Smal
     if ((int)blockIdx.x < w) {
       ok = small_wait(P, gp - 1, prev_workers, &s_ok);
       if (ok) {
-        if (cur.kind == 0) {
-          if (!small_gemm_phase(cur.g, cur.a, P, smem, s_ring, item, &s_xbar, xuse)) s_fail = 1;
-          csync();
-          ok = s_fail == 0;
-        } else {
+        if (cur.kind == 0)
+          ok = small_gemm_phase(cur.g, cur.a, P, smem, s_ring, item, &s_xbar, xuse, &s_fail);
+        else
           small_attention_phase<DH>(cur.a, blockIdx.x, smem);
-        }
         if (ok) small_arrive(P, gp);
       }
     }
@@ -1036,10 +1041,13 @@ __global__ void __launch_bounds__(kSmallThreads, 1) small_loop_kernel(const Smal
       return;
     }
     prev_workers = w;
-    // the next descriptor has landed, and every compute thread is done with
-    // this one before its slot is refilled
-    cp_async_wait<0>();
-    csync();
+    if ((int)blockIdx.x >= w) {
+      // an idle CTA: the next descriptor has landed, and every compute thread
+      // is done with this one before its slot is refilled (a working CTA's
+      // phase ended with that barrier)
+      cp_async_wait<0>();
+      csync();
+    }
     slot = slot == 2 ? 0 : slot + 1;
   }
 }
