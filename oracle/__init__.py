@@ -9,4 +9,4 @@ product.  See ``oracle/dit.py`` for the sources each function follows.
 from .dit import (Model, action_decoder, action_encoder, ada_layer_norm, attention,  # noqa: F401
                   category_linear, cross_key_mask, cross_kv, dit, dit_block, euler_schedule, gelu, get_action,
                   layer_norm, linear, prepare_sample, relu, silu, sinusoidal_embedding,
-                  state_encoder, swish, timestep_embedding, to_f64, velocity)
+                  state_encoder, swish, timestep_embedding, to_f64, training_loss, velocity)

@@ -376,3 +376,40 @@ def get_action(weights: Dict[str, np.ndarray], geom, backbone_features, vl_mask,
             x = x + dt * velocity(m, x, td, s, kvs, c)
         outs.append(x)
     return np.stack(outs)
+
+
+def training_loss(weights: Dict[str, np.ndarray], geom, backbone_features, vl_mask, state, embodiment_id,
+                  actions, noise, t, action_mask, model: Optional[Model] = None, image_mask=None):
+    """Flow-matching training objective of the action head, forward only
+    ([ARCH] "Flow matching diffusion", "Training objective").
+
+    Per sample b with time t_b: x_t = (1 - t_b) noise_b + t_b actions_b; the
+    target velocity is actions_b - noise_b; the prediction is the velocity
+    field at x_t with t_discretized = floor(t_b * buckets) (as in inference).
+    READING: t is an input (the page samples it from Beta(1.5, 1); the random
+    draw is passed in).  READING: the loss is the masked mean of the
+    element-wise squared error, sum(mask * (pred - v)^2) / (sum(mask) + 1e-6)
+    (the printed code multiplies a mean-reduced mse_loss by the mask; the mask
+    and the denominator only make sense element-wise).
+    Returns (loss, pred [B, H, A]) in float64.
+    """
+    m = model if model is not None else Model(weights, geom)
+    ids = np.asarray(embodiment_id).reshape(-1)
+    n = int(getattr(geom, "attend_text_every_n_blocks", 0))
+    a = to_f64(actions)
+    e = to_f64(noise)
+    tt = to_f64(t).reshape(-1)
+    preds = []
+    for b in range(len(ids)):
+        c = int(ids[b])
+        if not 0 <= c < geom.num_embodiments:
+            raise ValueError(f"embodiment_id {c} out of range")
+        s, kvs = prepare_sample(m, backbone_features[b], vl_mask[b], state[b], c,
+                                None if image_mask is None else image_mask[b], n)
+        xt = (1.0 - tt[b]) * e[b] + tt[b] * a[b]
+        td = math.floor(tt[b] * geom.num_timestep_buckets)
+        preds.append(velocity(m, xt, float(td), s, kvs, c))
+    pred = np.stack(preds)
+    mask = to_f64(action_mask)
+    loss = float((mask * (pred - (a - e)) ** 2).sum() / (mask.sum() + 1e-6))
+    return loss, pred

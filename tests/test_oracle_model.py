@@ -490,3 +490,105 @@ def test_vlln_zero_gain_leaves_only_its_bias(WV):
     other = dict(inp)
     other["backbone_features"] = -3.0 * inp["backbone_features"] + 1.0
     np.testing.assert_allclose(_run(W0, other, g=GV), _run(W0, inp, g=GV), rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- training objective (forward)
+
+def _train_inputs(seed=21, batch=2):
+    inp = _inputs(batch=batch, ids=(0, 1)[:batch], seed=seed)
+    r = np.random.default_rng(seed)
+    shape = inp["init_noise"].shape
+    acts = r.standard_normal(shape).astype(np.float32)
+    mask = (r.uniform(size=shape) < 0.7).astype(np.float32)
+    return inp, acts, mask
+
+
+def _loss(W, inp, acts, noise, t, mask, g=G):
+    return oracle.training_loss(W, g, inp["backbone_features"], inp["vl_mask"], inp["state"],
+                                inp["embodiment_id"], acts, noise, np.asarray(t, np.float64), mask)
+
+
+def test_training_loss_of_a_zero_velocity_head_is_the_masked_target_energy(W):
+    """pred = 0 (decoder output layer zeroed): the loss is
+    sum(mask * (a - e)^2) / (sum(mask) + 1e-6), whatever t."""
+    W0 = _copy(W)
+    W0["act_dec.l2.W"][:] = 0
+    W0["act_dec.l2.b"][:] = 0
+    inp, acts, mask = _train_inputs()
+    noise = inp["init_noise"]
+    target = acts.astype(np.float64) - noise.astype(np.float64)
+    m64 = mask.astype(np.float64)
+    want = float((m64 * target ** 2).sum() / (m64.sum() + 1e-6))
+    for t in ([0.3, 0.9], [0.0, 1.0]):
+        loss, pred = _loss(W0, inp, acts, noise, t, mask)
+        assert np.all(pred == 0)
+        assert loss == pytest.approx(want, rel=1e-12)
+
+
+def test_training_prediction_at_t0_is_the_first_euler_velocity(W):
+    """t = 0: x_t is the noise and t_discretized is 0, so the predicted velocity
+    is v(noise, 0) = get_action(K = 1) - noise."""
+    inp, acts, mask = _train_inputs()
+    _, pred = _loss(W, inp, acts, inp["init_noise"], [0.0, 0.0], mask)
+    ref = _run(W, inp, K=1) - inp["init_noise"].astype(np.float64)
+    np.testing.assert_allclose(pred, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_training_prediction_at_t_half_is_the_second_euler_velocity(W):
+    """With actions = noise = x1 (so x_t = x1 for every t) and t = 0.5
+    (t_discretized 500), the prediction is the velocity of the second step of
+    the K = 2 loop: (x2 - x1) / 0.5, with x1 = noise + 0.5 v(noise, 0)."""
+    inp, _, mask = _train_inputs()
+    e = inp["init_noise"].astype(np.float64)
+    v0 = _run(W, inp, K=1) - e
+    x1 = e + 0.5 * v0
+    x2 = _run(W, inp, K=2)
+    _, pred = _loss(W, inp, x1, x1, [0.5, 0.5], mask)
+    np.testing.assert_allclose(pred, (x2 - x1) / 0.5, rtol=1e-9, atol=1e-10)
+
+
+def test_training_loss_interpolates_noise_and_actions(W):
+    """x_t = (1 - t) noise + t actions: at t = 1 the prediction depends on the
+    actions only (changing the noise changes only the target), at t = 0 on the
+    noise only."""
+    inp, acts, mask = _train_inputs()
+    e = inp["init_noise"]
+    _, p1 = _loss(W, inp, acts, e, [1.0, 1.0], mask)
+    _, p1b = _loss(W, inp, acts, (e + 1.0).astype(np.float32), [1.0, 1.0], mask)
+    np.testing.assert_array_equal(p1, p1b)
+    _, p0 = _loss(W, inp, acts, e, [0.0, 0.0], mask)
+    _, p0b = _loss(W, inp, (acts + 1.0).astype(np.float32), e, [0.0, 0.0], mask)
+    np.testing.assert_array_equal(p0, p0b)
+
+
+def test_training_loss_of_a_perfect_predictor_is_zero(W):
+    """At t = 0 the prediction is v(noise, 0) whatever the actions are; with
+    actions = noise + v(noise, 0) the target actions - noise equals that
+    prediction, so the loss vanishes (and a flipped target would give 4 v^2)."""
+    inp, _, mask = _train_inputs()
+    e = inp["init_noise"].astype(np.float64)
+    v0 = _run(W, inp, K=1) - e
+    loss, pred = _loss(W, inp, e + v0, inp["init_noise"], [0.0, 0.0], mask)
+    np.testing.assert_allclose(pred, v0, rtol=1e-12, atol=1e-12)
+    assert loss < 1e-20
+    loss_off, _ = _loss(W, inp, e + v0 + 0.5, inp["init_noise"], [0.0, 0.0], mask)
+    m64 = mask.astype(np.float64)
+    assert loss_off == pytest.approx(0.25 * m64.sum() / (m64.sum() + 1e-6), rel=1e-9)
+
+
+def test_training_time_is_truncated_to_its_bucket(W):
+    """t_discretized = floor(t * buckets): with actions = noise (x_t the same
+    for every t) the prediction depends on the bucket alone, so t = 0.5009
+    predicts as t = 0.5 (bucket 500) and t = 0.4999 as t = 0.499 (bucket 499),
+    and buckets 499 and 500 predict differently."""
+    inp, _, mask = _train_inputs()
+    e = inp["init_noise"]
+
+    def pred(t):
+        return _loss(W, inp, e, e, [t, t], mask)[1]
+
+    p500 = pred(0.5)
+    np.testing.assert_array_equal(pred(0.5009), p500)
+    p499 = pred(0.499)
+    np.testing.assert_array_equal(pred(0.4999), p499)
+    assert np.abs(p500 - p499).max() > 1e-6
