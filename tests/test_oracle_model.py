@@ -592,3 +592,85 @@ def test_training_time_is_truncated_to_its_bucket(W):
     p499 = pred(0.499)
     np.testing.assert_array_equal(pred(0.4999), p499)
     assert np.abs(p500 - p499).max() > 1e-6
+
+
+# ---------------------------------------------------------------- composition of the pieces
+
+def test_action_encoder_ends_in_its_third_layer(W):
+    """W3[c] = 0 leaves b3[c] on every action token, whatever the actions and t
+    (the encoder's last step is the W3 layer, [ARCH] multi-embodiment action
+    encoder)."""
+    W0 = _copy(W)
+    W0["act_enc.W3.W"][1] = 0
+    m = oracle.Model(W0, G)
+    x = rng.normal(size=(G.action_horizon, G.action_dim))
+    for td in (0.0, 750.0):
+        out = oracle.action_encoder(m, x, td, 1)
+        np.testing.assert_array_equal(out, np.broadcast_to(W0["act_enc.W3.b"][1].astype(np.float64), out.shape))
+    assert not np.allclose(oracle.action_encoder(oracle.Model(W, G), x, 0.0, 1), W["act_enc.W3.b"][1])
+
+
+def test_final_layer_is_output_adaln_then_proj_out_then_decoder(W):
+    """out.ada.w = 0 with bias (scale = -1, shift = sigma) turns the final AdaLN
+    into the constant sigma, so each step's velocity is
+    decoder_c(proj_out(sigma)) for every token and input, and the K-step loop
+    adds it once: x_K = noise + v (computed here with torch's linear and bmm)."""
+    import torch
+    W0 = _copy(W)
+    D = G.hidden
+    sigma = rng.normal(size=D).astype(np.float32)
+    W0["out.ada.w"][:] = 0
+    W0["out.ada.b"][:D] = -1.0
+    W0["out.ada.b"][D:] = sigma
+    inp = _inputs(batch=2, ids=[1, 0], seed=9)
+    out = _run(W0, inp, K=4)
+    t = lambda a: torch.from_numpy(np.asarray(a, np.float64))
+    y = torch.nn.functional.linear(t(sigma), t(W0["out.proj.w"]), t(W0["out.proj.b"]))
+    for b, c in enumerate((1, 0)):
+        h1 = torch.relu(torch.bmm(y.view(1, 1, D), t(W0["act_dec.l1.W"][c:c + 1])) + t(W0["act_dec.l1.b"][c]))
+        v = torch.bmm(h1, t(W0["act_dec.l2.W"][c:c + 1])) + t(W0["act_dec.l2.b"][c])
+        want = inp["init_noise"][b].astype(np.float64) + v.numpy().reshape(1, G.action_dim)
+        np.testing.assert_allclose(out[b], want, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("layer", [0, 1])
+def test_attention_branch_sees_h_only_through_its_adaln(W, layer):
+    """With the MLP branch zeroed, block(h) - h is the attention branch, whose
+    queries (and, in self layers, keys and values) come from AdaLN(h).  A layer
+    norm without eps ignores a per-row scale and shift of h, so the branch is
+    the same for h and alpha_row * h + beta_row."""
+    g = dataclasses.replace(G, ln_eps=0.0)
+    W0 = _copy(W)
+    W0[f"blk{layer}.ff2.w"][:] = 0
+    W0[f"blk{layer}.ff2.b"][:] = 0
+    m = oracle.Model(W0, g)
+    inp = _inputs(seed=4)
+    _, kvs = oracle.prepare_sample(m, inp["backbone_features"][0], inp["vl_mask"][0], inp["state"][0], 0)
+    h = rng.normal(size=(G.action_horizon + 1, G.hidden))
+    temb = oracle.timestep_embedding(m, 250.0)
+    alpha = rng.uniform(0.5, 3.0, size=(h.shape[0], 1))
+    beta = rng.normal(size=(h.shape[0], 1))
+    h2 = alpha * h + beta
+    kv = None if layer % 2 else kvs[layer]
+    br = oracle.dit_block(m, layer, h, temb, kv) - h
+    br2 = oracle.dit_block(m, layer, h2, temb, kv) - h2
+    np.testing.assert_allclose(br2, br, rtol=1e-9, atol=1e-12)
+    assert np.abs(br).max() > 1e-3
+
+
+def test_modulation_sees_temb_only_through_silu(W):
+    """t_enc.l2 = (0, -60) makes temb = -60, where SiLU is below 1e-24: every
+    AdaLN (blocks and output) is then left with its bias, so zeroing all AdaLN
+    weights changes nothing (AdaLN input SiLU(temb), [ARCH] norm1(h, temb))."""
+    W1 = _copy(W)
+    W1["t_enc.l2.w"][:] = 0
+    W1["t_enc.l2.b"][:] = -60.0
+    W2 = _copy(W1)
+    for name in W2:
+        if name.endswith("ada.w"):
+            W2[name][:] = 0
+    inp = _inputs(batch=2, ids=[0, 1], seed=6)
+    np.testing.assert_allclose(_run(W1, inp, K=2), _run(W2, inp, K=2), rtol=1e-12, atol=1e-12)
+    W3 = _copy(W1)
+    W3["t_enc.l2.b"][:] = 2.0
+    assert not np.allclose(_run(W3, inp, K=2), _run(dict(W3, **{k: W2[k] for k in W2 if k.endswith("ada.w")}), inp, K=2))
