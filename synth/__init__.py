@@ -34,7 +34,7 @@ import numpy as np
 
 __all__ = [
     "Geometry", "Workload", "GEOM_FULL", "GEOM_TINY", "WORKLOADS", "workload", "make_image_mask",
-    "splitmix64_stream", "uniform53", "normal", "randint", "tensor_seed",
+    "splitmix64_stream", "uniform53", "normal", "randint", "tensor_seed", "fnv1a64",
     "f32_to_bf16_bits", "bf16_bits_to_f32", "weight_shapes", "make_weights",
     "make_inputs",
 ]
@@ -62,12 +62,18 @@ def splitmix64_stream(seed: int, n: int, offset: int = 0) -> np.ndarray:
         return _mix64(state)
 
 
-def tensor_seed(base_seed: int, name: str) -> int:
-    """Per-tensor seed: SplitMix64 finaliser of (base * golden) xor FNV-1a(name)."""
+def fnv1a64(text: str) -> int:
+    """64-bit FNV-1a hash of the UTF-8 bytes of `text`."""
     h = 0xCBF29CE484222325
-    for byte in name.encode():
+    for byte in text.encode():
         h ^= byte
         h = (h * 0x100000001B3) & 0xFFFFFFFFFFFFFFFF
+    return h
+
+
+def tensor_seed(base_seed: int, name: str) -> int:
+    """Per-tensor seed: SplitMix64 finaliser of (base * golden) xor FNV-1a(name)."""
+    h = fnv1a64(name)
     with np.errstate(over="ignore"):
         z = (np.uint64(base_seed & 0xFFFFFFFFFFFFFFFF) * _GOLDEN) ^ np.uint64(h)
         return int(_mix64(np.array([z], dtype=np.uint64))[0])
