@@ -139,6 +139,30 @@ def time_oracle(W, w, samples: int):
     return samples / dt, cores, dt
 
 
+# ------------------------------------------------------------------ B = 1 roofline
+
+def b1_algorithmic_bytes(g, seq: int, num_steps: int) -> int:
+    """Minimum HBM bytes of one single-sample call's Euler loop: every step
+    streams the bf16 weights of the 32 DiT blocks (self: Q|K|V, O, FF1, FF2;
+    cross: Q, O, FF1, FF2), of the action encoder (W1, the action half of W2,
+    W3), proj_out and the decoder (one category), and reads the cross layers'
+    K/V cache of `seq` valid tokens."""
+    D, F, A, L = g.hidden, g.mlp_hidden, g.action_dim, g.num_layers
+    self_layer = 3 * D * D + D * D + 2 * F * D
+    cross_layer = 2 * D * D + 2 * F * D
+    head = A * D + D * D + D * D + D * D + D * D + D * A
+    kv = (L // 2) * 2 * seq * D * 2
+    return num_steps * (((L // 2) * (self_layer + cross_layer) + head) * 2 + kv)
+
+
+def latency_roofline(g, seq: int, num_steps: int, p50_ms: float, hbm_gbs: float) -> dict:
+    """HBM roofline of the B = 1 call at its p50 latency."""
+    b = b1_algorithmic_bytes(g, seq, num_steps)
+    ach = b / (p50_ms / 1e3) / 1e9
+    return {"bound": "hbm", "algorithmic_bytes": b, "achieved": ach, "peak": hbm_gbs, "unit": "GB/s",
+            "frac": ach / hbm_gbs}
+
+
 # ------------------------------------------------------------------ replicas (one per GPU, no data-path collective)
 
 def ranks_from_env():
@@ -286,6 +310,7 @@ def main():
         lat = {"p50_ms": float(np.percentile(ts, 50)), "p99_ms": float(np.percentile(ts, 99)),
                "mean_ms": float(ts.mean()), "calls": int(len(ts)),
                "workload": "B=1, backbone [1,300,2048] bf16 all valid, id 0, K=4"}
+        lat["roofline"] = latency_roofline(wl.geom, wl.seq, wl.num_steps, lat["p50_ms"], load_peaks()[0])
 
     # ---- end to end through the host-buffer entry point (pinned host memory)
     e2e = None
