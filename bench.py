@@ -50,7 +50,7 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-profile", action="store_true")
-    p.add_argument("--oracle-samples", type=int, default=2)
+    p.add_argument("--oracle-samples", type=int, default=24)
     p.add_argument("--batch", type=int, default=None, help="override the throughput batch (profiling runs)")
     p.add_argument("--seq", type=int, default=None, help="override the throughput backbone length (profiling runs)")
     return p.parse_args()
