@@ -53,3 +53,24 @@ def test_b1_bytes_of_the_latency_workload():
     r = bench.latency_roofline(w.geom, w.seq, w.num_steps, 4.73, 6452.8)
     assert r["frac"] == pytest.approx(b / 4.73e-3 / 1e9 / 6452.8)
     assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+
+
+def test_reference_arm_prints_one_complete_line(monkeypatch, capsys):
+    """`bench.py --impl reference` times the oracle and prints one JSON line
+    with the contract's keys (run here on the tiny workload)."""
+    import argparse
+    import json
+    monkeypatch.setattr(bench, "THROUGHPUT", "tiny")
+    args = argparse.Namespace(gpus=1, steps=2, warmup=1)
+    bench.run_reference(args, rank=0)
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == bench.UNIT
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    bench.run_reference(args, rank=1)                     # other ranks print nothing
+    assert capsys.readouterr().out.strip() == ""
