@@ -25,12 +25,39 @@ from ._lib import (GDIT_BF16, GDIT_F32, GDIT_FLAG_NO_GRAPH, GDIT_FLAG_NO_SMALL, 
                    GditError, check, lib)
 from .build import build  # noqa: F401
 
-__all__ = ["ActionHead", "GditError", "lib", "build", "GDIT_BF16", "GDIT_F32",
+__all__ = ["ActionHead", "GditError", "lib", "build", "check_io_shapes", "GDIT_BF16", "GDIT_F32",
            "GDIT_FLAG_NO_GRAPH", "GDIT_FLAG_NO_SMALL", "GDIT_FLAG_STRICT_PROFILES"]
 
 
 def _ptr(t) -> int:
     return int(t.data_ptr())
+
+
+def check_io_shapes(cfg, feats, mask, state, ids, noise, out, image_mask=None):
+    """The library reads and writes the I/O buffers by the batch and sequence
+    it is given, so every buffer must have the shape that implies (a smaller
+    one would be read or written past its end).  Raises ValueError.
+
+    feats [B, S, backbone_dim]; vl_mask and image_mask [B, S]; state
+    [B, 1, state_dim] (or [B, state_dim]); embodiment_id [B];
+    init_noise and out [B, action_horizon, action_dim]."""
+    shp = lambda t: tuple(int(d) for d in t.shape)
+    if len(shp(feats)) != 3:
+        raise ValueError(f"backbone_features must be [batch, seq, {cfg.backbone_dim}], got {shp(feats)}")
+    B, S, dvl = shp(feats)
+    if dvl != cfg.backbone_dim:
+        raise ValueError(f"backbone_features last dim {dvl} != backbone_dim {cfg.backbone_dim}")
+    want = {"vl_mask": (mask, [(B, S)]),
+            "state": (state, [(B, 1, cfg.state_dim), (B, cfg.state_dim)]),
+            "embodiment_id": (ids, [(B,)]),
+            "init_noise": (noise, [(B, cfg.action_horizon, cfg.action_dim)]),
+            "out": (out, [(B, cfg.action_horizon, cfg.action_dim)])}
+    if image_mask is not None:
+        want["image_mask"] = (image_mask, [(B, S)])
+    for name, (t, shapes) in want.items():
+        if shp(t) not in shapes:
+            raise ValueError(f"{name} has shape {shp(t)}, expected {' or '.join(map(str, shapes))}")
+    return B, S
 
 
 class ActionHead:
@@ -81,14 +108,18 @@ class ActionHead:
             bb = GDIT_F32
         else:
             raise TypeError("backbone_features must be bfloat16 or float32")
-        B, S = int(feats.shape[0]), int(feats.shape[1])
-        for t, dt in ((mask, torch.uint8), (state, torch.float32), (ids, torch.int32), (noise, torch.float32)):
+        if out is None:
+            out = torch.empty_like(noise)
+        for t, dt in ((mask, torch.uint8), (state, torch.float32), (ids, torch.int32), (noise, torch.float32),
+                      (out, torch.float32)):
             if t.dtype != dt or not t.is_contiguous() or not t.is_cuda:
                 raise TypeError(f"expected a contiguous CUDA tensor of {dt}")
         if not feats.is_contiguous() or not feats.is_cuda:
             raise TypeError("backbone_features must be a contiguous CUDA tensor")
-        if out is None:
-            out = torch.empty_like(noise)
+        for t in (feats, mask, state, ids, noise, out):
+            if t.device.index != self.cfg.device:
+                raise ValueError(f"tensor on {t.device}, the head is on cuda:{self.cfg.device}")
+        B, S = check_io_shapes(self.cfg, feats, mask, state, ids, noise, out)
         return bb, B, S, out
 
     def get_action(self, feats, mask, state, ids, noise, num_steps: int = 4, out=None, stream=None,
@@ -104,8 +135,9 @@ class ActionHead:
                                        int(num_steps), _ptr(out), B, S, st), self.h)
             return out
         if image_mask.dtype != torch.uint8 or not image_mask.is_contiguous() or not image_mask.is_cuda \
-                or tuple(image_mask.shape) != (B, S):
-            raise TypeError("image_mask must be a contiguous CUDA uint8 tensor [batch, seq]")
+                or image_mask.device.index != self.cfg.device:
+            raise TypeError("image_mask must be a contiguous uint8 tensor on the head's device")
+        check_io_shapes(self.cfg, feats, mask, state, ids, noise, out, image_mask)
         check(_lib.gdit_get_action_vl(self.h, _ptr(feats), bb, _ptr(mask), _ptr(image_mask), _ptr(state), _ptr(ids),
                                       _ptr(noise), int(num_steps), _ptr(out), B, S, st), self.h)
         return out
@@ -123,7 +155,9 @@ class ActionHead:
         noise = np.ascontiguousarray(noise, dtype=np.float32)
         if out is None:
             out = np.empty_like(noise)
-        B, S = feats.shape[0], feats.shape[1]
+        if out.dtype != np.float32 or not out.flags.c_contiguous or not out.flags.writeable:
+            raise TypeError("out must be a writable contiguous float32 array")
+        B, S = check_io_shapes(self.cfg, feats, mask, state, ids, noise, out)
         check(_lib.gdit_get_action_host(self.h, feats.ctypes.data, bb, mask.ctypes.data, state.ctypes.data,
                                         ids.ctypes.data, noise.ctypes.data, int(num_steps), out.ctypes.data,
                                         B, S, stream or 0), self.h)

@@ -159,6 +159,10 @@ void gdit_destroy(gdit_handle* h);
  *   out_actions        device f32 [batch, action_horizon, action_dim]; may alias init_noise
  *   batch in [1, max_batch], seq in [1, max_backbone_seq]
  *   cuda_stream        cudaStream_t (NULL = legacy default stream)
+ * Buffer sizes are the caller's contract: the library reads and writes every
+ * buffer by (batch, seq) and the handle's dimensions and cannot see a device
+ * buffer's size, so a smaller buffer is read or written past its end.  (The
+ * Python binding checks the tensors' shapes before the call.)
  * Asynchronous on cuda_stream.  The first call of a new (batch, seq, K) profile
  * captures a CUDA graph of the whole loop (unless GDIT_FLAG_NO_GRAPH); with
  * GDIT_FLAG_STRICT_PROFILES that profile must have been gdit_prepare()d.

@@ -157,3 +157,34 @@ def test_vlln_weights_come_in_pairs_of_the_backbone_width(L, tinyW):
     bad["vlln.b"] = np.zeros(dvl + 1, np.float32)
     rc, _, msg = _create(L, _cfg(synth.GEOM_TINY), bad)
     assert rc == _lib.GDIT_EINVAL and "vlln.b" in msg
+
+
+def test_io_shapes_are_checked_before_any_pointer_is_passed():
+    """The binding refuses buffers whose shapes disagree with the batch and
+    sequence of the features: the library would read or write past them."""
+    from flow_matching_dit_b200 import check_io_shapes
+    g = synth.GEOM_TINY
+    cfg = _cfg(g)
+    B, S = 3, 40
+    ok = dict(feats=np.zeros((B, S, g.backbone_dim), np.float32), mask=np.zeros((B, S), np.uint8),
+              state=np.zeros((B, 1, g.state_dim), np.float32), ids=np.zeros(B, np.int32),
+              noise=np.zeros((B, g.action_horizon, g.action_dim), np.float32),
+              out=np.zeros((B, g.action_horizon, g.action_dim), np.float32))
+    assert check_io_shapes(cfg, **ok) == (B, S)
+    assert check_io_shapes(cfg, **dict(ok, state=np.zeros((B, g.state_dim), np.float32))) == (B, S)
+    assert check_io_shapes(cfg, **ok, image_mask=np.zeros((B, S), np.uint8)) == (B, S)
+    bad = {
+        "feats": np.zeros((B, S, g.backbone_dim + 1), np.float32),
+        "mask": np.zeros((B, S - 1), np.uint8),
+        "state": np.zeros((B - 1, 1, g.state_dim), np.float32),
+        "ids": np.zeros(B + 1, np.int32),
+        "noise": np.zeros((B, g.action_horizon - 1, g.action_dim), np.float32),
+        "out": np.zeros((B - 1, g.action_horizon, g.action_dim), np.float32),
+    }
+    for name, arr in bad.items():
+        with pytest.raises(ValueError):
+            check_io_shapes(cfg, **dict(ok, **{name: arr}))
+    with pytest.raises(ValueError):
+        check_io_shapes(cfg, **ok, image_mask=np.zeros((B, S + 1), np.uint8))
+    with pytest.raises(ValueError):
+        check_io_shapes(cfg, **dict(ok, feats=np.zeros((B * S, g.backbone_dim), np.float32)))
