@@ -188,3 +188,61 @@ def test_io_shapes_are_checked_before_any_pointer_is_passed():
         check_io_shapes(cfg, **ok, image_mask=np.zeros((B, S + 1), np.uint8))
     with pytest.raises(ValueError):
         check_io_shapes(cfg, **dict(ok, feats=np.zeros((B * S, g.backbone_dim), np.float32)))
+
+
+class _FakeCuda:
+    """Stands in for a contiguous CUDA tensor: dtype, shape and device only
+    (the pointer is never dereferenced: the handle below is NULL)."""
+
+    def __init__(self, shape, dtype, index=0):
+        import torch
+        self.shape, self.dtype, self.is_cuda = tuple(shape), dtype, True
+        self.device = torch.device("cuda", index)
+
+    def is_contiguous(self):
+        return True
+
+    def data_ptr(self):
+        return 0
+
+
+def test_device_call_path_validates_then_reaches_the_library(L):
+    """ActionHead.get_action's Python path on realistic inputs: it accepts
+    them, passes them to the library (a NULL handle: GDIT_EINVAL, nothing is
+    dereferenced), and rejects wrong shapes, dtypes and devices first."""
+    import torch
+    from flow_matching_dit_b200 import ActionHead, GditError
+    g = synth.GEOM_TINY
+    head = object.__new__(ActionHead)
+    head.cfg = _cfg(g)
+    head.cfg.device = 0
+    head.h = None
+    B, S = 2, 64
+    args = [_FakeCuda((B, S, g.backbone_dim), torch.bfloat16), _FakeCuda((B, S), torch.uint8),
+            _FakeCuda((B, 1, g.state_dim), torch.float32), _FakeCuda((B,), torch.int32),
+            _FakeCuda((B, g.action_horizon, g.action_dim), torch.float32)]
+    out = _FakeCuda((B, g.action_horizon, g.action_dim), torch.float32)
+    for kw in ({}, {"image_mask": _FakeCuda((B, S), torch.uint8)}):
+        with pytest.raises(GditError) as e:
+            head.get_action(*args, num_steps=4, out=out, stream=0, **kw)
+        assert e.value.code == _lib.GDIT_EINVAL
+    with pytest.raises(ValueError):
+        head.get_action(*args[:4], _FakeCuda((B, g.action_horizon + 1, g.action_dim), torch.float32),
+                        out=out, stream=0)
+    with pytest.raises(TypeError):
+        head.get_action(args[0], args[1], args[2], _FakeCuda((B,), torch.int64), args[4], out=out, stream=0)
+    with pytest.raises(ValueError):
+        head.get_action(*args, out=_FakeCuda(out.shape, torch.float32, index=1), stream=0)
+    with pytest.raises(TypeError):
+        head.get_action(*args, out=out, stream=0, image_mask=_FakeCuda((B, S), torch.bool))
+    with pytest.raises(ValueError):
+        head.get_action(*args, out=out, stream=0, image_mask=_FakeCuda((B, S - 1), torch.uint8))
+    # the host-buffer path on numpy inputs of the same shapes
+    inp = synth.make_inputs(synth.workload("tiny", batch=B, fixed_ids=(0, 1)))
+    with pytest.raises(GditError) as e:
+        head.get_action_host(inp["backbone_features"], inp["vl_mask"], inp["state"], inp["embodiment_id"],
+                             inp["init_noise"], 4)
+    assert e.value.code == _lib.GDIT_EINVAL
+    with pytest.raises(ValueError):
+        head.get_action_host(inp["backbone_features"], inp["vl_mask"][:, :-1], inp["state"],
+                             inp["embodiment_id"], inp["init_noise"], 4)
