@@ -243,4 +243,4 @@ def gemm_static_scratch(A, B, bias, C=None, bn: int = 64, splits: int = 1, strea
 def debug_wait_expiry(device: int = 0, limit_ns: int = 1_000_000) -> int:
     """Status of one bounded wait on an mbarrier that nothing arrives at
     (gdit_debug_wait_expiry): GDIT_ETIMEOUT is the expected result."""
-    return _lib.lib().gdit_debug_wait_expiry(int(device), int(limit_ns))
+    return _lib.gdit_debug_wait_expiry(int(device), int(limit_ns))

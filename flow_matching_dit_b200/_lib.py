@@ -167,3 +167,7 @@ def gdit_test_gemm(*a):
 
 def gdit_gemm_static_scratch(*a):
     return lib().gdit_gemm_static_scratch(*a)
+
+
+def gdit_debug_wait_expiry(device, limit_ns):
+    return lib().gdit_debug_wait_expiry(device, limit_ns)

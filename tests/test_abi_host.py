@@ -246,3 +246,8 @@ def test_device_call_path_validates_then_reaches_the_library(L):
     with pytest.raises(ValueError):
         head.get_action_host(inp["backbone_features"], inp["vl_mask"][:, :-1], inp["state"],
                              inp["embodiment_id"], inp["init_noise"], 4)
+
+
+def test_binding_forwards_every_entry_point_under_its_own_name():
+    for name in _lib.exported_names():
+        assert callable(getattr(_lib, name, None)), name
