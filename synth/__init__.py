@@ -26,9 +26,10 @@ from __future__ import annotations
 
 import math
 import os
+import threading
 from concurrent.futures import ThreadPoolExecutor
-from dataclasses import dataclass, field, replace
-from typing import Dict, List, Optional, Tuple
+from dataclasses import dataclass, replace
+from typing import Dict, Optional, Tuple
 
 import numpy as np
 
@@ -94,9 +95,6 @@ def _normal_pairs(seed: int, first_pair: int, m: int) -> np.ndarray:
     z[0::2] = r * np.cos(ang)
     z[1::2] = r * np.sin(ang)
     return z
-
-
-import threading
 
 
 def _parallel_ok() -> bool:
