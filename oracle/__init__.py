@@ -4,6 +4,8 @@ TEST INFRASTRUCTURE ONLY: imported by ``tests/``, ``__graft_entry__.smoke()`` an
 the ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py``.  The product
 path (``flow_matching_dit_b200``) never imports it, and it never imports the
 product.  See ``oracle/dit.py`` for the sources each function follows.
+``oracle.grad`` (imported on its own: it needs torch) adds the gradients of
+the training loss.
 """
 
 from .dit import (Model, action_decoder, action_encoder, ada_layer_norm, attention,  # noqa: F401
