@@ -190,6 +190,17 @@ def whole_job_rate(world: int, units_per_rank_step: int, steps: int, seconds: fl
     return world * units_per_rank_step * steps / seconds
 
 
+# ------------------------------------------------------------------ the workload both arms report
+
+def throughput_config(w, world: int) -> dict:
+    """The `config` of the JSON line, the same for our arm and the reference arm."""
+    g = w.geom
+    return {"workload": f"DiT action head B={w.batch} S={w.seq} K={w.num_steps} (throughput sweep)",
+            "batch": w.batch, "seq": w.seq, "num_steps": w.num_steps, "layers": g.num_layers, "hidden": g.hidden,
+            "embodiments": g.num_embodiments, "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2 (1.36 GB bf16 weights, 4.3 GB KV cache per call)"}
+
+
 # ------------------------------------------------------------------ reference arm
 
 def run_reference(args, rank):
@@ -220,8 +231,7 @@ def run_reference(args, rank):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "DiT action head B=256 S=256 K=4 (throughput sweep); each step one sampled chunk",
-                   "batch": w.batch, "seq": w.seq, "num_steps": w.num_steps},
+        "config": throughput_config(w, args.gpus),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": f"1 chunk of the B=256 workload per step ({args.steps} steps)"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -373,10 +383,7 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"DiT action head B={w.batch} S={w.seq} K={K} (throughput sweep)", "batch": w.batch,
-                       "seq": w.seq, "num_steps": K, "layers": g.num_layers, "hidden": g.hidden,
-                       "embodiments": g.num_embodiments, "parallelism": f"replicas x{world}",
-                       "l2": "inputs larger than L2 (1.36 GB bf16 weights, 4.3 GB KV cache per call)"},
+            "config": throughput_config(w, world),
             "latency_b1": lat, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": (launches_per_call * args.steps) if launches_per_call else None,
             "clocks": clk,

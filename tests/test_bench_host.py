@@ -70,6 +70,9 @@ def test_reference_arm_prints_one_complete_line(monkeypatch, capsys):
                 "higher_is_better", "scaling", "dtype", "data", "config", "cpu_baseline", "e2e"):
         assert key in d, key
     assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == bench.UNIT
+    assert d["metric"] == bench.METRIC and d["higher_is_better"] is True
+    # the same workload description as our arm's line
+    assert d["config"] == bench.throughput_config(synth.WORKLOADS["tiny"], 1)
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     bench.run_reference(args, rank=1)                     # other ranks print nothing
