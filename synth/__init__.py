@@ -37,7 +37,7 @@ __all__ = [
     "Geometry", "Workload", "GEOM_FULL", "GEOM_TINY", "WORKLOADS", "workload", "make_image_mask",
     "splitmix64_stream", "uniform53", "normal", "randint", "tensor_seed", "fnv1a64",
     "f32_to_bf16_bits", "bf16_bits_to_f32", "weight_shapes", "make_weights",
-    "make_inputs",
+    "make_inputs", "make_training_inputs",
 ]
 
 _GOLDEN = np.uint64(0x9E3779B97F4A7C15)
@@ -344,3 +344,29 @@ def make_inputs(w: Workload, seed: int = 1, batch: Optional[int] = None) -> Dict
         "embodiment_id": ids,
         "init_noise": noise.astype(np.float32).reshape(B, g.action_horizon, g.action_dim),
     }
+
+
+def make_training_inputs(w: Workload, seed: int = 2, batch: Optional[int] = None,
+                         alpha: float = 1.5) -> Dict[str, np.ndarray]:
+    """The random draws of one training step of the action head, which the
+    training objective takes as inputs.
+
+    actions [B,H,A] float32 ~ N(0, 1) (synthetic ground-truth chunks);
+    noise [B,H,A] float32 ~ N(0, 1); t [B] float64 ~ Beta(alpha, 1) (the
+    architecture page draws t from Beta(1.5, 1)), by inverse CDF: Beta(alpha, 1)
+    has CDF x^alpha, so t = u^(1/alpha) for u uniform in [0, 1);
+    action_mask [B,H,A] float32: 1 on the first a_b action dimensions of sample
+    b, a_b uniform in 1..A (embodiments with fewer action dimensions are
+    padded to A, and the padding is masked)."""
+    g = w.geom
+    B = w.batch if batch is None else batch
+    H, A = g.action_horizon, g.action_dim
+    n = B * H * A
+    acts = normal(tensor_seed(seed, "train_actions"), n).astype(np.float32).reshape(B, H, A)
+    noise = normal(tensor_seed(seed, "train_noise"), n).astype(np.float32).reshape(B, H, A)
+    t = uniform53(tensor_seed(seed, "train_t"), B) ** (1.0 / alpha)
+    dims = randint(tensor_seed(seed, "train_action_dims"), B, 1, A)
+    mask = np.zeros((B, H, A), dtype=np.float32)
+    for b in range(B):
+        mask[b, :, : dims[b]] = 1.0
+    return {"actions": acts, "noise": noise, "t": t, "action_mask": mask}

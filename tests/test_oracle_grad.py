@@ -100,3 +100,25 @@ def test_parameters_off_the_path_get_zero_gradient():
     loss, grads = _grads(g, W, inp, acts, np.zeros_like(mask), t)
     assert loss == 0.0
     assert all(not np.any(v) for v in grads.values())
+
+
+def test_gradient_on_the_generators_training_draws():
+    """The training recipe of the input generator (t ~ Beta(1.5, 1), masked
+    action-dimension padding): the gradient still matches central differences."""
+    w = dataclasses.replace(synth.WORKLOADS["tiny"], batch=3, fixed_ids=(1, 0, 1))
+    g = w.geom
+    W = {k: np.asarray(v, np.float64) for k, v in synth.make_weights(g).items()}
+    inp = synth.make_inputs(w, seed=12)
+    tr = synth.make_training_inputs(w, seed=12)
+    args = (g, inp["backbone_features"], inp["vl_mask"], inp["state"], inp["embodiment_id"],
+            tr["actions"], tr["noise"], tr["t"], tr["action_mask"])
+    loss, grads = training_loss_and_grads(W, *args)
+    assert np.isfinite(loss) and loss > 0
+    r = np.random.default_rng(2)
+    d = {k: r.standard_normal(v.shape) * (np.std(v) + 1e-3) for k, v in W.items()}
+    h = 1e-5
+    lp, _ = oracle.training_loss({k: W[k] + h * d[k] for k in W}, *args)
+    lm, _ = oracle.training_loss({k: W[k] - h * d[k] for k in W}, *args)
+    an = sum(float((grads[k] * d[k]).sum()) for k in W)
+    tol_abs = 100 * np.finfo(np.float64).eps * max(abs(lp), abs(lm)) / (2 * h)
+    assert (lp - lm) / (2 * h) == pytest.approx(an, rel=2e-6, abs=tol_abs)

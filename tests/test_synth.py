@@ -98,3 +98,34 @@ def test_inputs_follow_the_workload_recipe(name):
             assert 200 <= sv <= 600
         else:
             assert sv == S
+
+
+def test_training_times_follow_beta_one_and_a_half_one():
+    """t ~ Beta(1.5, 1): CDF x^1.5, mean 1.5 / 2.5 = 0.6, variance
+    1.5 / (2.5^2 * 3.5)."""
+    w = synth.workload("tiny", batch=40000)
+    t = synth.make_training_inputs(w)["t"]
+    n = len(t)
+    assert t.min() >= 0.0 and t.max() < 1.0
+    var = 1.5 / (2.5 ** 2 * 3.5)
+    assert abs(t.mean() - 0.6) < 5 * (var / n) ** 0.5
+    assert abs(t.var() - var) < 0.01 * var + 5e-4
+    for x in (0.1, 0.25, 0.5, 0.75, 0.9):
+        p = x ** 1.5
+        assert abs((t <= x).mean() - p) < 5 * (p * (1 - p) / n) ** 0.5
+
+
+def test_training_inputs_shapes_and_action_mask_prefixes():
+    w = synth.workload("tiny", batch=64)
+    d = synth.make_training_inputs(w)
+    g = w.geom
+    assert d["actions"].shape == d["noise"].shape == d["action_mask"].shape == (64, g.action_horizon, g.action_dim)
+    assert d["t"].shape == (64,)
+    assert not np.array_equal(d["actions"], d["noise"])
+    dims = d["action_mask"][:, 0, :].sum(axis=1).astype(int)
+    assert dims.min() >= 1 and dims.max() <= g.action_dim and len(set(dims)) > 10
+    for b in range(64):
+        assert d["action_mask"][b, :, : dims[b]].all() and not d["action_mask"][b, :, dims[b]:].any()
+    again = synth.make_training_inputs(w)
+    for k in d:
+        np.testing.assert_array_equal(d[k], again[k])
