@@ -251,3 +251,20 @@ def test_device_call_path_validates_then_reaches_the_library(L):
 def test_binding_forwards_every_entry_point_under_its_own_name():
     for name in _lib.exported_names():
         assert callable(getattr(_lib, name, None)), name
+
+
+def test_every_handle_entry_point_rejects_a_null_handle(L):
+    """Checked before anything else (no pointer is dereferenced, no CUDA call)."""
+    E = _lib.GDIT_EINVAL
+    assert L.gdit_prepare(None, 1, 1, 4, _lib.GDIT_BF16, None) == E
+    assert L.gdit_debug_routing(None, None, None, None) == E
+    n = ctypes.c_int()
+    assert L.gdit_debug_kv(None, 0, None, None, ctypes.byref(n)) == E
+    stats = (_lib.gdit_kernel_stat * 4)()
+    assert L.gdit_profile_get_action(None, None, 0, None, None, None, None, 4, None, 1, 1, None, stats, 4) == E
+
+
+def test_gemm_hooks_reject_null_matrices_on_the_host(L):
+    for f in (L.gdit_test_gemm, L.gdit_gemm_static_scratch):
+        assert f(None, None, None, None, 128, 128, 64, 128, 1, None) == _lib.GDIT_EINVAL
+        assert "NULL matrix" in L.gdit_last_error(None).decode()
