@@ -83,8 +83,9 @@ extern "C" {
  * Constraints (else GDIT_EINVAL): num_layers even and >= 2; head_dim 32 or 64;
  * hidden in {128, 256, 512, 1024, 2048}; mlp_hidden, backbone_dim multiples of
  * 64; action_dim and state_dim multiples of 32 and <= 256; action_horizon in
- * [1, 63]; num_embodiments in [1, 64]; time_freq_dim even; max_batch in
- * [1, 4096]; max_backbone_seq >= 1. */
+ * [1, 63]; num_embodiments in [1, 64]; time_freq_dim even and >= 2;
+ * num_timestep_buckets >= 1; ln_eps > 0; max_batch in [1, 4096];
+ * max_backbone_seq in [1, 65536]; attend_text_every_n_blocks >= 0. */
 typedef struct {
   int num_layers, hidden, num_heads, head_dim, mlp_hidden, backbone_dim;
   int action_dim, state_dim, action_horizon, num_embodiments;

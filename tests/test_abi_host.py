@@ -92,6 +92,12 @@ def _create(L, cfg, W):
     ("num_embodiments", 65, "num_embodiments"),
     ("max_batch", 0, "max_batch"),
     ("attend_text_every_n_blocks", -1, "attend_text_every_n_blocks"),
+    ("max_backbone_seq", 65537, "max_backbone_seq"),
+    ("num_timestep_buckets", 0, "num_timestep_buckets"),
+    ("ln_eps", 0.0, "ln_eps"),
+    ("time_freq_dim", 255, "time_freq_dim"),
+    ("head_dim", 128, "head_dim"),
+    ("state_dim", 48, "state_dim"),
 ])
 def test_bad_config_rejected_on_host(L, tinyW, field, value, msg):
     cfg = _cfg(synth.GEOM_TINY, **{field: value})
