@@ -129,3 +129,17 @@ def test_training_inputs_shapes_and_action_mask_prefixes():
     again = synth.make_training_inputs(w)
     for k in d:
         np.testing.assert_array_equal(d[k], again[k])
+
+
+def test_training_draw_uses_the_pages_beta_parameters():
+    """The generator's default t distribution is the printed config's
+    Beta(noise_beta_alpha, noise_beta_beta); its inverse-CDF draw needs beta = 1."""
+    import inspect
+    import json
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "training_time_beta.json")
+    cfg = json.load(open(path))
+    assert cfg["noise_beta_beta"] == 1.0
+    assert inspect.signature(synth.make_training_inputs).parameters["alpha"].default == cfg["noise_beta_alpha"]
+    assert synth.GEOM_FULL.num_timestep_buckets == cfg["num_timestep_buckets"]
+    assert synth.WORKLOADS["sweep256"].num_steps == cfg["num_inference_timesteps"]
