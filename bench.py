@@ -50,6 +50,8 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-profile", action="store_true")
+    p.add_argument("--no-workloads", action="store_true", help="skip the per-workload table")
+    p.add_argument("--workload-calls", type=int, default=30)
     p.add_argument("--oracle-samples", type=int, default=24)
     p.add_argument("--batch", type=int, default=None, help="override the throughput batch (profiling runs)")
     p.add_argument("--seq", type=int, default=None, help="override the throughput backbone length (profiling runs)")
@@ -139,20 +141,51 @@ def time_oracle(W, w, samples: int):
     return samples / dt, cores, dt
 
 
-# ------------------------------------------------------------------ B = 1 roofline
+# ------------------------------------------------------------------ algorithmic work of one call
+
+NOMINAL_BF16_TFLOPS = 2250.0   # B200 dense bf16 tensor peak (spec sheet), for context beside the measured peaks
+
+
+def call_work(g, batch: int, valid_tokens: int, num_steps: int, used_categories: int) -> dict:
+    """Minimum HBM bytes and dense FLOPs of one get_action call.
+
+    Bytes: the bf16 weights each Euler step multiplies by (the 32 DiT blocks
+    without the cross layers' K/V projections, proj_out, and the action
+    encoder and decoder of every category used), once per step; the cross
+    K/V weights and the state encoder (per used category) once per call; the
+    valid backbone tokens read once; the K/V cache written once and read every
+    step; x, the output and the state.  The per-K AdaLN tables and the
+    timestep half of the action encoder's W2 are cached, so not counted.
+    FLOPs: 2 M N K of every dense contraction over the rows that need it
+    (valid tokens for the K/V projection, the B x N token rows in the blocks,
+    the B x H action rows in the encoder, proj_out and decoder), plus
+    attention 4 N Sv D per sample and cross layer and 4 N^2 D per sample and
+    self layer."""
+    D, F, A, L = g.hidden, g.mlp_hidden, g.action_dim, g.num_layers
+    Dvl, Sd, H = g.backbone_dim, g.state_dim, g.action_horizon
+    N = H + 1
+    Lc = L // 2
+    B, tok, K, C = batch, valid_tokens, num_steps, used_categories
+    self_w = 3 * D * D + D * D + 2 * F * D
+    cross_w = 2 * D * D + 2 * F * D
+    enc_w = A * D + D * D + D * D          # W1, W2 (action half), W3
+    dec_w = D * D + D * A
+    step_w = Lc * (self_w + cross_w) + D * D + C * (enc_w + dec_w)
+    once_w = Lc * 2 * D * Dvl + C * (Sd * D + D * D)
+    kv_cache = tok * Lc * 2 * D * 2
+    io = B * H * A * 4 * 2 + B * Sd * 4
+    nbytes = K * step_w * 2 + once_w * 2 + tok * Dvl * 2 + kv_cache * (1 + K) + io
+    rows, arows = B * N, B * H
+    gemm = 2 * tok * (Lc * 2 * D) * Dvl + 2 * B * (Sd * D + D * D)
+    gemm += K * (2 * rows * Lc * (self_w + cross_w) + 2 * arows * (enc_w + D * D + dec_w))
+    attn = K * (Lc * 4 * N * tok * D + Lc * 4 * B * N * N * D)
+    return {"bytes": int(nbytes), "gemm_flops": int(gemm), "attn_flops": int(attn), "weights_per_step": int(step_w * 2)}
+
 
 def b1_algorithmic_bytes(g, seq: int, num_steps: int) -> int:
-    """Minimum HBM bytes of one single-sample call's Euler loop: every step
-    streams the bf16 weights of the 32 DiT blocks (self: Q|K|V, O, FF1, FF2;
-    cross: Q, O, FF1, FF2), of the action encoder (W1, the action half of W2,
-    W3), proj_out and the decoder (one category), and reads the cross layers'
-    K/V cache of `seq` valid tokens."""
-    D, F, A, L = g.hidden, g.mlp_hidden, g.action_dim, g.num_layers
-    self_layer = 3 * D * D + D * D + 2 * F * D
-    cross_layer = 2 * D * D + 2 * F * D
-    head = A * D + D * D + D * D + D * D + D * D + D * A
-    kv = (L // 2) * 2 * seq * D * 2
-    return num_steps * (((L // 2) * (self_layer + cross_layer) + head) * 2 + kv)
+    """Minimum HBM bytes of one single-sample call (one category, `seq` valid
+    backbone tokens): call_work's count."""
+    return call_work(g, 1, seq, num_steps, 1)["bytes"]
 
 
 def latency_roofline(g, seq: int, num_steps: int, p50_ms: float, hbm_gbs: float) -> dict:
@@ -161,6 +194,21 @@ def latency_roofline(g, seq: int, num_steps: int, p50_ms: float, hbm_gbs: float)
     ach = b / (p50_ms / 1e3) / 1e9
     return {"bound": "hbm", "algorithmic_bytes": b, "achieved": ach, "peak": hbm_gbs, "unit": "GB/s",
             "frac": ach / hbm_gbs}
+
+
+def workload_roofline(work: dict, batch: int, mean_ms: float, peaks) -> dict:
+    """Roofline of a whole call: weight streaming (HBM) for batches of at most
+    8 samples, tensor cores (dense bf16 GEMM FLOPs) from 32 up."""
+    hbm, tf_burst, tf_sus, src = peaks
+    sec = mean_ms / 1e3
+    if batch <= 8:
+        ach = work["bytes"] / sec / 1e9
+        return {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                "peak_kind": f"HBM copy ({src})"}
+    ach = work["gemm_flops"] / sec / 1e12
+    return {"bound": "tensor", "achieved": ach, "peak": tf_burst, "unit": "TFLOP/s", "frac": ach / tf_burst,
+            "frac_of_sustained": ach / tf_sus, "frac_of_nominal": ach / NOMINAL_BF16_TFLOPS,
+            "peak_kind": f"burst bf16 ({src})"}
 
 
 # ------------------------------------------------------------------ replicas (one per GPU, no data-path collective)
@@ -241,6 +289,27 @@ def run_reference(args, rank):
 
 # ------------------------------------------------------------------ our arm
 
+# every workload of the task, timed one call after the other (inputs resident in HBM)
+WORKLOAD_TABLE = ("latency", "sweep1", "sweep8", "sweep32", "sweep128", "sweep256", "batched", "long_chunk")
+
+
+def time_calls(head, d, K, out, stream, calls: int, warmup: int):
+    """Device time of each of `calls` consecutive calls (CUDA events on the
+    launching stream between calls) and of all of them together, in ms."""
+    import torch
+    for _ in range(warmup):
+        head.get_action(*d, num_steps=K, out=out)
+    torch.cuda.synchronize()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(calls + 1)]
+    evs[0].record(stream)
+    for i in range(calls):
+        head.get_action(*d, num_steps=K, out=out)
+        evs[i + 1].record(stream)
+    torch.cuda.synchronize()
+    per = [evs[i].elapsed_time(evs[i + 1]) for i in range(calls)]
+    return per, evs[0].elapsed_time(evs[-1])
+
+
 def main():
     args = parse()
     rank, world, local = ranks_from_env()
@@ -263,7 +332,10 @@ def main():
     g = w.geom
     W = synth.make_weights(g)
     max_seq = max(w.seq, wl.seq) if args.latency_calls > 0 else w.seq
-    head = ActionHead(g, W, max_batch=w.batch, max_seq=max_seq, device=local)
+    if not args.no_workloads:
+        max_seq = max(max_seq, max(synth.WORKLOADS[n].seq for n in WORKLOAD_TABLE if n != "long_chunk"))
+    head = ActionHead(g, W, max_batch=max(w.batch, 256 if not args.no_workloads else 1), max_seq=max_seq,
+                      device=local)
 
     def dev_inputs(wk, seed):
         inp = synth.make_inputs(wk, seed=seed)
@@ -322,6 +394,33 @@ def main():
                "workload": "B=1, backbone [1,300,2048] bf16 all valid, id 0, K=4"}
         lat["roofline"] = latency_roofline(wl.geom, wl.seq, wl.num_steps, lat["p50_ms"], load_peaks()[0])
 
+    # ---- every workload: chunks/s, p50/p99 per call, roofline of the whole call
+    table = None
+    if rank == 0 and not args.no_workloads:
+        table = {}
+        peaks = load_peaks()
+        for name in WORKLOAD_TABLE:
+            wk = synth.WORKLOADS[name]
+            hw = head
+            if wk.geom != g:     # another horizon: a handle of its own
+                hw = ActionHead(wk.geom, W, max_batch=wk.batch, max_seq=wk.seq, device=local)
+            winp, dw = dev_inputs(wk, 1)
+            outw = torch.empty_like(dw[4])
+            per, total_ms = time_calls(hw, dw, wk.num_steps, outw, stream, args.workload_calls, 5)
+            assert hw.sync_status() == 0
+            if hw is not head:
+                hw.close()
+            work = call_work(wk.geom, wk.batch, int(winp["vl_mask"].sum()), wk.num_steps,
+                             len(set(winp["embodiment_id"].tolist())))
+            mean_ms = total_ms / len(per)
+            table[name] = {
+                "workload": wk.description, "batch": wk.batch, "seq": wk.seq, "horizon": wk.geom.action_horizon,
+                "num_steps": wk.num_steps, "chunks_per_s": wk.batch / (mean_ms / 1e3),
+                "p50_ms": float(np.percentile(per, 50)), "p99_ms": float(np.percentile(per, 99)),
+                "mean_ms": mean_ms, "calls": len(per), "algorithmic_bytes": work["bytes"],
+                "gemm_flops": work["gemm_flops"], "attn_flops": work["attn_flops"],
+                "roofline": workload_roofline(work, wk.batch, mean_ms, peaks)}
+
     # ---- end to end through the host-buffer entry point (pinned host memory)
     e2e = None
     if not args.no_e2e:
@@ -361,8 +460,11 @@ def main():
             traffic = json.load(open(tpath)).get(top["name"])
         if top["name"].startswith("gemm"):
             ach = top["flops"] / (top["total_ms"] / 1e3) / 1e12
-            roof = {"bound": "tensor", "kernel": top["name"], "achieved": ach, "peak": tf_sus, "unit": "TFLOP/s",
-                    "frac": ach / tf_sus, "frac_of_burst": ach / tf_burst, "peak_kind": f"sustained bf16 ({src})",
+            # each launch is timed on its own (events around it, one eager call of
+            # about 40 ms): the burst peak is the denominator
+            roof = {"bound": "tensor", "kernel": top["name"], "achieved": ach, "peak": tf_burst, "unit": "TFLOP/s",
+                    "frac": ach / tf_burst, "frac_of_sustained": ach / tf_sus,
+                    "frac_of_nominal": ach / NOMINAL_BF16_TFLOPS, "peak_kind": f"burst bf16 ({src})",
                     "traffic": traffic, "launches": top["launches"], "ms": top["total_ms"]}
         else:
             ach = top["bytes"] / (top["total_ms"] / 1e3) / 1e9
@@ -384,7 +486,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": throughput_config(w, world),
-            "latency_b1": lat, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "latency_b1": lat, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "workloads": table,
             "gpu_launches": (launches_per_call * args.steps) if launches_per_call else None,
             "clocks": clk,
         }

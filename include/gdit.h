@@ -274,12 +274,14 @@ int gdit_test_gemm(const void* A, const void* B, const float* bias, float* C,
  * which every GPU that loads the library keeps until the process exits.
  * Limits (else GDIT_EINVAL): ceil(M/128) * ceil(N/bn) <= 4096 and, when
  * splits > 1, splits * M * N <= 1048576.
- * The first call on each device looks up the array's device address; make
- * that first call before any stream capture on that device.  Every call
- * shares the array and leaves its contents behind: calls that overlap on the
- * GPU (several streams, several host threads) race and give wrong results.
- * The call clears the status word and the counters itself, then synchronizes
- * cuda_stream.  Returns GDIT_OK, GDIT_EINVAL or GDIT_ETIMEOUT. */
+ * Set-up: the first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture begins on that device.  Every call shares the
+ * array and leaves its contents behind: calls that overlap on the GPU
+ * (several streams, several host threads) race and give wrong results.  Each
+ * call clears the status word and the tile counters on cuda_stream, launches
+ * the GEMM, reads the status word back and synchronizes cuda_stream before it
+ * returns.  Returns GDIT_OK, GDIT_EINVAL or GDIT_ETIMEOUT. */
 int gdit_gemm_static_scratch(const void* A, const void* B, const float* bias, float* C,
                              int M, int N, int K, int bn, int splits, void* cuda_stream);
 

@@ -15,44 +15,96 @@ import bench  # noqa: E402
 import synth  # noqa: E402
 
 
-def _bytes_from_weight_table(g, seq, K):
-    """Every step streams each bf16 weight matrix that the loop multiplies by,
-    for one category: all block matrices except the cross layers' K/V
-    projections (applied once per call to the backbone), the action encoder
-    with only the action half of W2 (its timestep half is a per-K table),
-    proj_out and the decoder.  Plus the cross layers' K/V cache reads."""
+def _count_from_weight_table(g, batch, tok, K, used):
+    """Bytes and GEMM FLOPs of one call, counted matrix by matrix from the
+    weight table.  Every step streams each bf16 weight matrix that the loop
+    multiplies by (category matrices once per used category): all block
+    matrices except the cross layers' K/V projections (applied once per call to
+    the valid backbone tokens), the action encoder with only the action half
+    of W2 (its timestep half is a per-K table), proj_out and the decoder.  Once
+    per call: the cross K/V weights and the state encoder.  Plus the valid
+    backbone tokens, the K/V cache written once and read every step, and the
+    f32 noise, output and state.  FLOPs are 2 x rows x params of every
+    matrix, rows being the valid tokens (K/V), the B x N token rows (block
+    matrices), B (state encoder) or the B x H action rows (the rest)."""
     shapes = synth.weight_shapes(g)
-    n = 0
+    N, H = g.action_horizon + 1, g.action_horizon
+    step = once = 0
+    flops = 0
     for name, shp in shapes.items():
         parts = name.split(".")
         if name.startswith("blk") and name.endswith(".w") and parts[1] in ("q", "k", "v", "o", "ff1", "ff2"):
-            layer = int(parts[0][3:])
-            if layer % 2 == 0 and parts[1] in ("k", "v"):
-                continue
-            n += int(np.prod(shp))
+            n = int(np.prod(shp))
+            if int(parts[0][3:]) % 2 == 0 and parts[1] in ("k", "v"):
+                once += n
+                flops += 2 * tok * n
+            else:
+                step += n
+                flops += K * 2 * batch * N * n
         elif name in ("act_enc.W1.W", "act_enc.W3.W", "act_dec.l1.W", "act_dec.l2.W"):
-            n += int(np.prod(shp[1:]))
+            n = int(np.prod(shp[1:]))
+            step += used * n
+            flops += K * 2 * batch * H * n
         elif name == "act_enc.W2.W":
-            n += int(np.prod(shp[1:])) // 2
+            n = int(np.prod(shp[1:])) // 2
+            step += used * n
+            flops += K * 2 * batch * H * n
         elif name == "out.proj.w":
-            n += int(np.prod(shp))
-    kv = (g.num_layers // 2) * 2 * seq * g.hidden * 2
-    return K * (2 * n + kv)
+            n = int(np.prod(shp))
+            step += n
+            flops += K * 2 * batch * H * n
+        elif name in ("state_enc.l1.W", "state_enc.l2.W"):
+            n = int(np.prod(shp[1:]))
+            once += used * n
+            flops += 2 * batch * n
+    kv = tok * (g.num_layers // 2) * 2 * g.hidden * 2
+    io = 2 * batch * H * g.action_dim * 4 + batch * g.state_dim * 4
+    nbytes = 2 * (K * step + once) + tok * g.backbone_dim * 2 + (1 + K) * kv + io
+    return nbytes, flops
 
 
-@pytest.mark.parametrize("name", ["latency", "tiny"])
-def test_b1_algorithmic_bytes_match_the_weight_table(name):
+@pytest.mark.parametrize("name", ["latency", "tiny", "sweep256", "batched", "long_chunk"])
+def test_call_work_matches_the_weight_table(name):
     w = synth.WORKLOADS[name]
-    assert bench.b1_algorithmic_bytes(w.geom, w.seq, w.num_steps) == _bytes_from_weight_table(w.geom, w.seq, w.num_steps)
+    inp = synth.make_inputs(w) if name != "sweep256" else None
+    B = w.batch
+    tok = int(inp["vl_mask"].sum()) if inp is not None else B * w.seq
+    used = len(set(inp["embodiment_id"].tolist())) if inp is not None else 32
+    got = bench.call_work(w.geom, B, tok, w.num_steps, used)
+    nbytes, flops = _count_from_weight_table(w.geom, B, tok, w.num_steps, used)
+    assert got["bytes"] == nbytes
+    assert got["gemm_flops"] == flops
 
 
 def test_b1_bytes_of_the_latency_workload():
+    """4 x 746.7 MB of step weights + 134.2 MB of cross K/V weights + 2.2 MB of
+    state encoder + 1.2 MB of backbone tokens + the K/V cache (19.7 MB) written
+    once and read 4 times."""
     w = synth.WORKLOADS["latency"]
     b = bench.b1_algorithmic_bytes(w.geom, w.seq, w.num_steps)
-    assert b == 3_065_511_936            # 4 x (746.7 MB weights + 19.7 MB K/V)
+    assert b == 3_222_851_840
     r = bench.latency_roofline(w.geom, w.seq, w.num_steps, 4.73, 6452.8)
     assert r["frac"] == pytest.approx(b / 4.73e-3 / 1e9 / 6452.8)
     assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+
+
+def test_sweep256_flops_split():
+    """B = 256, S = 256: the K/V projection is 2 x 65536 x 32768 x 2048 =
+    8.80 TFLOP and the whole call 21.79 TFLOP of dense GEMM."""
+    w = synth.WORKLOADS["sweep256"]
+    got = bench.call_work(w.geom, 256, 256 * 256, 4, 32)
+    assert 2 * 65536 * 32768 * 2048 == 8_796_093_022_208
+    assert got["gemm_flops"] == pytest.approx(21.787e12, rel=1e-3)
+
+
+def test_workload_roofline_picks_the_bound():
+    peaks = (6452.8, 1676.2, 1404.4, "measured")
+    work = {"bytes": 3.2e9, "gemm_flops": 2.0e13}
+    r = bench.workload_roofline(work, 8, 2.0, peaks)
+    assert r["bound"] == "hbm" and r["frac"] == pytest.approx(3.2e9 / 2e-3 / 1e9 / 6452.8)
+    r = bench.workload_roofline(work, 32, 20.0, peaks)
+    assert r["bound"] == "tensor" and r["frac"] == pytest.approx(2e13 / 20e-3 / 1e12 / 1676.2)
+    assert r["frac_of_nominal"] == pytest.approx(2e13 / 20e-3 / 1e12 / 2250.0)
 
 
 def test_reference_arm_prints_one_complete_line(monkeypatch, capsys):

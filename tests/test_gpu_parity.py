@@ -219,28 +219,50 @@ def test_cross_kv_projection_matches_oracle(head_full, full_model):
             np.testing.assert_allclose(got, ref, rtol=2 ** -8, atol=1e-3)
 
 
-def test_batched_workload_sampled(head_full, full_weights, full_model):
+def rows_one_per_embodiment(ids):
+    """The first batch row of every embodiment id present, in row order: each
+    category's segment of the grouped GEMMs is compared at least once."""
+    ids = np.asarray(ids).reshape(-1)
+    first = {}
+    for r, c in enumerate(ids.tolist()):
+        first.setdefault(c, r)
+    return sorted(first.values())
+
+
+def test_batched_workload_every_row(head_full, full_weights, full_model):
+    """B = 32, ragged valid lengths 200..600 padded to 600: every row, so every
+    sample's packed key range and every category segment is compared."""
     w = synth.WORKLOADS["batched"]
     inp = synth.make_inputs(w)
     gpu, st = run_gpu(head_full, inp, w.num_steps)
     assert st == 0
-    rows = [0, 13, 27, 31]
+    rows = list(range(w.batch))
     ref = run_oracle(full_weights, w.geom, inp, w.num_steps, samples=rows, model=full_model)
-    assert_parity(gpu[rows], ref, inp["init_noise"][rows], "batched B=32 S<=600 (rows 0,13,27,31)")
+    assert_parity(gpu, ref, inp["init_noise"], "batched B=32 S<=600 (all rows)")
 
 
-def test_sweep256_workload_sampled(head_full, full_weights, full_model):
-    w = synth.WORKLOADS["sweep256"]
+@pytest.mark.parametrize("name", ["sweep8", "sweep32", "sweep128", "sweep256"])
+def test_sweep_workloads(head_full, full_weights, full_model, name):
+    """The throughput sweep at S = 256: every row up to B = 32; at B = 128 and
+    256 one row of every embodiment (all 32 categories occur), so every
+    segment of the grouped per-embodiment GEMMs, and the 128-row tiles that
+    straddle segment boundaries, feed a compared row."""
+    w = synth.WORKLOADS[name]
     inp = synth.make_inputs(w)
     gpu, st = run_gpu(head_full, inp, w.num_steps)
     assert st == 0
     assert np.isfinite(gpu).all()
-    rows = [0, 100, 255]
+    if w.batch <= 32:
+        rows = list(range(w.batch))
+    else:
+        rows = rows_one_per_embodiment(inp["embodiment_id"])
+        assert sorted(set(inp["embodiment_id"][rows].tolist())) == list(range(32))
     ref = run_oracle(full_weights, w.geom, inp, w.num_steps, samples=rows, model=full_model)
-    assert_parity(gpu[rows], ref, inp["init_noise"][rows], "sweep B=256 (rows 0,100,255)")
+    assert_parity(gpu[rows], ref, inp["init_noise"][rows], f"{name} ({len(rows)} rows)")
 
 
-def test_long_chunk_workload_sampled(full_weights):
+def test_long_chunk_workload_every_row(full_weights, full_model):
+    """B = 8, H = 50 (51 tokens per sample), S = 512, K = 8: every row."""
     require_gpu()
     from flow_matching_dit_b200 import ActionHead
     w = synth.WORKLOADS["long_chunk"]
@@ -248,9 +270,10 @@ def test_long_chunk_workload_sampled(full_weights):
     with ActionHead(w.geom, full_weights, max_batch=8, max_seq=512) as head:
         gpu, st = run_gpu(head, inp, w.num_steps)
     assert st == 0
-    rows = [5]
-    ref = run_oracle(full_weights, w.geom, inp, w.num_steps, samples=rows)
-    assert_parity(gpu[rows], ref, inp["init_noise"][rows], "long chunk B=8 H=50 K=8 (row 5)")
+    rows = list(range(w.batch))
+    model = oracle.Model(full_weights, w.geom)
+    ref = run_oracle(full_weights, w.geom, inp, w.num_steps, samples=rows, model=model)
+    assert_parity(gpu, ref, inp["init_noise"], "long chunk B=8 H=50 K=8 (all rows)")
 
 
 # ---------------------------------------------------------------- single-sample persistent loop

@@ -26,15 +26,22 @@ def _inputs(M, N, K, seed):
     return A, B, bias
 
 
-def test_two_calls_match_the_allocating_entry_point():
+@pytest.mark.parametrize("M, N, K, bn, splits, seed", [
+    (17, 1024, 1024, 64, 4, 1),       # split-K: partials and tile counters in the fixed array
+    (65, 512, 768, 128, 3, 2),
+    (300, 1024, 512, 128, 1, 4),      # one split: the direct epilogue, no partials
+])
+def test_two_calls_in_a_row_match_the_allocating_entry_point(M, N, K, bn, splits, seed):
+    """Two calls in a row on the same inputs: the second starts from the
+    scratch contents the first left behind and must give the same result."""
     require_gpu()
     from flow_matching_dit_b200 import gemm_static_scratch, test_gemm
-    for (M, N, K, bn, splits, seed) in ((17, 1024, 1024, 64, 4, 1), (65, 512, 768, 128, 3, 2)):
-        A, B, bias = _inputs(M, N, K, seed)
-        ref = test_gemm(A, B, bias, bn=bn, splits=splits).cpu().double().numpy()
+    A, B, bias = _inputs(M, N, K, seed)
+    ref = test_gemm(A, B, bias, bn=bn, splits=splits).cpu().double().numpy()
+    exact = A.cpu().double().numpy() @ B.cpu().double().numpy().T + bias.cpu().double().numpy()
+    for _ in range(2):
         got = gemm_static_scratch(A, B, bias, bn=bn, splits=splits).cpu().double().numpy()
         np.testing.assert_allclose(got, ref, rtol=1e-5, atol=2e-5 * np.sqrt(K))
-        exact = A.cpu().double().numpy() @ B.cpu().double().numpy().T + bias.cpu().double().numpy()
         np.testing.assert_allclose(got, exact, rtol=1e-5, atol=2e-5 * np.sqrt(K))
 
 
@@ -45,4 +52,8 @@ def test_sizes_beyond_the_fixed_array_are_rejected():
     A, B, bias = _inputs(512, 4096, 512, 3)          # 4 splits x 512 x 4096 floats > 2^20
     with pytest.raises(GditError) as e:
         gemm_static_scratch(A, B, bias, bn=64, splits=4)
+    assert e.value.code == GDIT_EINVAL
+    A, B, bias = _inputs(128 * 65, 4096, 64, 5)      # 65 x 64 = 4160 output tiles > 4096 counters
+    with pytest.raises(GditError) as e:
+        gemm_static_scratch(A, B, bias, bn=64, splits=1)
     assert e.value.code == GDIT_EINVAL
