@@ -52,7 +52,7 @@ def parse():
     p.add_argument("--no-profile", action="store_true")
     p.add_argument("--no-workloads", action="store_true", help="skip the per-workload table")
     p.add_argument("--workload-calls", type=int, default=30)
-    p.add_argument("--oracle-samples", type=int, default=24)
+    p.add_argument("--oracle-samples", type=int, default=4)
     p.add_argument("--batch", type=int, default=None, help="override the throughput batch (profiling runs)")
     p.add_argument("--seq", type=int, default=None, help="override the throughput backbone length (profiling runs)")
     return p.parse_args()
@@ -117,28 +117,19 @@ class Clocks:
 # ------------------------------------------------------------------ CPU oracle
 
 def time_oracle(W, w, samples: int):
-    """The fp64 oracle, as it stands, on `samples` batch rows of workload w
-    (one untimed row first: it converts the weights it touches)."""
-    import oracle
-    try:
-        from threadpoolctl import threadpool_info
-    except Exception:
-        threadpool_info = None
+    """The C++ CPU oracle (its float instantiation, as it stands) on `samples`
+    batch rows of workload w, on all host cores.  The weights are converted to
+    float once, outside the timed region.  Returns (chunks/s, threads, s)."""
+    from oracle import cpp_oracle
     inp = synth.make_inputs(w)
-    model = oracle.Model(W, w.geom)
+    prep = cpp_oracle.Weights(W, w.geom, np.float32)
     args = (W, w.geom, inp["backbone_features"], inp["vl_mask"], inp["state"], inp["embodiment_id"],
             inp["init_noise"], w.num_steps)
-    oracle.get_action(*args, samples=[0], model=model)
-    rows = list(range(1, 1 + samples))
+    rows = list(range(samples))
     t0 = time.perf_counter()
-    oracle.get_action(*args, samples=rows, model=model)
+    cpp_oracle.get_action(*args, samples=rows, dtype=np.float32, prepared=prep)
     dt = time.perf_counter() - t0
-    cores = os.cpu_count() or 1
-    if threadpool_info is not None:
-        n = [p.get("num_threads", 0) for p in threadpool_info() if p.get("user_api") == "blas"]
-        if n:
-            cores = max(n)
-    return samples / dt, cores, dt
+    return samples / dt, cpp_oracle.max_threads(), dt
 
 
 # ------------------------------------------------------------------ algorithmic work of one call
@@ -232,6 +223,36 @@ def max_over_ranks(x: float, world: int, device) -> float:
     return float(t.item())
 
 
+def shard_rows(global_batch: int, rank: int, world: int):
+    """Rows [start, stop) of a global batch that `rank` serves: contiguous,
+    sizes differing by at most one, earlier ranks taking the extra rows."""
+    base, extra = divmod(global_batch, world)
+    start = rank * base + min(rank, extra)
+    return start, start + base + (1 if rank < extra else 0)
+
+
+def gather_rows(local, global_batch: int, world: int):
+    """The ranks' slices of a batch-major tensor (rows as shard_rows gives
+    them) put back together on every rank: one all_gather of equal-sized,
+    zero-padded slices.  Samples are independent, so this is the only
+    collective the batch-sharded path needs, and it is outside the timed
+    region."""
+    import torch
+    import torch.distributed as dist
+    if world <= 1:
+        return local
+    cap = -(-global_batch // world)
+    pad = torch.zeros((cap,) + tuple(local.shape[1:]), dtype=local.dtype, device=local.device)
+    pad[: local.shape[0]] = local
+    parts = [torch.empty_like(pad) for _ in range(world)]
+    dist.all_gather(parts, pad)
+    out = []
+    for r in range(world):
+        a, b = shard_rows(global_batch, r, world)
+        out.append(parts[r][: b - a])
+    return torch.cat(out)
+
+
 def whole_job_rate(world: int, units_per_rank_step: int, steps: int, seconds: float) -> float:
     """Units per second of the whole job: every rank processed
     units_per_rank_step units in each of `steps` steps, within `seconds`."""
@@ -252,36 +273,33 @@ def throughput_config(w, world: int) -> dict:
 # ------------------------------------------------------------------ reference arm
 
 def run_reference(args, rank):
+    """The reference arm: the C++ CPU oracle (float instantiation, all host
+    cores), one chunk of the throughput workload per step."""
     if rank != 0:
         return
+    from oracle import cpp_oracle
     w = synth.WORKLOADS[THROUGHPUT]
     W = synth.make_weights(w.geom)
-    samples = 1
-    times = []
-    import oracle
     inp = synth.make_inputs(w)
-    model = oracle.Model(W, w.geom)
+    prep = cpp_oracle.Weights(W, w.geom, np.float32)
     a = (W, w.geom, inp["backbone_features"], inp["vl_mask"], inp["state"], inp["embodiment_id"],
          inp["init_noise"], w.num_steps)
+    times = []
     for i in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        oracle.get_action(*a, samples=[i % w.batch], model=model)
+        cpp_oracle.get_action(*a, samples=[i % w.batch], dtype=np.float32, prepared=prep)
         if i >= args.warmup:
             times.append(time.perf_counter() - t0)
     per = float(np.mean(times))
-    value = samples / per
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([p.get("num_threads", 0) for p in threadpool_info() if p.get("user_api") == "blas"] or [os.cpu_count()])
-    except Exception:
-        cores = os.cpu_count()
+    value = 1.0 / per
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": throughput_config(w, args.gpus),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"1 chunk of the B=256 workload per step ({args.steps} steps)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpp_oracle.max_threads(), "kind": "oracle",
+                         "sample": f"1 chunk of the B={w.batch} workload per step ({args.steps} steps), "
+                                   "C++ oracle, float"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -371,6 +389,12 @@ def main():
     assert head.sync_status() == 0
     ms_per_step = ms / args.steps
     value = whole_job_rate(world, w.batch, args.steps, ms / 1e3)
+    if world > 1:
+        # the job's global batch is world x B rows, rank r serving rows
+        # shard_rows(world * B, r, world); its actions are gathered once,
+        # outside the timed region
+        gathered = gather_rows(out, world * w.batch, world)
+        assert gathered.shape[0] == world * w.batch
 
     # ---- B = 1 latency (device inputs, one call at a time)
     lat = None
@@ -477,8 +501,8 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, secs = time_oracle(W, w, args.oracle_samples)
         cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
-               "sample": f"{args.oracle_samples} chunks of the B=256 workload (rows 1..{args.oracle_samples}), "
-                         f"fp64 numpy, {secs:.1f} s"}
+               "sample": f"{args.oracle_samples} chunks of the B={w.batch} workload (rows 0..{args.oracle_samples - 1}), "
+                         f"C++ oracle (float, OpenMP), {secs:.1f} s"}
 
     if rank == 0:
         line = {
