@@ -27,6 +27,7 @@ GDIT_FLAG_STRICT_PROFILES = 1
 GDIT_FLAG_NO_GRAPH = 2
 GDIT_FLAG_NO_SMALL = 4
 GDIT_FLAG_NO_TMA_STORE = 8
+GDIT_FLAG_NO_PAIR = 16
 
 
 class gdit_config(ctypes.Structure):

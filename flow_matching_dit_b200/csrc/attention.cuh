@@ -137,6 +137,133 @@ __device__ __forceinline__ void attn_init(float (&o)[MT][DH / 8][4], float (&mro
   }
 }
 
+// One 16-key chunk (keys key0 .. key0 + 15 of the list [k_begin, k_begin +
+// n_keys)) folded into (o, mrow, lrow) with an online softmax (base 2).  The
+// chunk's K and V rows sit in shared memory: kaddr(r, c) / vaddr(r, c) give
+// the address of 16-byte column chunk c of row r (0..15) of the chunk.  Keys
+// past n_keys (and, with a.ksel >= 0, keys of the other kind) get -inf; their
+// V rows must hold finite values.
+template <int MT, int DH, typename KAddr, typename VAddr>
+__device__ __forceinline__ void attn_fold_chunk(const AttnArgs& a, int key0, int k_begin, int n_keys,
+                                                const __nv_bfloat16* sQ, KAddr kaddr, VAddr vaddr,
+                                                float (&o)[MT][DH / 8][4], float (&mrow)[MT][2],
+                                                float (&lrow)[MT][2]) {
+  constexpr int ROW = DH + 8;
+  const int lane = threadIdx.x & 31;
+  const int tig = lane & 3;    // thread in group
+  // the keys of this lane's score columns that the layer keeps (bit nt * 2 + j)
+  uint32_t keep = 0xFu;
+  if (a.ksel >= 0) {
+    keep = 0u;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int key = key0 + nt * 8 + tig * 2 + j;
+        if (key < n_keys && (int)__ldg(a.kflag + k_begin + key) == a.ksel) keep |= 1u << (nt * 2 + j);
+      }
+  }
+
+  // S = Q K^T for 16 keys (two n-tiles of 8).  Even and odd k-steps go to
+  // separate accumulators: a dependent chain of mma.sync is bound by its
+  // latency, and this halves the chain.
+  float s[MT][2][4], s1[MT][2][4];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        s[mt][nt][j] = 0.0f;
+        s1[mt][nt][j] = 0.0f;
+      }
+#pragma unroll
+  for (int ks = 0; ks < DH / 16; ++ks) {
+    // K fragments of both 8-key tiles in one ldmatrix: lanes 0-7 keys 0-7
+    // (k 0-7), 8-15 keys 0-7 (k 8-15), 16-23 keys 8-15 (k 0-7), 24-31 keys 8-15 (k 8-15)
+    uint32_t kb[2][2];
+    ldmatrix_x4(kb[0][0], kb[0][1], kb[1][0], kb[1][1],
+                kaddr((lane & 7) + ((lane >> 4) << 3), ks * 2 + ((lane >> 3) & 1)));
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      // Q fragments: lane supplies row (lane & 15) of the tile, k half (lane >> 4)
+      uint32_t a0, a1, a2, a3;
+      ldmatrix_x4(a0, a1, a2, a3, sQ + (mt * 16 + (lane & 15)) * ROW + ks * 16 + (lane >> 4) * 8);
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+        mma_bf16_16816((ks & 1) ? s1[mt][nt] : s[mt][nt], a0, a1, a2, a3, kb[nt][0], kb[nt][1]);
+    }
+  }
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) s[mt][nt][j] += s1[mt][nt][j];
+
+  // online softmax (base 2); masked keys get -inf.  Row groups of 8 with no
+  // query (past n_tok: zero Q rows, never stored) are skipped.
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {   // hr 0: row g, hr 1: row g + 8
+      if (mt * 16 + hr * 8 >= a.n_tok) continue;
+      float x[4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int key = key0 + nt * 8 + tig * 2 + j;
+          x[nt * 2 + j] = (key < n_keys && ((keep >> (nt * 2 + j)) & 1u)) ? s[mt][nt][hr * 2 + j] * a.scale_log2
+                                                                           : -INFINITY;
+        }
+      float cm = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+      cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 1));
+      cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 2));
+      const float m_old = mrow[mt][hr];
+      const float m_new = fmaxf(m_old, cm);
+      const float alpha = (m_new == -INFINITY) ? 1.0f : ex2_approx(m_old - m_new);
+      float psum = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float p = (m_new == -INFINITY) ? 0.0f : ex2_approx(x[j] - m_new);
+        x[j] = p;
+        psum += p;
+      }
+      mrow[mt][hr] = m_new;
+      lrow[mt][hr] = lrow[mt][hr] * alpha + psum;
+#pragma unroll
+      for (int nd = 0; nd < DH / 8; ++nd) {
+        o[mt][nd][hr * 2 + 0] *= alpha;
+        o[mt][nd][hr * 2 + 1] *= alpha;
+      }
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        s[mt][nt][hr * 2 + 0] = x[nt * 2 + 0];
+        s[mt][nt][hr * 2 + 1] = x[nt * 2 + 1];
+      }
+    }
+  }
+
+  // O += P V : P (16 x 16 keys) from the score accumulators, V via ldmatrix.trans
+#pragma unroll
+  for (int nd2 = 0; nd2 < DH / 16; ++nd2) {   // pairs of 8-wide dim tiles
+    uint32_t vb0, vb1, vb2, vb3;
+    const int r = lane & 7;
+    const int mtx = lane >> 3;          // matrix 0..3: (keys 0-7 | 8-15) x (dims nd | nd+1)
+    ldmatrix_x4_trans(vb0, vb1, vb2, vb3, vaddr((mtx & 1) * 8 + r, nd2 * 2 + (mtx >> 1)));
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      const uint32_t a0 = pack_bf16x2(s[mt][0][0], s[mt][0][1]);
+      const uint32_t a1 = pack_bf16x2(s[mt][0][2], s[mt][0][3]);
+      const uint32_t a2 = pack_bf16x2(s[mt][1][0], s[mt][1][1]);
+      const uint32_t a3 = pack_bf16x2(s[mt][1][2], s[mt][1][3]);
+      mma_bf16_16816(o[mt][nd2 * 2 + 0], a0, a1, a2, a3, vb0, vb1);
+      mma_bf16_16816(o[mt][nd2 * 2 + 1], a0, a1, a2, a3, vb2, vb3);
+    }
+  }
+}
+
 // One warp: chunks c0, c0 + cstep, ... of the keys [k_begin, k_begin + n_keys)
 // of head h, folded into (o, mrow, lrow) with an online softmax.
 template <int MT, int DH, int RING_ = 3>
@@ -148,8 +275,6 @@ __device__ __forceinline__ void attn_stream_chunks(const AttnArgs& a, int h, int
   constexpr int ROW = SM::ROW;
   constexpr int PIECES = DH / 8;
   const int lane = threadIdx.x & 31;
-  const int g = lane >> 2;     // row group of the mma fragments
-  const int tig = lane & 3;    // thread in group
   const int n_chunks = (n_keys + 15) >> 4;
   const __nv_bfloat16* kbase = a.k + h * a.kv_head_stride;
   const __nv_bfloat16* vbase = a.v + h * a.kv_head_stride;
@@ -200,108 +325,13 @@ __device__ __forceinline__ void attn_stream_chunks(const AttnArgs& a, int h, int
     }
     cp_async_wait<SM::RING - 1>();
     __syncwarp();
-    // the keys of this lane's score columns that the layer keeps (bit nt * 2 + j)
-    uint32_t keep = 0xFu;
-    if (a.ksel >= 0) {
-      keep = 0u;
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int key = chunk * 16 + nt * 8 + tig * 2 + j;
-          if (key < n_keys && (int)__ldg(a.kflag + k_begin + key) == a.ksel) keep |= 1u << (nt * 2 + j);
-        }
-    }
     const __nv_bfloat16* sk = ring + (it % SM::RING) * 2 * SM::CHUNK_ELEMS;
     const __nv_bfloat16* sv = sk + SM::CHUNK_ELEMS;
-
-    // S = Q K^T for 16 keys (two n-tiles of 8)
-    float s[MT][2][4];
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) s[mt][nt][j] = 0.0f;
-#pragma unroll
-    for (int ks = 0; ks < DH / 16; ++ks) {
-      // K fragments of both 8-key tiles in one ldmatrix: lanes 0-7 keys 0-7
-      // (k 0-7), 8-15 keys 0-7 (k 8-15), 16-23 keys 8-15 (k 0-7), 24-31 keys 8-15 (k 8-15)
-      uint32_t kb[2][2];
-      ldmatrix_x4(kb[0][0], kb[0][1], kb[1][0], kb[1][1],
-                  sk + ((lane & 7) + ((lane >> 4) << 3)) * ROW + ks * 16 + ((lane >> 3) & 1) * 8);
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        // Q fragments: lane supplies row (lane & 15) of the tile, k half (lane >> 4)
-        uint32_t a0, a1, a2, a3;
-        ldmatrix_x4(a0, a1, a2, a3, sQ + (mt * 16 + (lane & 15)) * ROW + ks * 16 + (lane >> 4) * 8);
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) mma_bf16_16816(s[mt][nt], a0, a1, a2, a3, kb[nt][0], kb[nt][1]);
-      }
-    }
-
-    // online softmax (base 2); masked keys get -inf.  Row groups of 8 with no
-    // query (past n_tok: zero Q rows, never stored) are skipped.
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-#pragma unroll
-      for (int hr = 0; hr < 2; ++hr) {   // hr 0: row g, hr 1: row g + 8
-        if (mt * 16 + hr * 8 >= a.n_tok) continue;
-        float x[4];
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int key = chunk * 16 + nt * 8 + tig * 2 + j;
-            x[nt * 2 + j] = (key < n_keys && ((keep >> (nt * 2 + j)) & 1u)) ? s[mt][nt][hr * 2 + j] * a.scale_log2
-                                                                             : -INFINITY;
-          }
-        float cm = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-        cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 1));
-        cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 2));
-        const float m_old = mrow[mt][hr];
-        const float m_new = fmaxf(m_old, cm);
-        const float alpha = (m_new == -INFINITY) ? 1.0f : ex2_approx(m_old - m_new);
-        float psum = 0.0f;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float p = (m_new == -INFINITY) ? 0.0f : ex2_approx(x[j] - m_new);
-          x[j] = p;
-          psum += p;
-        }
-        mrow[mt][hr] = m_new;
-        lrow[mt][hr] = lrow[mt][hr] * alpha + psum;
-#pragma unroll
-        for (int nd = 0; nd < DH / 8; ++nd) {
-          o[mt][nd][hr * 2 + 0] *= alpha;
-          o[mt][nd][hr * 2 + 1] *= alpha;
-        }
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          s[mt][nt][hr * 2 + 0] = x[nt * 2 + 0];
-          s[mt][nt][hr * 2 + 1] = x[nt * 2 + 1];
-        }
-      }
-    }
-
-    // O += P V : P (16 x 16 keys) from the score accumulators, V via ldmatrix.trans
-#pragma unroll
-    for (int nd2 = 0; nd2 < DH / 16; ++nd2) {   // pairs of 8-wide dim tiles
-      uint32_t vb0, vb1, vb2, vb3;
-      const int r = lane & 7;
-      const int mtx = lane >> 3;          // matrix 0..3: (keys 0-7 | 8-15) x (dims nd | nd+1)
-      const __nv_bfloat16* vp = sv + ((mtx & 1) * 8 + r) * ROW + (nd2 * 2 + (mtx >> 1)) * 8;
-      ldmatrix_x4_trans(vb0, vb1, vb2, vb3, vp);
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        const uint32_t a0 = pack_bf16x2(s[mt][0][0], s[mt][0][1]);
-        const uint32_t a1 = pack_bf16x2(s[mt][0][2], s[mt][0][3]);
-        const uint32_t a2 = pack_bf16x2(s[mt][1][0], s[mt][1][1]);
-        const uint32_t a3 = pack_bf16x2(s[mt][1][2], s[mt][1][3]);
-        mma_bf16_16816(o[mt][nd2 * 2 + 0], a0, a1, a2, a3, vb0, vb1);
-        mma_bf16_16816(o[mt][nd2 * 2 + 1], a0, a1, a2, a3, vb2, vb3);
-      }
-    }
+    // padded rows of ROW elements: 16-byte column chunk cc of key row r
+    attn_fold_chunk<MT, DH>(
+        a, chunk * 16, k_begin, n_keys, sQ,
+        [&](int r, int cc) { return sk + r * ROW + cc * 8; },
+        [&](int r, int cc) { return sv + r * ROW + cc * 8; }, o, mrow, lrow);
     __syncwarp();   // the slot is refilled by a later issue
   }
   cp_async_wait<0>();

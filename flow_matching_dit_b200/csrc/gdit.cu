@@ -123,6 +123,25 @@ CUtensorMap make_tmap(const void* ptr, long long rows, long long cols, long long
   return m;
 }
 
+// The K/V cache as a 2-D tensor of head_dim-wide bf16 rows, for TMA boxes of
+// box_rows rows with the shared-memory swizzle of one row (128 bytes for
+// head_dim 64, 64 bytes for 32).
+CUtensorMap make_kv_tmap(const void* ptr, long long rows, int head_dim, int box_rows) {
+  REQUIRE(((uintptr_t)ptr & 15u) == 0, "TMA base pointer not 16-byte aligned");
+  REQUIRE(head_dim == 32 || head_dim == 64, "head_dim %d", head_dim);
+  CUtensorMap m;
+  cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
+  cuuint32_t box[2] = {(cuuint32_t)head_dim, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = encode_fn()(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           head_dim == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) throw GditError(GDIT_ECUDA, fmt("cuTensorMapEncodeTiled (K/V cache) failed (%d)", (int)r));
+  return m;
+}
+
 // Output map for the TMA-store epilogue: [rows, cols] with row pitch `pitch`
 // elements, 32-row boxes of 128 bytes (bf16: 64 columns, f32: 32), 128-byte swizzle.
 CUtensorMap make_out_tmap(const void* ptr, bool f32, long long rows, long long cols, long long pitch) {
@@ -169,6 +188,7 @@ struct GemmOp {
   GemmArgs args;
   int bn = 64;
   int grid = 1;
+  bool pair = false;   // CTA-pair kernel (256-row tiles, cta_group::2)
   // algorithmic accounting: rows actually multiplied are known after routing
   int rows_kind = 0;   // 0 fixed M, 1 = total valid tokens, 2 = all rows (grouped)
   long long weight_bytes = 0;
@@ -189,12 +209,66 @@ void enable_tma_out(GemmOp& op) {
   a.tma_out = 1;
 }
 
+// Move a dense TMA-store GEMM to the CTA-pair kernel when its 256-row tiles
+// still occupy about as many SMs as the 128-row tiles would: the pair tile
+// reads a third less operand data from L2 per unit of tensor work.
+void enable_pair(GemmOp& op, const void* A, const void* W, int num_sms) {
+  GemmArgs& a = op.args;
+  if (!a.tma_out || (op.bn != 256 && op.bn != 128) || a.m_dev != nullptr) return;
+  const long long nt = (a.N + op.bn - 1) / op.bn;
+  const long long pair_tiles = ((a.M + kPairBM - 1) / kPairBM) * nt;
+  const long long one_tiles = ((a.M + kBM - 1) / kBM) * nt;
+  const long long pair_sms = std::min<long long>(2 * pair_tiles, num_sms - num_sms % 2);
+  const long long one_sms = std::min<long long>(one_tiles, num_sms);
+  if (10 * pair_sms < 9 * one_sms) return;
+  op.pair = true;
+  op.ta = make_tmap(A, a.M, a.K, a.K, 128);
+  op.tb = make_tmap(W, a.N, a.K, a.K, op.bn / 2);
+  op.grid = (int)(2 * std::min<long long>(pair_tiles, num_sms / 2));
+}
+
 template <int BN>
 void set_gemm_attr() {
   CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmCfg<BN>::SMEM));
 }
 
+template <int BN>
+void set_gemm_pair_attr() {
+  CUDA_TRY(cudaFuncSetAttribute(gemm_tc_pair_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                GemmPairCfg<BN>::SMEM));
+}
+
+// CTA-pair GEMM: clusters of two CTAs (grid even), optionally after the
+// previous kernel by programmatic dependent launch.
+template <int BN>
+void launch_gemm_pair(const GemmOp& op, const GemmArgs& a, cudaStream_t s, bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(op.grid);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = GemmPairCfg<BN>::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
+  CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_tc_pair_kernel<BN>, op.ta, op.tb, op.to, a));
+}
+
 void launch_gemm(const GemmOp& op, const GemmArgs& a, cudaStream_t s, bool pdl) {
+  if (op.pair) {
+    if (op.bn == 256)
+      launch_gemm_pair<256>(op, a, s, pdl);
+    else if (op.bn == 128)
+      launch_gemm_pair<128>(op, a, s, pdl);
+    else
+      throw GditError(GDIT_EINVAL, fmt("bad CTA-pair tile width %d", op.bn));
+    return;
+  }
   switch (op.bn) {
     case 32:
       launch_k(s, pdl, gemm_tc_kernel<32>, dim3(op.grid), dim3(kGemmThreads), GemmCfg<32>::SMEM, op.ta, op.tb, op.to, a);
@@ -357,18 +431,65 @@ struct gdit_handle {
   Recorder* rec = nullptr;   // non-null during gdit_profile_get_action
   int last_B = 0;
 
+  // Host-side fault injection, read from GDIT_FAULT at create
+  // ("alloc:N,graph:N,upload:N"): the N-th device allocation, CUDA-graph
+  // instantiation or weight upload of this handle (counted from 1) fails the
+  // way the real call would.  Nothing on the device is made to fail.
+  struct Faults {
+    long long alloc = 0, graph = 0, upload = 0;      // 0: never
+    long long n_alloc = 0, n_graph = 0, n_upload = 0;
+  } fault;
+
   template <typename T>
   T* dalloc(size_t count) {
+    if (++fault.n_alloc == fault.alloc)
+      throw GditError(GDIT_ENOMEM, fmt("injected fault: device allocation %lld failed", fault.n_alloc));
     void* p = nullptr;
     CUDA_TRY(cudaMalloc(&p, std::max<size_t>(count * sizeof(T), 256)));
     allocs.push_back(p);
     return static_cast<T*>(p);
+  }
+
+  // host -> device copy of weight data (synchronous)
+  void upload(void* dst, const void* src, size_t bytes) {
+    if (++fault.n_upload == fault.upload)
+      throw GditError(GDIT_ECUDA, fmt("injected fault: weight upload %lld failed", fault.n_upload));
+    CUDA_TRY(cudaMemcpy(dst, src, bytes, cudaMemcpyHostToDevice));
   }
 };
 
 namespace {
 
 // ------------------------------------------------------------------ validation
+
+// GDIT_FAULT = comma-separated "kind:N" with kind alloc, graph or upload and
+// N >= 1 (see gdit_handle::Faults).
+void parse_faults(const char* spec, gdit_handle::Faults& f) {
+  if (spec == nullptr || spec[0] == '\0') return;
+  std::string s(spec);
+  size_t pos = 0;
+  while (pos <= s.size()) {
+    size_t end = s.find(',', pos);
+    if (end == std::string::npos) end = s.size();
+    const std::string item = s.substr(pos, end - pos);
+    const size_t colon = item.find(':');
+    REQUIRE(colon != std::string::npos, "GDIT_FAULT item '%s' is not kind:N", item.c_str());
+    const std::string kind = item.substr(0, colon);
+    char* stop = nullptr;
+    const long long n = std::strtoll(item.c_str() + colon + 1, &stop, 10);
+    REQUIRE(stop != nullptr && *stop == '\0' && n >= 1, "GDIT_FAULT item '%s': N must be an integer >= 1",
+            item.c_str());
+    if (kind == "alloc")
+      f.alloc = n;
+    else if (kind == "graph")
+      f.graph = n;
+    else if (kind == "upload")
+      f.upload = n;
+    else
+      throw GditError(GDIT_EINVAL, fmt("GDIT_FAULT kind '%s' is not alloc, graph or upload", kind.c_str()));
+    pos = end + 1;
+  }
+}
 
 void validate_config(const gdit_config& c) {
   REQUIRE(c.num_layers >= 2 && c.num_layers % 2 == 0, "num_layers must be even and >= 2 (got %d)", c.num_layers);
@@ -522,7 +643,7 @@ struct Uploader {
   void put_rows(__nv_bfloat16* dst, const HostW& w, size_t count) {
     hb.resize(count);
     for (size_t i = 0; i < count; ++i) hb[i] = f32_to_bf16_rne(w.at((int64_t)i));
-    CUDA_TRY(cudaMemcpy(dst, hb.data(), count * 2, cudaMemcpyHostToDevice));
+    h->upload(dst, hb.data(), count * 2);
   }
   __nv_bfloat16* matrix(const HostW& w) {
     __nv_bfloat16* d = mat((size_t)w.numel);
@@ -537,20 +658,20 @@ struct Uploader {
       for (int o = 0; o < out; ++o)
         for (int i = 0; i < nin; ++i)
           hb[((size_t)c * out + o) * nin + i] = f32_to_bf16_rne(w.at(((int64_t)c * in + in0 + i) * out + o));
-    CUDA_TRY(cudaMemcpy(d, hb.data(), hb.size() * 2, cudaMemcpyHostToDevice));
+    h->upload(d, hb.data(), hb.size() * 2);
     return d;
   }
   float* vec(const HostW& w) {
     float* d = h->dalloc<float>((size_t)w.numel);
     hf.resize((size_t)w.numel);
     for (int64_t i = 0; i < w.numel; ++i) hf[i] = w.at(i);
-    CUDA_TRY(cudaMemcpy(d, hf.data(), hf.size() * 4, cudaMemcpyHostToDevice));
+    h->upload(d, hf.data(), hf.size() * 4);
     return d;
   }
   void vec_into(float* d, const HostW& w) {
     hf.resize((size_t)w.numel);
     for (int64_t i = 0; i < w.numel; ++i) hf[i] = w.at(i);
-    CUDA_TRY(cudaMemcpy(d, hf.data(), hf.size() * 4, cudaMemcpyHostToDevice));
+    h->upload(d, hf.data(), hf.size() * 4);
   }
 };
 
@@ -719,6 +840,10 @@ void set_kernel_attrs() {
   set_gemm_attr<64>();
   set_gemm_attr<128>();
   set_gemm_attr<256>();
+  set_gemm_pair_attr<128>();
+  set_gemm_pair_attr<256>();
+  max_shared_carveout(gemm_tc_pair_kernel<128>);
+  max_shared_carveout(gemm_tc_pair_kernel<256>);
   CUDA_TRY(cudaFuncSetAttribute(small_loop_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 SmallSmem<64>::TOTAL));
   CUDA_TRY(cudaFuncSetAttribute(small_loop_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -810,7 +935,13 @@ GemmOp plan_gemm(gdit_handle* h, const void* A, long long a_rows, int K, const v
 bool small_loop_fits(const gdit_config& c, int N, int num_sms) {
   const long long D = c.hidden, F = c.mlp_hidden, A = c.action_dim;
   if (N > kSmallMaxTok || D > kSmallMaxD || c.num_layers > kSmallMaxLayers || c.num_heads > num_sms) return false;
+  // the K/V cache rows (with one box of slack) are addressed by 32-bit TMA coordinates
+  if ((long long)(c.num_layers / 2) * 2 * c.num_heads * ((long long)c.max_batch * c.max_backbone_seq + kSmallAttnKB) >=
+      (1LL << 31))
+    return false;
   if ((long long)N * (D + 8) * 2 > kSmLnScratch) return false;   // LN output rows below the LN scratch
+  // LN: the staged f32 rows and the two modulation vectors, after the output rows
+  if ((long long)small_ln_stage_offset(N, (int)D) + (long long)(N + 2) * D * 4 > kSmLnScratch) return false;
   for (long long K : {A, D, F}) {
     if (K % 16 != 0 || (K > kSmallKC && K % kSmallKC != 0)) return false;
     if ((long long)N * (K + 8) * 2 > kSmXBytes) return false;
@@ -918,6 +1049,12 @@ std::unique_ptr<Profile> build_profile(gdit_handle* h, int B, int S, int K, int 
     p->ff2[l].weight_bytes = (long long)D * F * 2;
     if ((h->cfg.flags & GDIT_FLAG_NO_TMA_STORE) == 0)
       for (GemmOp* g : {&p->q[l], &p->o[l], &p->ff1[l], &p->ff2[l]}) enable_tma_out(*g);
+    if ((h->cfg.flags & GDIT_FLAG_NO_PAIR) == 0) {
+      enable_pair(p->q[l], h->u, m.wq[l], h->num_sms);
+      enable_pair(p->o[l], h->o, m.wo[l], h->num_sms);
+      enable_pair(p->ff1[l], h->u, m.wff1[l], h->num_sms);
+      enable_pair(p->ff2[l], h->f, m.wff2[l], h->num_sms);
+    }
   }
   // norm_out + proj_out on every token; only the H action rows are kept (compact)
   p->proj = plan_gemm(h, h->u, rows, D, m.proj_w, D, D, EPI_BF16, rows, 0, 0, 1);
@@ -971,6 +1108,8 @@ std::unique_ptr<Profile> build_profile(gdit_handle* h, int B, int S, int K, int 
       y.wff1 = m.wff1[l]; y.bff1 = m.bff1[l]; y.wff2 = m.wff2[l]; y.bff2 = m.bff2[l];
       y.kv = (l % 2 == 0) ? h->kv + (size_t)(l / 2) * h->max_tok * 2 * D : nullptr;
     }
+    sp.kv_map = make_kv_tmap(h->kv, (long long)h->Lc * 2 * h->cfg.num_heads * h->max_tok, h->cfg.head_dim,
+                             kSmallAttnKB);
     sp.counters = h->phase_counters;
     sp.phases = h->phase_table;
     sp.err = h->status;
@@ -1202,6 +1341,10 @@ Profile& get_profile(gdit_handle* h, int B, int S, int K, int bf16, bool allow_b
       throw;
     }
     CUDA_TRY(cudaStreamEndCapture(h->cap_stream, &graph));
+    if (++h->fault.n_graph == h->fault.graph) {
+      cudaGraphDestroy(graph);
+      throw GditError(GDIT_ECUDA, fmt("injected fault: graph instantiation %lld failed", h->fault.n_graph));
+    }
     cudaError_t e = cudaGraphInstantiate(&p->exec, graph, 0);
     cudaGraphDestroy(graph);
     CUDA_TRY(e);
@@ -1303,6 +1446,8 @@ int gdit_create(const gdit_config* cfg, const gdit_tensor* weights, int n_weight
     REQUIRE(cfg != nullptr && out != nullptr, "cfg and out must not be NULL");
     validate_config(*cfg);
     auto W = check_weights(*cfg, weights, n_weights);   // host-only checks first
+    gdit_handle::Faults faults;
+    parse_faults(getenv("GDIT_FAULT"), faults);
     int ndev = 0;
     if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) throw GditError(GDIT_ENODEV, "no CUDA device");
     REQUIRE(cfg->device >= 0 && cfg->device < ndev, "device %d out of range", cfg->device);
@@ -1328,6 +1473,7 @@ int gdit_create(const gdit_config* cfg, const gdit_tensor* weights, int n_weight
     h->strict = (cfg->flags & GDIT_FLAG_STRICT_PROFILES) != 0;
     const char* pdl_env = getenv("GDIT_PDL");
     h->pdl = !(pdl_env && pdl_env[0] == '0');
+    h->fault = faults;
     set_kernel_attrs();
     upload_model(h, W);
     alloc_workspace(h);
@@ -1600,6 +1746,7 @@ int gdit_profile_get_action(gdit_handle* h, const void* backbone_features, int b
 int gdit_test_gemm(const void* A, const void* B, const float* bias, float* C, int M, int N, int K, int bn, int splits,
                    void* cuda_stream) {
   const bool tma_out = getenv("GDIT_TEST_TMA_OUT") != nullptr;   // unit-test knob: exercise the TMA-store epilogue
+  const bool pair = getenv("GDIT_TEST_PAIR") != nullptr;         // unit-test knob: the CTA-pair kernel (with TMA store)
   g_create_error.clear();
   return guarded(nullptr, [&] {
     REQUIRE(A && B && C, "NULL matrix");
@@ -1641,11 +1788,18 @@ int gdit_test_gemm(const void* A, const void* B, const float* bias, float* C, in
     op.ta = make_tmap(A, M, K, K, kBM);
     op.tb = make_tmap(B, N, K, K, bn);
     op.to = op.ta;
+    op.grid = (int)std::min<long long>(mt * nt * splits, sms);
     if (tma_out && splits == 1) {
       op.to = make_out_tmap(C, true, M, N, N);
       op.args.tma_out = 1;
+      if (pair && (bn == 128 || bn == 256)) {
+        op.pair = true;
+        op.ta = make_tmap(A, M, K, K, 128);
+        op.tb = make_tmap(B, N, K, K, bn / 2);
+        const long long pt = ((M + kPairBM - 1) / kPairBM) * nt;
+        op.grid = (int)(2 * std::min<long long>(pt, sms / 2));
+      }
     }
-    op.grid = (int)std::min<long long>(mt * nt * splits, sms);
     launch_gemm(op, op.args, s, false);
     CUDA_TRY(cudaStreamSynchronize(s));
     unsigned e = 0;

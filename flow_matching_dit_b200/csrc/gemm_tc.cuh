@@ -77,6 +77,7 @@ struct GemmArgs {
 
   int tma_out;              // 1: output through the TMA map (dense, one split, plain [M, N] layout)
   unsigned* err;
+
 };
 
 template <int BN>
@@ -293,6 +294,86 @@ __device__ __forceinline__ void gemm_epilogue32(const GemmArgs& a, int g, int m,
   }
 }
 
+// TMA-store epilogue of one accumulator tile on one epilogue warp: TMEM lanes
+// of this warp's quarter (taddr), i.e. output rows [ym, ym + 32), column
+// chunks half, half + 2, ... of [n0, n0 + BN); f32 boxes hold 32 columns,
+// bf16 boxes 64.  Each chunk is staged in one of this warp's NBOX 4 KB boxes
+// (128-byte swizzle, conflict-free 16-byte stores; `seq` counts the warp's
+// chunks, so consecutive chunks alternate boxes) and one lane issues a bulk
+// tensor store, or a bulk reduce-add for the residual adds.  Both TMEM loads
+// of a 64-column chunk are issued before one wait.
+template <int BN, int NBOX>
+__device__ __forceinline__ void gemm_epilogue_tma(const GemmArgs& a, const CUtensorMap* tmO, uint8_t* boxes,
+                                                  uint32_t taddr, int n0, int ym, int half, int lane, int& seq) {
+  const bool f32out = a.epi == EPI_RESID_F32 || a.epi == EPI_F32;
+  const int ccols = f32out ? 32 : 64;
+  const int rs = lane & 7;   // swizzle phase of this thread's row
+#pragma unroll 1
+  for (int cs = half; cs < BN / ccols; cs += 2, ++seq) {
+    const int n = n0 + cs * ccols;
+    uint8_t* box = boxes + (seq % NBOX) * 4096;
+    float v[64];
+    {
+      uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[0]);
+      uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[32]);
+      tmem_ld32(taddr + cs * ccols, lo);
+      if (!f32out) tmem_ld32(taddr + cs * ccols + 32, hi);
+      tmem_ld_wait();
+    }
+    // the store NBOX chunks ago has finished reading this box
+    if (lane == 0) bulk_wait_read<NBOX - 1>();
+    __syncwarp();
+    if (f32out) {
+      if (a.bias != nullptr) {
+        const float4* bp = reinterpret_cast<const float4*>(a.bias + n);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float4 b = __ldg(bp + j);
+          v[4 * j] += b.x; v[4 * j + 1] += b.y; v[4 * j + 2] += b.z; v[4 * j + 3] += b.w;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<float4*>(box + lane * 128 + ((j ^ rs) << 4)) =
+            make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    } else {
+      if (a.bias != nullptr) {
+        const float4* bp = reinterpret_cast<const float4*>(a.bias + n);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float4 b = __ldg(bp + j);
+          v[4 * j] += b.x; v[4 * j + 1] += b.y; v[4 * j + 2] += b.z; v[4 * j + 3] += b.w;
+        }
+      }
+      if (a.epi == EPI_GELU_BF16) {
+#pragma unroll
+        for (int j = 0; j < 64; ++j) v[j] = gelu_erf(v[j]);
+      } else if (a.epi == EPI_RELU_BF16) {
+#pragma unroll
+        for (int j = 0; j < 64; ++j) v[j] = fmaxf(v[j], 0.0f);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        uint4 w;
+        w.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
+        w.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+        w.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+        w.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+        *reinterpret_cast<uint4*>(box + lane * 128 + ((j ^ rs) << 4)) = w;
+      }
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      if (a.epi == EPI_RESID_F32)
+        tma_reduce_add_2d(tmO, box, n, ym);
+      else
+        tma_store_2d(tmO, box, n, ym);
+      bulk_commit();
+    }
+  }
+}
+
 template <int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -448,6 +529,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int half = (warp - 2) >> 2;   // column chunks half, half + 2, ... of the tile
     const int row = q * 32 + lane;
     int it = 0;
+    int eseq = 0;   // TMA-store chunks of this warp
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
       TileInfo ti;
       gemm_decode(a, sched, t, ti);
@@ -463,80 +545,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int n0 = ti.n_idx * BN;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
       if (a.tma_out) {
-        // rows [m0 + 32q, +32) of the tile; f32 boxes hold 32 columns, bf16 boxes 64
-        const bool f32out = a.epi == EPI_RESID_F32 || a.epi == EPI_F32;
-        const int ccols = f32out ? 32 : 64;
-        const int ym = ti.m0 + q * 32;
-        const int rs = lane & 7;   // swizzle phase of this thread's row
-#pragma unroll 1
-        for (int cs = half; cs < BN / ccols; cs += 2) {
-          const int n = n0 + cs * ccols;
-          float v[64];
-          {
-            uint32_t r[32];
-            tmem_ld32(taddr + cs * ccols, r);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-            if (!f32out) {
-              tmem_ld32(taddr + cs * ccols + 32, r);
-              tmem_ld_wait();
-#pragma unroll
-              for (int j = 0; j < 32; ++j) v[32 + j] = __uint_as_float(r[j]);
-            }
-          }
-          uint8_t* box = stg + (warp - 2) * 4096;
-          if (lane == 0) bulk_wait_read<0>();   // this warp's previous store has read its box
-          __syncwarp();
-          if (f32out) {
-            if (a.bias != nullptr) {
-              const float4* bp = reinterpret_cast<const float4*>(a.bias + n);
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                const float4 b = bp[j];
-                v[4 * j] += b.x; v[4 * j + 1] += b.y; v[4 * j + 2] += b.z; v[4 * j + 3] += b.w;
-              }
-            }
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              *reinterpret_cast<float4*>(box + lane * 128 + ((j ^ rs) << 4)) =
-                  make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-          } else {
-            if (a.bias != nullptr) {
-              const float4* bp = reinterpret_cast<const float4*>(a.bias + n);
-#pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                const float4 b = bp[j];
-                v[4 * j] += b.x; v[4 * j + 1] += b.y; v[4 * j + 2] += b.z; v[4 * j + 3] += b.w;
-              }
-            }
-            if (a.epi == EPI_GELU_BF16) {
-#pragma unroll
-              for (int j = 0; j < 64; ++j) v[j] = gelu_erf(v[j]);
-            } else if (a.epi == EPI_RELU_BF16) {
-#pragma unroll
-              for (int j = 0; j < 64; ++j) v[j] = fmaxf(v[j], 0.0f);
-            }
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              uint4 w;
-              w.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
-              w.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
-              w.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
-              w.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
-              *reinterpret_cast<uint4*>(box + lane * 128 + ((j ^ rs) << 4)) = w;
-            }
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            if (a.epi == EPI_RESID_F32)
-              tma_reduce_add_2d(&tmO, box, n, ym);
-            else
-              tma_store_2d(&tmO, box, n, ym);
-            bulk_commit();
-          }
-        }
+        // rows [m0 + 32q, +32) of the tile
+        gemm_epilogue_tma<BN, 1>(a, &tmO, stg + (warp - 2) * 4096, taddr, n0, ti.m0 + q * 32, half, lane, eseq);
         tc_fence_before();
         mbar_arrive(&tempty[buf]);
       } else if (a.splits == 1) {
@@ -616,6 +626,231 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+// ====================================================================== CTA-pair GEMM
+//
+// Dense GEMMs with a plain TMA-store output (the DiT linears at large batch)
+// run on CTA pairs: a cluster of two CTAs on two SMs owns a 256 x BN output
+// tile.  Each CTA loads its 128 rows of A and its BN/2 rows of B (weights)
+// into its own shared memory; one thread of the even CTA issues
+// tcgen05.mma.cta_group::2 (256 x BN x 16), which reads both CTAs' operands
+// and leaves each CTA's 128 accumulator rows in that CTA's TMEM.  Per SM and
+// k-block that is 16 KB of A and BN/2 x 128 bytes of B from L2, a third less
+// than the 128 x BN tile of one CTA for the same tensor work; the 1-CTA tile
+// is bound by that L2-to-shared-memory traffic.
+//
+// Protocol: the stage barriers `full` live in the even CTA (both CTAs' TMA
+// loads count their bytes there); `empty` and `tfull` live in both CTAs and
+// the MMA thread's commits arrive on both; `tempty` lives in the even CTA and
+// counts one arrival per epilogue warp of both CTAs.  Both CTAs walk the same
+// tile sequence.  Every wait is bounded; both CTAs always reach the final
+// cluster barrier, after which TMEM is released.
+
+constexpr int kPairBM = 256;
+
+template <int BN>
+struct GemmPairCfg {
+  static constexpr int A_BYTES = 128 * kBK * 2;
+  static constexpr int B_BYTES = (BN / 2) * kBK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;              // per CTA
+  static constexpr int NBOX = 2;                                     // staging boxes per epilogue warp
+  static constexpr int STG_BYTES = kEpiWarps * NBOX * 4096;
+  static constexpr int STAGES = (227 * 1024 - 1024 - STG_BYTES - 256) / STAGE_BYTES;
+  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + STG_BYTES + 256;
+  static constexpr uint32_t IDESC = idesc_bf16_f32(kPairBM, BN);
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+};
+
+// Tile t of a pair GEMM: 256-row block m_idx, column tile n_idx (row blocks
+// grouped by 8 so that consecutive tiles reuse the same weight columns in L2).
+__device__ __forceinline__ void gemm_pair_decode(int t, int mt, int nt, int& m0, int& n_idx) {
+  constexpr int GM = 8;
+  const int group_size = GM * nt;
+  const int gid = t / group_size;
+  const int first_m = gid * GM;
+  const int gm = min(mt - first_m, GM);
+  const int r = t - gid * group_size;
+  m0 = (first_m + r % gm) * kPairBM;
+  n_idx = r / gm;
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmO, const GemmArgs a) {
+  using Cfg = GemmPairCfg<BN>;
+  constexpr int STAGES = Cfg::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint32_t tmem_holder;
+  __shared__ volatile int s_abort;
+
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * Cfg::A_BYTES;
+  uint8_t* stg = smem + STAGES * Cfg::STAGE_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(stg + Cfg::STG_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 2 * kEpiWarps);
+    }
+    fence_mbar_init();
+    s_abort = 0;
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmO);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&tmem_holder, Cfg::TMEM_COLS);
+    tmem_relinquish_pair();
+    tc_fence_before();
+  }
+  // both CTAs' barriers exist before either CTA signals the other's
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_holder;
+  const uint32_t full_l = mapa_shared(&full[0], 0);       // the even CTA's stage barriers
+  const uint32_t tempty_l = mapa_shared(&tempty[0], 0);   // the even CTA's accumulator-free barriers
+
+  const int mt = (a.M + kPairBM - 1) / kPairBM;
+  const int nt = (a.N + BN - 1) / BN;
+  const int total = mt * nt;
+  const int cid = blockIdx.x >> 1;
+  const int ncl = gridDim.x >> 1;
+  const int nkb = (a.K + kBK - 1) / kBK;
+
+  // The weights depend on no earlier kernel: the first tile's B stages are
+  // requested before the dependency wait.
+  int pre = 0;
+  if (warp == 0 && lane == 0 && cid < total) {
+    int m0, n_idx;
+    gemm_pair_decode(cid, mt, nt, m0, n_idx);
+    pre = min(nkb, STAGES);
+    const int brow = n_idx * BN + (int)rank * (BN / 2);
+    for (int i = 0; i < pre; ++i) {
+      if (leader) mbar_arrive_expect_tx(&full[i], 2 * Cfg::STAGE_BYTES);
+      tma_load_2d_pair(sB + i * Cfg::B_BYTES, &tmB, full_l + 8u * i, i * kBK, brow);
+    }
+  }
+  pdl_wait();
+  pdl_launch_dependents();
+  __syncthreads();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int t = cid; t < total && ok; t += ncl) {
+        int m0, n_idx;
+        gemm_pair_decode(t, mt, nt, m0, n_idx);
+        const int arow = m0 + (int)rank * 128;
+        const int brow = n_idx * BN + (int)rank * (BN / 2);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (pre > 0) {
+            tma_load_2d_pair(sA + stage * Cfg::A_BYTES, &tmA, full_l + 8u * stage, kb * kBK, arow);
+            --pre;
+          } else {
+            if (!mbar_wait(&empty[stage], phase ^ 1u, a.err)) { ok = false; s_abort = 1; break; }
+            if (s_abort) { ok = false; break; }
+            if (leader) mbar_arrive_expect_tx(&full[stage], 2 * Cfg::STAGE_BYTES);
+            tma_load_2d_pair(sA + stage * Cfg::A_BYTES, &tmA, full_l + 8u * stage, kb * kBK, arow);
+            tma_load_2d_pair(sB + stage * Cfg::B_BYTES, &tmB, full_l + 8u * stage, kb * kBK, brow);
+          }
+          ++issued;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // Tail: every stage released by the MMA commits (which arrive on this
+      // CTA's empty barriers), so none is pending when the CTA exits.
+      const unsigned long long t0 = globaltimer_ns();
+      for (int i = 0; i < min(issued, STAGES); ++i) {
+        while (!mbar_try_wait(&empty[stage], phase ^ 1u) && globaltimer_ns() - t0 < 10000000ull) {
+        }
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (leader && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int t = cid; t < total && ok; t += ncl, ++it) {
+        const int buf = it & 1;
+        const uint32_t aphase = (it >> 1) & 1;
+        if (!mbar_wait(&tempty[buf], aphase ^ 1u, a.err)) { s_abort = 1; break; }
+        tc_fence_after();
+        const uint32_t d = tmem_base + buf * BN;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, a.err) || s_abort) { ok = false; s_abort = 1; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * Cfg::A_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * Cfg::B_BYTES);
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k)
+            umma_bf16_pair(d, smem_desc_sw128(a_addr + k * 32), smem_desc_sw128(b_addr + k * 32), Cfg::IDESC,
+                           (kb > 0 || k > 0) ? 1u : 0u);
+          umma_commit_pair(&empty[stage], 0x3);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        umma_commit_pair(&tfull[buf], 0x3);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..9, both CTAs)
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
+    int it = 0;
+    int eseq = 0;   // TMA-store chunks of this warp
+    for (int t = cid; t < total; t += ncl, ++it) {
+      int m0, n_idx;
+      gemm_pair_decode(t, mt, nt, m0, n_idx);
+      const int buf = it & 1;
+      const uint32_t aphase = (it >> 1) & 1;
+      int ready = 0;
+      if (lane == 0) ready = mbar_wait(&tfull[buf], aphase, a.err) && !s_abort;
+      ready = __shfl_sync(0xffffffffu, ready, 0);
+      if (!ready) { s_abort = 1; break; }
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
+      gemm_epilogue_tma<BN, Cfg::NBOX>(a, &tmO, stg + (warp - 2) * Cfg::NBOX * 4096, taddr, n_idx * BN,
+                                       m0 + (int)rank * 128 + q * 32, half, lane, eseq);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_l + 8u * buf);
+    }
+    if (lane == 0) bulk_wait<0>();   // stores complete before the CTA exits
+  }
+  __syncthreads();
+  // neither CTA leaves while the other may still read its shared memory or
+  // signal its barriers
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
   }
 }
 

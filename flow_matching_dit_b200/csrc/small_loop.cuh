@@ -64,6 +64,17 @@ constexpr int kSmBias = kSmHold + kSmallMaxUnits * kSmallMaxTok * kSmallUF * 4; 
 constexpr int kSmallSmem = kSmBias + kSmallMaxUnits * kSmallUF * 4;
 constexpr int kSmRedBytes = kSmallWarps * kSmallMaxUnits * kSmallMaxTok * kSmallUF * 4;   // over X
 static_assert(kSmRedBytes <= kSmXBytes, "reduction buffer fits the X area");
+
+// Cross attention at B = 1 (one head per CTA): the Q tile at the start of the
+// X area, the 8 warps' (max, sum) after it, then up to kSmallAttnBlocks TMA
+// boxes of kSmallAttnKB keys of K, followed by as many of V (1024-aligned for
+// the 128-byte swizzle).
+constexpr int kSmallAttnKB = 128;
+constexpr int kSmallAttnBlocks = 4;
+constexpr int kSmAttnML = 4864;
+constexpr int kSmAttnKV = 8192;
+static_assert(kSmAttnKV + 1024 + 2 * kSmallAttnBlocks * kSmallAttnKB * 128 <= kSmXBytes,
+              "K/V boxes (aligned up to 1024 bytes) fit the X area");
 static_assert(kSmallMaxUnits <= kSmallSlots, "one K-chunk of every unit of a phase is resident at once");
 static_assert(kSmallSmem <= 227 * 1024 - 1024, "shared memory budget");
 
@@ -86,6 +97,9 @@ struct SmallLayer {
 };
 
 struct SmallPlan {
+  // the K/V cache as a 2-D tensor [layers x {K, V} x heads x max_tok rows, head_dim]
+  // for TMA boxes of kSmallAttnKB rows (swizzled like a key row)
+  CUtensorMap kv_map;
   int D, F, A, H, N, nh, dh, L, K, C;
   float eps, scale_log2;
   long long max_tok;
@@ -143,6 +157,11 @@ __device__ __forceinline__ void l2_prefetch(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
+__device__ __forceinline__ void l2_prefetch_hint(const void* p, uint32_t bytes, uint64_t policy) {
+  asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], %1, %2;" ::"l"(p), "r"(bytes), "l"(policy)
+               : "memory");
+}
+
 // barrier of the 8 compute warps (the producer warp never joins it)
 __device__ __forceinline__ void csync() { named_bar_sync(1, kSmallCompute); }
 
@@ -158,12 +177,10 @@ __device__ __forceinline__ void red_release_add(int* p, int v) {
   asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
 
 struct alignas(16) SmallPhase {
   int kind;          // 0 GEMM, 1 attention
+  int kv_row;        // cross attention: first row of this layer's K block in kv_map
   SmallGemm g;
   AttnArgs a;
 };
@@ -225,6 +242,7 @@ __device__ __forceinline__ void small_describe(const SmallPlan& P, int c, int k,
         } else {
           a.q = P.qkv; a.q_ld = D; a.k = Ly.kv; a.v = Ly.kv + (size_t)P.nh * P.max_tok * P.dh; a.kv_ld = P.dh;
           a.kv_head_stride = P.max_tok * P.dh; a.kofs = P.vofs;
+          ph.kv_row = (int)((long long)(l / 2) * 2 * P.nh * P.max_tok);
         }
         break;
       }
@@ -274,6 +292,9 @@ struct SmallCtx {
   const SmallPhase* phases;
   const int* vofs;
   int dh;
+  int nh;
+  long long max_tok;
+  const CUtensorMap* kv_map;
 };
 
 // Thread 0 waits (acquire) until `target` CTAs have arrived on `phase`; the
@@ -341,6 +362,11 @@ __device__ __forceinline__ void small_producer(const SmallCtx& P, int total, uin
   const int lane = threadIdx.x & 31;
   uint32_t item = 0;
   bool ok = true;
+  // The weights are read once per Euler step and 0.75 GB of them pass
+  // through L2 per step: they are marked first to evict, so that the
+  // activations, the per-step tables and the K/V cache (read every step)
+  // stay in L2.
+  const uint64_t stream_policy = policy_evict_first();
   auto l2_ahead = [&](int gp) {   // the chunks of phase gp (if any) towards L2
     if (lane != 0 || gp >= total) return;
     const SmallPhase& ph = P.phases[gp];
@@ -348,7 +374,8 @@ __device__ __forceinline__ void small_producer(const SmallCtx& P, int total, uin
       const SmallGemm& g = ph.g;
       const int nu = small_my_units(g);
       for (int j = 0; j < nu; ++j)
-        l2_prefetch(g.W + (size_t)small_unit(j) * kSmallUF * g.K, (uint32_t)(kSmallUF * g.K * 2));
+        l2_prefetch_hint(g.W + (size_t)small_unit(j) * kSmallUF * g.K, (uint32_t)(kSmallUF * g.K * 2),
+                         stream_policy);
     } else if (ph.a.kofs != nullptr && (int)blockIdx.x < ph.a.num_heads) {
       // K and V of this CTA's head: contiguous rows of the head-major cache
       const uint32_t bytes = (uint32_t)P.vofs[1] * (uint32_t)P.dh * 2u;
@@ -380,7 +407,7 @@ __device__ __forceinline__ void small_producer(const SmallCtx& P, int total, uin
         if (lane < kSmallUF) {
           uint8_t* dst = smem + kSmRing + slot * kSlotBytes + lane * kSlotRow * 2;
           const __nv_bfloat16* src = g.W + ((size_t)small_unit(j) * kSmallUF + lane) * g.K + (size_t)c * kc;
-          bulk_g2s(dst, src, (uint32_t)kc * 2u, &R.full[slot]);
+          bulk_g2s_hint(dst, src, (uint32_t)kc * 2u, &R.full[slot], stream_policy);
         }
       }
     }
@@ -442,11 +469,43 @@ __device__ __forceinline__ void small_issue_side(const SmallGemm& g, int nu, uin
   cp_async_commit();
 }
 
-// LN(h rows) -> bf16 X rows.  Thread t owns columns [4t, 4t + 4) of every
-// row: it loads them from L2 into registers, the CTA reduces each row's sum
+// Shared-memory offset of the f32 rows staged for LayerNorm (after the bf16
+// output rows); the two modulation vectors follow them.
+__device__ __host__ __forceinline__ int small_ln_stage_offset(int rows, int D) {
+  return (rows * (D + 8) * 2 + 127) & ~127;
+}
+
+// Warp 0: the f32 residual rows that the phase normalises and its two
+// modulation vectors, by bulk copies into shared memory on `xbar`.  The
+// copy engine keeps the whole 70 KB in flight at once; loads through the
+// threads' registers are limited by the SM's outstanding-miss capacity and
+// took several L2 round trips.
+__device__ __forceinline__ void small_issue_ln(const SmallGemm& g, const SmallCtx& P, uint8_t* smem,
+                                               uint64_t* xbar) {
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x >= 32) return;
+  const int D = g.K;
+  const uint32_t row_bytes = (uint32_t)D * 4u;
+  if (lane == 0) {
+    fence_proxy_async_global();
+    fence_proxy_async_smem();
+    mbar_arrive_expect_tx(xbar, (uint32_t)(g.rows + 2) * row_bytes);
+  }
+  __syncwarp();
+  uint8_t* st = smem + small_ln_stage_offset(g.rows, D);
+  const float* h0 = P.h + (size_t)g.h_row_off * D;
+  for (int r = lane; r < g.rows + 2; r += 32) {
+    const float* src = r < g.rows ? h0 + (size_t)r * D : (r == g.rows ? g.p0 : g.p1);
+    bulk_g2s(st + (size_t)r * row_bytes, src, row_bytes, xbar);
+  }
+}
+
+// LN(h rows) -> bf16 X rows, from the rows staged by small_issue_ln.  Thread
+// t owns columns [4t, 4t + 4) of every row: it reads them from shared memory
+// (consecutive threads, consecutive 16 bytes), the CTA reduces each row's sum
 // and sum of squares (warp shuffles, then the 8 warps' totals through shared
 // memory), and the thread writes its columns of every normalised row with the
-// AdaLN ((1 + p0), p1) or affine (p0, p1) modulation, loaded once.
+// AdaLN ((1 + p0), p1) or affine (p0, p1) modulation.
 __device__ __forceinline__ void small_ln_rows(const SmallGemm& g, const SmallCtx& P, uint8_t* smem) {
   constexpr int G = 17;   // rows per round (N = H + 1 = 17 in one)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -456,21 +515,21 @@ __device__ __forceinline__ void small_ln_rows(const SmallGemm& g, const SmallCtx
   float* part = reinterpret_cast<float*>(smem + kSmLnScratch);   // [warp][row][2]
   float* stat = part + kSmallWarps * G * 2;                     // [row][2]
   __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(smem);
+  const float4* st = reinterpret_cast<const float4*>(smem + small_ln_stage_offset(g.rows, D)) + tid;
   const float4 zero = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
   float4 a = zero, b = zero;
   if (has) {
-    a = __ldg(reinterpret_cast<const float4*>(g.p0) + tid);
-    b = __ldg(reinterpret_cast<const float4*>(g.p1) + tid);
+    a = st[(size_t)g.rows * d4];
+    b = st[(size_t)(g.rows + 1) * d4];
   }
   if (g.ln_mode == 0) {
     a.x += 1.0f; a.y += 1.0f; a.z += 1.0f; a.w += 1.0f;
   }
-  const float4* hcol = reinterpret_cast<const float4*>(P.h + (size_t)g.h_row_off * D) + tid;
   for (int r0 = 0; r0 < g.rows; r0 += G) {
     const int nr = min(G, g.rows - r0);
     float4 v[G];
 #pragma unroll
-    for (int i = 0; i < G; ++i) v[i] = (has && i < nr) ? __ldcg(hcol + (size_t)(r0 + i) * d4) : zero;
+    for (int i = 0; i < G; ++i) v[i] = (has && i < nr) ? st[(size_t)(r0 + i) * d4] : zero;
     float sm[G], sq[G];
 #pragma unroll
     for (int i = 0; i < G; ++i) {
@@ -539,10 +598,12 @@ __device__ __forceinline__ void small_issue_qkv(const AttnArgs& a, int D, uint8_
     bulk_g2s(dst + (size_t)r * qrow * 2, a.q + (size_t)r * a.q_ld, (uint32_t)(3 * D * 2), xbar);
 }
 
-// One warp per head (heads warp, warp + 8, ...), all N <= 32 keys at once, one
-// 16-query tile after the other: S = Q K^T (four 8-key tiles), softmax over
-// the valid keys (base 2), O = P V, rows divided by their sums.  Rows and keys
-// past N read the last token (finite values) and are masked or never stored.
+// One warp per head (heads warp, warp + 8, ...), all N <= 32 keys and both
+// 16-query tiles at once: S = Q K^T (2 x 4 tiles of 16 x 8; even and odd
+// k-steps into separate accumulators, so the dependent mma.sync chains are
+// half as long), softmax over the valid keys (base 2), O = P V, rows divided
+// by their sums.  Rows and keys past N read the last token (finite values)
+// and are masked or never stored.
 template <int DH>
 __device__ __forceinline__ void small_self_attention_dh(const AttnArgs& a, int D, uint8_t* smem) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -554,30 +615,40 @@ __device__ __forceinline__ void small_self_attention_dh(const AttnArgs& a, int D
     const __nv_bfloat16* Qh = qkv + h * DH;
     const __nv_bfloat16* Kh = qkv + D + h * DH;
     const __nv_bfloat16* Vh = qkv + 2 * D + h * DH;
-#pragma unroll 1
-    for (int mt = 0; mt * 16 < N; ++mt) {
-      float s[4][4];
+    float s[2][2][4][4];   // [k-step parity][query tile][key tile of 8][fragment]
 #pragma unroll
-      for (int nt = 0; nt < 4; ++nt)
+    for (int p = 0; p < 2; ++p)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) s[nt][e] = 0.0f;
-      const int qr = min(mt * 16 + (lane & 15), N - 1);
+      for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-      for (int ks = 0; ks < DH / 16; ++ks) {
-        uint32_t a0, a1, a2, a3;
-        ldmatrix_x4(a0, a1, a2, a3, Qh + (size_t)qr * qrow + ks * 16 + (lane >> 4) * 8);
-        // K fragments: keys (lane & 7) + 8 (lane >> 4) of each 16-key pair, k half (lane >> 3) & 1
+        for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-        for (int kp = 0; kp < 2; ++kp) {
-          const int key = min(kp * 16 + (lane & 7) + ((lane >> 4) << 3), N - 1);
-          uint32_t k0, k1, k2, k3;
-          ldmatrix_x4(k0, k1, k2, k3, Kh + (size_t)key * qrow + ks * 16 + ((lane >> 3) & 1) * 8);
-          mma_bf16_16816(s[2 * kp], a0, a1, a2, a3, k0, k1);
-          mma_bf16_16816(s[2 * kp + 1], a0, a1, a2, a3, k2, k3);
+          for (int e = 0; e < 4; ++e) s[p][mt][nt][e] = 0.0f;
+#pragma unroll
+    for (int ks = 0; ks < DH / 16; ++ks) {
+      uint32_t q[2][4];
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        const int qr = min(mt * 16 + (lane & 15), N - 1);
+        ldmatrix_x4(q[mt][0], q[mt][1], q[mt][2], q[mt][3], Qh + (size_t)qr * qrow + ks * 16 + (lane >> 4) * 8);
+      }
+      // K fragments: keys (lane & 7) + 8 (lane >> 4) of each 16-key pair, k half (lane >> 3) & 1
+#pragma unroll
+      for (int kp = 0; kp < 2; ++kp) {
+        const int key = min(kp * 16 + (lane & 7) + ((lane >> 4) << 3), N - 1);
+        uint32_t k0, k1, k2, k3;
+        ldmatrix_x4(k0, k1, k2, k3, Kh + (size_t)key * qrow + ks * 16 + ((lane >> 3) & 1) * 8);
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+          mma_bf16_16816(s[ks & 1][mt][2 * kp], q[mt][0], q[mt][1], q[mt][2], q[mt][3], k0, k1);
+          mma_bf16_16816(s[ks & 1][mt][2 * kp + 1], q[mt][0], q[mt][1], q[mt][2], q[mt][3], k2, k3);
         }
       }
-      // softmax over keys 0..N-1 of each query row (a row's 32 keys: 4 tiles x 4 lanes x 2)
-      float inv[2];
+    }
+    // softmax over keys 0..N-1 of each query row (a row's 32 keys: 4 tiles x 4 lanes x 2)
+    float inv[2][2];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
       for (int hr = 0; hr < 2; ++hr) {
         float m = -INFINITY;
@@ -586,8 +657,9 @@ __device__ __forceinline__ void small_self_attention_dh(const AttnArgs& a, int D
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int key = nt * 8 + tig * 2 + e;
-            const float x = key < N ? s[nt][hr * 2 + e] * a.scale_log2 : -INFINITY;
-            s[nt][hr * 2 + e] = x;
+            const float sv = s[0][mt][nt][hr * 2 + e] + s[1][mt][nt][hr * 2 + e];
+            const float x = key < N ? sv * a.scale_log2 : -INFINITY;
+            s[0][mt][nt][hr * 2 + e] = x;
             m = fmaxf(m, x);
           }
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
@@ -597,36 +669,47 @@ __device__ __forceinline__ void small_self_attention_dh(const AttnArgs& a, int D
         for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const float p = exp2f(s[nt][hr * 2 + e] - m);
-            s[nt][hr * 2 + e] = p;
+            const float p = exp2f(s[0][mt][nt][hr * 2 + e] - m);
+            s[0][mt][nt][hr * 2 + e] = p;
             l += p;
           }
         l += __shfl_xor_sync(0xffffffffu, l, 1);
         l += __shfl_xor_sync(0xffffffffu, l, 2);
-        inv[hr] = 1.0f / l;
+        inv[mt][hr] = 1.0f / l;
       }
-      // O = P V over the two 16-key chunks; V fragments by ldmatrix.trans
-      float o[DH / 8][4];
+    // O = P V over the two 16-key chunks; V fragments by ldmatrix.trans, shared by both query tiles
+    float o[2][DH / 8][4];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
       for (int nd = 0; nd < DH / 8; ++nd)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) o[nd][e] = 0.0f;
+        for (int e = 0; e < 4; ++e) o[mt][nd][e] = 0.0f;
 #pragma unroll
-      for (int kc = 0; kc < 2; ++kc) {
-        const uint32_t p0 = pack_bf16x2(s[2 * kc][0], s[2 * kc][1]);
-        const uint32_t p1 = pack_bf16x2(s[2 * kc][2], s[2 * kc][3]);
-        const uint32_t p2 = pack_bf16x2(s[2 * kc + 1][0], s[2 * kc + 1][1]);
-        const uint32_t p3 = pack_bf16x2(s[2 * kc + 1][2], s[2 * kc + 1][3]);
-        const int r = lane & 7, mtx = lane >> 3;   // matrices: (keys 0-7 | 8-15) x (dims nd | nd + 8)
-        const int key = min(kc * 16 + (mtx & 1) * 8 + r, N - 1);
+    for (int kc = 0; kc < 2; ++kc) {
+      uint32_t pf[2][4];
 #pragma unroll
-        for (int nd2 = 0; nd2 < DH / 16; ++nd2) {
-          uint32_t vb0, vb1, vb2, vb3;
-          ldmatrix_x4_trans(vb0, vb1, vb2, vb3, Vh + (size_t)key * qrow + (nd2 * 2 + (mtx >> 1)) * 8);
-          mma_bf16_16816(o[nd2 * 2 + 0], p0, p1, p2, p3, vb0, vb1);
-          mma_bf16_16816(o[nd2 * 2 + 1], p0, p1, p2, p3, vb2, vb3);
+      for (int mt = 0; mt < 2; ++mt) {
+        pf[mt][0] = pack_bf16x2(s[0][mt][2 * kc][0], s[0][mt][2 * kc][1]);
+        pf[mt][1] = pack_bf16x2(s[0][mt][2 * kc][2], s[0][mt][2 * kc][3]);
+        pf[mt][2] = pack_bf16x2(s[0][mt][2 * kc + 1][0], s[0][mt][2 * kc + 1][1]);
+        pf[mt][3] = pack_bf16x2(s[0][mt][2 * kc + 1][2], s[0][mt][2 * kc + 1][3]);
+      }
+      const int r = lane & 7, mtx = lane >> 3;   // matrices: (keys 0-7 | 8-15) x (dims nd | nd + 8)
+      const int key = min(kc * 16 + (mtx & 1) * 8 + r, N - 1);
+#pragma unroll
+      for (int nd2 = 0; nd2 < DH / 16; ++nd2) {
+        uint32_t vb0, vb1, vb2, vb3;
+        ldmatrix_x4_trans(vb0, vb1, vb2, vb3, Vh + (size_t)key * qrow + (nd2 * 2 + (mtx >> 1)) * 8);
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+          mma_bf16_16816(o[mt][nd2 * 2 + 0], pf[mt][0], pf[mt][1], pf[mt][2], pf[mt][3], vb0, vb1);
+          mma_bf16_16816(o[mt][nd2 * 2 + 1], pf[mt][0], pf[mt][1], pf[mt][2], pf[mt][3], vb2, vb3);
         }
       }
+    }
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
       for (int hr = 0; hr < 2; ++hr) {
         const int row = mt * 16 + g + hr * 8;
@@ -634,10 +717,9 @@ __device__ __forceinline__ void small_self_attention_dh(const AttnArgs& a, int D
 #pragma unroll
           for (int nd = 0; nd < DH / 8; ++nd)
             *reinterpret_cast<uint32_t*>(xs + (size_t)row * xrow + h * DH + nd * 8 + tig * 2) =
-                pack_bf16x2(o[nd][hr * 2] * inv[hr], o[nd][hr * 2 + 1] * inv[hr]);
+                pack_bf16x2(o[mt][nd][hr * 2] * inv[mt][hr], o[mt][nd][hr * 2 + 1] * inv[mt][hr]);
         }
       }
-    }
   }
 }
 
@@ -681,6 +763,94 @@ __device__ __forceinline__ void small_epilogue(const SmallGemm& g, int n, int to
   }
 }
 
+// Operands of the MMA loop of one GEMM phase on one compute warp.
+struct SmallMmaIn {
+  const __nv_bfloat16* xa0;     // token tile 0: this lane's ldmatrix row of the X rows
+  const __nv_bfloat16* xb_lo;   // token tile 1: this lane's fragment rows 16 + gr and 24 + gr
+  const __nv_bfloat16* xb_hi;
+  bool lo1, hi1, two;           // those rows exist; the phase has a second token tile
+  int wrow;                     // this lane's ldmatrix offset in a weight slot
+  int ks0, ks1;                 // this warp's k-steps (16 wide) of every chunk
+  int kc, nch;                  // chunk width (K columns) and chunk count
+  uint32_t base;                // the CTA's weight-chunk count before the phase
+};
+
+// The MMAs of one GEMM phase on one compute warp: for chunk c of the phase,
+// wait for every unit's weight slot, then run this warp's k-steps of the
+// chunk against every unit (token fragments loaded once per k-step), then
+// release the slots.  A dependent chain of mma.sync is bound by the
+// instruction's latency, which is long next to the few MMAs a warp issues per
+// phase here: each (unit, token tile) keeps NS accumulator sets, k-step i
+// going to set i % NS, so no chain is longer than kSmallMaxKs / NS.  The sets
+// are summed into acc at the end.
+constexpr int kSmallMaxKs = kSmallKC / 16 / kSmallWarps;   // k-steps of one warp in one chunk
+template <int NU, int NS>
+__device__ __forceinline__ void small_mma_units(const SmallMmaIn& in, uint8_t* smem, SmallRing& R,
+                                                const SmallCtx& P, bool& ok, float (&acc)[kSmallMaxUnits][2][4]) {
+  const int lane = threadIdx.x & 31;
+  float a_s[NU][NS][2][4];
+#pragma unroll
+  for (int j = 0; j < NU; ++j)
+#pragma unroll
+    for (int q = 0; q < NS; ++q)
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) a_s[j][q][t][e] = 0.0f;
+  for (int c = 0; c < in.nch; ++c) {
+    const __nv_bfloat16* wsj[NU];
+#pragma unroll
+    for (int j = 0; j < NU; ++j) {
+      const uint32_t it = in.base + (uint32_t)(c * NU + j);
+      const int slot = (int)(it % kSmallSlots);
+      if (ok && !mbar_wait(&R.full[slot], (it / kSmallSlots) & 1u, P.err)) ok = false;
+      wsj[j] = reinterpret_cast<const __nv_bfloat16*>(smem + kSmRing + slot * kSlotBytes) + in.wrow;
+    }
+    if (!ok) continue;
+    const int kx = c * in.kc;
+#pragma unroll
+    for (int i = 0; i < kSmallMaxKs; ++i) {
+      const int s = in.ks0 + i;
+      if (s < in.ks1) {
+        const int k = s * 16;
+        uint32_t a[4], a1[4] = {0u, 0u, 0u, 0u};
+        ldmatrix_x4(a[0], a[1], a[2], a[3], in.xa0 + kx + k);
+        if (in.two) {
+          const int kk = kx + k;
+          a1[0] = in.lo1 ? *reinterpret_cast<const uint32_t*>(in.xb_lo + kk) : 0u;
+          a1[1] = in.hi1 ? *reinterpret_cast<const uint32_t*>(in.xb_hi + kk) : 0u;
+          a1[2] = in.lo1 ? *reinterpret_cast<const uint32_t*>(in.xb_lo + kk + 8) : 0u;
+          a1[3] = in.hi1 ? *reinterpret_cast<const uint32_t*>(in.xb_hi + kk + 8) : 0u;
+        }
+#pragma unroll
+        for (int j = 0; j < NU; ++j) {
+          uint32_t b0, b1;
+          ldmatrix_x2(b0, b1, wsj[j] + k);
+          mma_bf16_16816(a_s[j][i % NS][0], a[0], a[1], a[2], a[3], b0, b1);
+          if (in.two) mma_bf16_16816(a_s[j][i % NS][1], a1[0], a1[1], a1[2], a1[3], b0, b1);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0)
+#pragma unroll
+      for (int j = 0; j < NU; ++j) mbar_arrive(&R.empty[(in.base + (uint32_t)(c * NU + j)) % kSmallSlots]);
+  }
+#pragma unroll
+  for (int j = 0; j < kSmallMaxUnits; ++j)
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float v = 0.0f;
+        if (j < NU) {
+#pragma unroll
+          for (int q = 0; q < NS; ++q) v += a_s[j < NU ? j : 0][q][t][e];
+        }
+        acc[j][t][e] = v;
+      }
+}
+
 // One GEMM phase on the compute warps.  Chunk `item` of the CTA's running
 // count sits in slot item % kSmallSlots, filled for the (item / kSmallSlots)-th
 // time; a phase's items go chunk by chunk (every unit's K-chunk 0, then 1 ...)
@@ -699,7 +869,12 @@ __device__ __forceinline__ bool small_gemm_phase(const SmallGemm& g, const AttnA
     ok = mbar_wait(xbar, xuse & 1u, P.err);
     ++xuse;
   } else if (g.x_mode == 1) {
-    small_ln_rows(g, P, smem);
+    small_issue_ln(g, P, smem, xbar);
+    if (!mbar_wait(xbar, xuse & 1u, P.err)) *fail = 1;
+    ++xuse;
+    csync();                       // a failed wait is seen by every thread
+    ok = *fail == 0;
+    if (ok) small_ln_rows(g, P, smem);
     csync();
   } else {
     small_issue_qkv(att, g.K, smem, xbar);
@@ -722,99 +897,22 @@ __device__ __forceinline__ bool small_gemm_phase(const SmallGemm& g, const AttnA
   const bool lo1 = 16 + gr < g.rows, hi1 = 24 + gr < g.rows;
   const __nv_bfloat16* xb_lo = xs + (size_t)(lo1 ? 16 + gr : 0) * xrow + 2 * tig;
   const __nv_bfloat16* xb_hi = xs + (size_t)(hi1 ? 24 + gr : 0) * xrow + 2 * tig;
-  auto tile1 = [&](int kk, uint32_t (&f)[4]) {
-    f[0] = lo1 ? *reinterpret_cast<const uint32_t*>(xb_lo + kk) : 0u;
-    f[1] = hi1 ? *reinterpret_cast<const uint32_t*>(xb_hi + kk) : 0u;
-    f[2] = lo1 ? *reinterpret_cast<const uint32_t*>(xb_lo + kk + 8) : 0u;
-    f[3] = hi1 ? *reinterpret_cast<const uint32_t*>(xb_hi + kk + 8) : 0u;
-  };
-  // weight fragments: ldmatrix.x4 over k, k + 8, k + 16, k + 24 (two k-steps)
+  // weight fragments: ldmatrix.x2 over k, k + 8 (rows lane & 7, k half (lane >> 3) & 1)
   const int wrow = (lane & 7) * kSlotRow + (lane >> 3) * 8;
-  // accumulators per (unit, token tile); unit 0 keeps a second chain for the
-  // odd k-steps, so that single-unit phases still have independent MMAs
-  float acc[kSmallMaxUnits][2][4], acc2[2][4];
-#pragma unroll
-  for (int j = 0; j < kSmallMaxUnits; ++j)
-#pragma unroll
-    for (int t = 0; t < 2; ++t)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[j][t][e] = 0.0f;
-#pragma unroll
-  for (int t = 0; t < 2; ++t)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) acc2[t][e] = 0.0f;
-  // chunk c of every unit (items base + c * nu + j): wait for all, then each
-  // k-step loads the token fragments once and runs them against every unit
   const uint32_t base = item;
-  for (int c = 0; c < nch; ++c) {
-    const __nv_bfloat16* wsj[kSmallMaxUnits];
-#pragma unroll
-    for (int j = 0; j < kSmallMaxUnits; ++j) {
-      wsj[j] = nullptr;
-      if (j < nu) {
-        const uint32_t it = base + (uint32_t)(c * nu + j);
-        const int slot = (int)(it % kSmallSlots);
-        if (ok && !mbar_wait(&R.full[slot], (it / kSmallSlots) & 1u, P.err)) ok = false;
-        wsj[j] = reinterpret_cast<const __nv_bfloat16*>(smem + kSmRing + slot * kSlotBytes) + wrow;
-      }
-    }
-    if (ok) {
-      const int kx = c * kc;
-      int s = ks0;
-      for (; s + 1 < ks1; s += 2) {
-        const int k = s * 16;
-        uint32_t a[4], e[4], a1[4], e1[4];
-        ldmatrix_x4(a[0], a[1], a[2], a[3], xa0 + kx + k);
-        ldmatrix_x4(e[0], e[1], e[2], e[3], xa0 + kx + k + 16);
-        if (two) {
-          tile1(kx + k, a1);
-          tile1(kx + k + 16, e1);
-        }
-#pragma unroll
-        for (int j = 0; j < kSmallMaxUnits; ++j) {
-          if (j < nu) {
-            uint32_t b[4];
-            ldmatrix_x4(b[0], b[1], b[2], b[3], wsj[j] + k);
-            float(&o0)[4] = j == 0 ? acc2[0] : acc[j][0];
-            float(&o1)[4] = j == 0 ? acc2[1] : acc[j][1];
-            mma_bf16_16816(acc[j][0], a[0], a[1], a[2], a[3], b[0], b[1]);
-            mma_bf16_16816(o0, e[0], e[1], e[2], e[3], b[2], b[3]);
-            if (two) {
-              mma_bf16_16816(acc[j][1], a1[0], a1[1], a1[2], a1[3], b[0], b[1]);
-              mma_bf16_16816(o1, e1[0], e1[1], e1[2], e1[3], b[2], b[3]);
-            }
-          }
-        }
-      }
-      if (s < ks1) {   // odd step count (narrow K)
-        const int k = s * 16;
-        uint32_t a[4], a1[4];
-        ldmatrix_x4(a[0], a[1], a[2], a[3], xa0 + kx + k);
-        if (two) tile1(kx + k, a1);
-#pragma unroll
-        for (int j = 0; j < kSmallMaxUnits; ++j) {
-          if (j < nu) {
-            uint32_t b0, b1;
-            ldmatrix_x2(b0, b1, wsj[j] + k);
-            mma_bf16_16816(acc[j][0], a[0], a[1], a[2], a[3], b0, b1);
-            if (two) mma_bf16_16816(acc[j][1], a1[0], a1[1], a1[2], a1[3], b0, b1);
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0)
-        for (int j = 0; j < nu; ++j) mbar_arrive(&R.empty[(base + (uint32_t)(c * nu + j)) % kSmallSlots]);
-    }
+  float acc[kSmallMaxUnits][2][4];
+  SmallMmaIn in{xa0, xb_lo, xb_hi, lo1, hi1, two, wrow, ks0, ks1, kc, nch, base};
+  switch (nu) {
+    case 1: small_mma_units<1, 4>(in, smem, R, P, ok, acc); break;
+    case 2: small_mma_units<2, 4>(in, smem, R, P, ok, acc); break;
+    case 3: small_mma_units<3, 2>(in, smem, R, P, ok, acc); break;
+    default: small_mma_units<4, 2>(in, smem, R, P, ok, acc); break;
   }
   item = base + (uint32_t)(nch * nu);
   // all warps stay together from here on, also on a timeout
   cp_async_wait<0>();   // bias / old values
   csync();
   float* red = reinterpret_cast<float*>(smem);   // over the X area, no longer read
-#pragma unroll
-  for (int t = 0; t < 2; ++t)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) acc[0][t][e] += acc2[t][e];
 #pragma unroll
   for (int j = 0; j < kSmallMaxUnits; ++j) {
     if (j < nu) {
@@ -859,95 +957,154 @@ __device__ __forceinline__ bool small_gemm_phase(const SmallGemm& g, const AttnA
 
 // ---------------------------------------------------------------- attention phase (one CTA per head)
 
+// Byte offset of 16-byte column chunk c of key row r in a TMA box of
+// head_dim-wide bf16 rows: the 128-byte swizzle for 128-byte rows (DH 64),
+// the 64-byte swizzle for 64-byte rows (DH 32).
 template <int DH>
-struct SmallAttnSmem {
-  using SM = AttnSmem<2, DH>;
-  // Q tile, a K/V ring per warp (each warp's partial O later overwrites its
-  // own ring), per-warp (max, sum) per row
-  static constexpr int RING_BYTES = SM::RING_ELEMS * 2;
-  static constexpr int O_BYTES = 32 * DH * 4;
-  static constexpr int TOTAL = (SM::Q_ELEMS + kSmallWarps * SM::RING_ELEMS) * 2 + kSmallWarps * 32 * 2 * 4;
-  static_assert(O_BYTES <= RING_BYTES, "a warp's partial output fits its ring");
-  static_assert(TOTAL <= kSmXBytes, "attention fits the X area");
-};
+__device__ __forceinline__ int small_kv_swz(int r, int c) {
+  if constexpr (DH == 64)
+    return r * 128 + ((c ^ (r & 7)) << 4);
+  else
+    return r * 64 + ((c ^ ((r >> 1) & 3)) << 4);
+}
 
+// Cross attention of one head on this CTA (B = 1).  Warp 0 requests the
+// head's K and V rows as 2-D TMA boxes of kSmallAttnKB keys (up to
+// kSmallAttnBlocks boxes of each at a time: longer key lists take several
+// passes); the box rows past the last key are zeroed once they land, so
+// their products are finite and masked.  Warp w folds the 16-key chunks
+// w, w + 8, ... of the resident keys into its online softmax; the 8 warps'
+// partial results are combined at the end (over the K/V area).
 template <int DH>
-__device__ __forceinline__ void small_attention_phase(const AttnArgs& a, int head, uint8_t* smem) {
-  using SM = AttnSmem<2, DH>;
-  using SS = SmallAttnSmem<DH>;
+__device__ __forceinline__ bool small_cross_attention(const SmallPhase& ph, const SmallCtx& P, int head,
+                                                      uint8_t* smem, uint64_t* xbar, uint32_t& xuse, int* fail) {
   constexpr int NW = kSmallWarps;
+  constexpr int BOX = kSmallAttnKB * DH * 2;
+  const AttnArgs& a = ph.a;
   __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem);
-  __nv_bfloat16* sKV = sQ + SM::Q_ELEMS;
-  float* sML = reinterpret_cast<float*>(smem + (SM::Q_ELEMS + NW * SM::RING_ELEMS) * 2);
+  float* sML = reinterpret_cast<float*>(smem + kSmAttnML);
+  // the swizzle pattern follows absolute shared-memory address bits: boxes
+  // start on a 1024-byte boundary
+  const uint32_t kv0 = smem_u32(smem + kSmAttnKV);
+  uint8_t* sK = smem + kSmAttnKV + (((kv0 + 1023u) & ~1023u) - kv0);
+  uint8_t* sV = sK + kSmallAttnBlocks * BOX;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gr = lane >> 2, tig = lane & 3;
   int k_begin, n_keys;
   attn_key_range(a, 0, k_begin, n_keys);
+  const int krow = ph.kv_row + head * (int)P.max_tok + k_begin;
+  const int vrow = ph.kv_row + (P.nh + head) * (int)P.max_tok + k_begin;
   attn_load_q<2, DH>(a, 0, head, sQ, threadIdx.x, kSmallCompute);
-  csync();
   float o[2][DH / 8][4];
   float mrow[2][2], lrow[2][2];
   attn_init<2, DH>(o, mrow, lrow);
-  __nv_bfloat16* ring = sKV + warp * SM::RING_ELEMS;
-  attn_stream_chunks<2, DH>(a, head, k_begin, n_keys, warp, NW, sQ, ring, o, mrow, lrow);
-  __syncwarp();   // the warp's ring is free: its partial output goes there
-  float* sO = reinterpret_cast<float*>(ring);
-#pragma unroll
-  for (int mt = 0; mt < 2; ++mt) {
-#pragma unroll
-    for (int hr = 0; hr < 2; ++hr) {
-      float l = lrow[mt][hr];
-      l += __shfl_xor_sync(0xffffffffu, l, 1);
-      l += __shfl_xor_sync(0xffffffffu, l, 2);
-      const int row = mt * 16 + gr + hr * 8;
-      if (tig == 0) {
-        sML[(warp * 32 + row) * 2 + 0] = mrow[mt][hr];
-        sML[(warp * 32 + row) * 2 + 1] = l;
-      }
-      float* orow = sO + row * DH;
-#pragma unroll
-      for (int nd = 0; nd < DH / 8; ++nd) {
-        orow[nd * 8 + tig * 2 + 0] = o[mt][nd][hr * 2 + 0];
-        orow[nd * 8 + tig * 2 + 1] = o[mt][nd][hr * 2 + 1];
+  const int nblk = (n_keys + kSmallAttnKB - 1) / kSmallAttnKB;
+  bool ok = true;
+  for (int b0 = 0; b0 < nblk; b0 += kSmallAttnBlocks) {
+    const int nb = min(kSmallAttnBlocks, nblk - b0);
+    if (threadIdx.x == 0) {
+      fence_proxy_async_smem();   // earlier reads of the area precede the copies
+      mbar_arrive_expect_tx(xbar, (uint32_t)(2 * nb * BOX));
+      for (int b = 0; b < nb; ++b) {
+        tma_load_2d(sK + b * BOX, P.kv_map, xbar, 0, krow + (b0 + b) * kSmallAttnKB);
+        tma_load_2d(sV + b * BOX, P.kv_map, xbar, 0, vrow + (b0 + b) * kSmallAttnKB);
       }
     }
-  }
-  csync();
-  __nv_bfloat16* obase = a.out + head * DH;
-  for (int i = threadIdx.x; i < a.n_tok * (DH / 2); i += kSmallCompute) {
-    const int row = i / (DH / 2);
-    const int d = (i - row * (DH / 2)) * 2;
-    float mt = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) mt = fmaxf(mt, sML[(w * 32 + row) * 2]);
-    float r0 = 0.0f, r1 = 0.0f;
-    if (mt != -INFINITY) {
-      float l = 0.0f;
-#pragma unroll
-      for (int w = 0; w < NW; ++w) {
-        const float mw = sML[(w * 32 + row) * 2];
-        const float f = (mw == -INFINITY) ? 0.0f : exp2f(mw - mt);
-        const float* ow = reinterpret_cast<const float*>(sKV + w * SM::RING_ELEMS) + row * DH;
-        l += f * sML[(w * 32 + row) * 2 + 1];
-        r0 += f * ow[d];
-        r1 += f * ow[d + 1];
-      }
-      const float inv = 1.0f / l;
-      r0 *= inv;
-      r1 *= inv;
+    if (!mbar_wait(xbar, xuse & 1u, P.err)) *fail = 1;
+    ++xuse;
+    // rows past the last key (in the last box) hold other tokens or nothing
+    // written yet: zero them (K and V)
+    const int valid = min(n_keys - b0 * kSmallAttnKB, nb * kSmallAttnKB);
+    for (int i = threadIdx.x; i < (nb * kSmallAttnKB - valid) * (DH / 8); i += kSmallCompute) {
+      const int r = valid + i / (DH / 8), c = i % (DH / 8);
+      const int off = (r / kSmallAttnKB) * BOX + small_kv_swz<DH>(r % kSmallAttnKB, c);
+      *reinterpret_cast<uint4*>(sK + off) = make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4*>(sV + off) = make_uint4(0, 0, 0, 0);
     }
-    *reinterpret_cast<uint32_t*>(obase + (size_t)row * a.out_ld + d) = pack_bf16x2(r0, r1);
+    csync();
+    ok = *fail == 0;
+    if (!ok) break;
+    for (int ch = warp; ch * 16 < valid; ch += NW) {
+      const int r0 = ch * 16;   // first row of the chunk among the resident keys
+      attn_fold_chunk<2, DH>(
+          a, b0 * kSmallAttnKB + r0, k_begin, n_keys, sQ,
+          [&](int r, int c) {
+            const int rr = r0 + r;
+            return sK + (rr / kSmallAttnKB) * BOX + small_kv_swz<DH>(rr % kSmallAttnKB, c);
+          },
+          [&](int r, int c) {
+            const int rr = r0 + r;
+            return sV + (rr / kSmallAttnKB) * BOX + small_kv_swz<DH>(rr % kSmallAttnKB, c);
+          },
+          o, mrow, lrow);
+    }
+    csync();   // the boxes are rewritten by the next pass, or by the partial results
   }
-  // one barrier ends the phase (as for a GEMM phase): stores before the
-  // arrival, shared memory and the descriptor slot free afterwards
+  if (ok) {
+    // per-warp partial results -> shared memory (over the K/V boxes), then the
+    // combination across warps, bf16 rows of the head's output columns
+    float* sO = reinterpret_cast<float*>(sK) + warp * 32 * DH;
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        float l = lrow[mt][hr];
+        l += __shfl_xor_sync(0xffffffffu, l, 1);
+        l += __shfl_xor_sync(0xffffffffu, l, 2);
+        const int row = mt * 16 + gr + hr * 8;
+        if (tig == 0) {
+          sML[(warp * 32 + row) * 2 + 0] = mrow[mt][hr];
+          sML[(warp * 32 + row) * 2 + 1] = l;
+        }
+        float* orow = sO + row * DH;
+#pragma unroll
+        for (int nd = 0; nd < DH / 8; ++nd) {
+          orow[nd * 8 + tig * 2 + 0] = o[mt][nd][hr * 2 + 0];
+          orow[nd * 8 + tig * 2 + 1] = o[mt][nd][hr * 2 + 1];
+        }
+      }
+    }
+    csync();
+    __nv_bfloat16* obase = a.out + head * DH;
+    for (int i = threadIdx.x; i < a.n_tok * (DH / 2); i += kSmallCompute) {
+      const int row = i / (DH / 2);
+      const int d = (i - row * (DH / 2)) * 2;
+      float mt = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) mt = fmaxf(mt, sML[(w * 32 + row) * 2]);
+      float r0 = 0.0f, r1 = 0.0f;
+      if (mt != -INFINITY) {
+        float l = 0.0f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+          const float mw = sML[(w * 32 + row) * 2];
+          const float f = (mw == -INFINITY) ? 0.0f : exp2f(mw - mt);
+          const float* ow = reinterpret_cast<const float*>(sK) + (w * 32 + row) * DH;
+          l += f * sML[(w * 32 + row) * 2 + 1];
+          r0 += f * ow[d];
+          r1 += f * ow[d + 1];
+        }
+        const float inv = 1.0f / l;
+        r0 *= inv;
+        r1 *= inv;
+      }
+      *reinterpret_cast<uint32_t*>(obase + (size_t)row * a.out_ld + d) = pack_bf16x2(r0, r1);
+    }
+  }
+  // one barrier ends the phase: stores before the arrival, shared memory and
+  // the descriptor slot free afterwards
   cp_async_wait<0>();
   csync();
+  return *fail == 0;
 }
 
 template <int DH>
 struct SmallSmem {
   static constexpr int TOTAL = kSmallSmem;
-  static_assert(SmallAttnSmem<DH>::TOTAL <= kSmXBytes, "attention fits the X area");
+  static_assert(32 * (DH + 8) * 2 <= kSmAttnML && kSmAttnML + kSmallWarps * 32 * 2 * 4 <= kSmAttnKV,
+                "attention Q tile and (max, sum) fit before the K/V boxes");
+  static_assert(kSmallWarps * 32 * DH * 4 <= kSmallAttnBlocks * kSmallAttnKB * DH * 2,
+                "the warps' partial outputs fit the K boxes");
 };
 
 __device__ __forceinline__ int small_category(const SmallPlan& P) {
@@ -991,7 +1148,8 @@ __global__ void __launch_bounds__(kSmallThreads, 1) small_loop_kernel(const Smal
   __shared__ __align__(8) uint64_t s_xbar;
   __shared__ int s_ok;
   __shared__ int s_fail;
-  const SmallCtx P = {plan->err, plan->counters, plan->h, plan->eps, plan->phases, plan->vofs, plan->dh};
+  const SmallCtx P = {plan->err,  plan->counters, plan->h,  plan->eps,     plan->phases,
+                      plan->vofs, plan->dh,       plan->nh, plan->max_tok, &plan->kv_map};
   const int total = small_phases_per_step(plan->L) * plan->K;
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSmallSlots; ++i) {
@@ -1026,7 +1184,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1) small_loop_kernel(const Smal
         if (cur.kind == 0)
           ok = small_gemm_phase(cur.g, cur.a, P, smem, s_ring, item, &s_xbar, xuse, &s_fail);
         else
-          small_attention_phase<DH>(cur.a, blockIdx.x, smem);
+          ok = small_cross_attention<DH>(cur, P, blockIdx.x, smem, &s_xbar, xuse, &s_fail);
         if (ok) small_arrive(P, gp);
       }
     }

@@ -72,6 +72,7 @@ extern "C" {
 #define GDIT_FLAG_NO_SMALL 4u         /* never use the single-sample persistent loop (batch 1 then runs the
                                          same per-layer kernels as larger batches) */
 #define GDIT_FLAG_NO_TMA_STORE 8u     /* DiT GEMMs store their outputs thread by thread instead of by TMA */
+#define GDIT_FLAG_NO_PAIR 16u         /* DiT GEMMs never run on CTA pairs (cta_group::2, 256-row tiles) */
 
 /* ------------------------------------------------------------------ config
  * Model geometry and capacity.  Every size is explicit.  Defaults of the

@@ -274,3 +274,13 @@ def test_gemm_hooks_reject_null_matrices_on_the_host(L):
     for f in (L.gdit_test_gemm, L.gdit_gemm_static_scratch):
         assert f(None, None, None, None, 128, 128, 64, 128, 1, None) == _lib.GDIT_EINVAL
         assert "NULL matrix" in L.gdit_last_error(None).decode()
+
+
+@pytest.mark.parametrize("spec", ["alloc", "alloc:0", "alloc:x", "disk:3", "graph:2,upload:-1"])
+def test_malformed_fault_injection_spec_is_rejected(L, tinyW, monkeypatch, spec):
+    """GDIT_FAULT (host-side fault injection) is parsed before any device
+    call: a malformed value is an invalid argument, named in the message."""
+    monkeypatch.setenv("GDIT_FAULT", spec)
+    rc, h, err = _create(L, _cfg(synth.GEOM_TINY), tinyW)
+    assert rc == _lib.GDIT_EINVAL and not h.value
+    assert "GDIT_FAULT" in err

@@ -38,6 +38,31 @@ def test_gemm_matches_float64(M, N, K, bn, splits, tma_out, monkeypatch):
     np.testing.assert_allclose(C, ref, rtol=1e-5, atol=2e-5 * np.sqrt(K))
 
 
+@pytest.mark.parametrize("M,N,K,bn", [
+    (256, 256, 64, 256),           # one pair tile, one K block
+    (4352, 1024, 1024, 256),       # the DiT shape at B = 256 (17 row blocks of 256)
+    (4352, 4096, 1024, 256),       # FF1: more pair tiles than clusters (persistent)
+    (544, 3072, 1024, 256),        # ragged last row block (544 = 2 x 256 + 32)
+    (300, 512, 2048, 128),         # narrow pair tiles, long K, ragged rows
+    (130, 256, 40, 128),           # the odd CTA's rows mostly past the end; K below one block
+])
+def test_pair_gemm_matches_float64(M, N, K, bn, monkeypatch):
+    """The CTA-pair kernel (cta_group::2 MMAs over two SMs, 256-row tiles,
+    TMA-store epilogue) against float64 products of the same bf16 inputs."""
+    require_gpu()
+    monkeypatch.setenv("GDIT_TEST_TMA_OUT", "1")
+    monkeypatch.setenv("GDIT_TEST_PAIR", "1")
+    import torch
+    from flow_matching_dit_b200 import test_gemm
+    g = torch.Generator().manual_seed(M * 5 + N + K)
+    A = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    B = torch.randn(N, K, generator=g).to(torch.bfloat16)
+    bias = torch.randn(N, generator=g)
+    C = test_gemm(A.cuda(), B.cuda(), bias.cuda(), bn=bn, splits=1).cpu().double().numpy()
+    ref = A.double().numpy() @ B.double().numpy().T + bias.double().numpy()
+    np.testing.assert_allclose(C, ref, rtol=1e-5, atol=2e-5 * np.sqrt(K))
+
+
 def test_gemm_rejects_bad_shapes():
     require_gpu()
     import torch

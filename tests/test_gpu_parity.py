@@ -344,6 +344,35 @@ def test_tma_store_epilogue_is_bitwise_equal_to_thread_stores(full_weights):
     np.testing.assert_array_equal(x, y)
 
 
+def test_pair_gemms_match_single_cta_gemms(head_full, full_weights):
+    """At B = 256 the DiT GEMMs run on CTA pairs (cta_group::2, 256-row tiles);
+    with GDIT_FLAG_NO_PAIR they run on single CTAs.  Both sum the same bf16
+    products in f32 in the same K order, so the actions agree to rounding."""
+    from flow_matching_dit_b200 import GDIT_FLAG_NO_PAIR, ActionHead
+    w = synth.WORKLOADS["sweep256"]
+    inp = synth.make_inputs(w, seed=37)
+    x, st = run_gpu(head_full, inp, w.num_steps)
+    assert st == 0
+    with ActionHead(w.geom, full_weights, max_batch=256, max_seq=256, flags=GDIT_FLAG_NO_PAIR) as b:
+        y, st2 = run_gpu(b, inp, w.num_steps)
+    assert st2 == 0
+    print("pair vs single-CTA max |diff|", float(np.abs(x - y).max()))
+    np.testing.assert_allclose(x, y, rtol=0, atol=1e-3)
+
+
+def test_cross_attention_on_ragged_keys_at_64_samples(head_full, full_weights, full_model):
+    """64 samples with valid lengths 200..600 padded to 600: 1024 (sample,
+    head) items, the warp schedule of the cross attention over ragged key
+    lists, against the oracle on rows spread over the batch."""
+    w = synth.workload("batched", batch=64)
+    inp = synth.make_inputs(w, seed=43)
+    x, st = run_gpu(head_full, inp, w.num_steps)
+    assert st == 0
+    rows = [0, 9, 33, 63]
+    ref = run_oracle(full_weights, w.geom, inp, w.num_steps, samples=rows, model=full_model)
+    assert_parity(x[rows], ref, inp["init_noise"][rows], "cross attention, B=64 ragged")
+
+
 def test_bounded_wait_expiry_is_reported_and_the_device_stays_usable(head_tiny, tiny_weights):
     """A wait on an mbarrier that nothing arrives at, through the library's
     bounded wait with a 1 ms limit: it gives up, reports GDIT_ETIMEOUT, and the
