@@ -31,7 +31,7 @@ struct AttnArgs {
   const __nv_bfloat16* v;
   long long kv_ld;          // row stride of K and V
   long long kv_head_stride; // offset between heads of K (and of V)
-  const int* kofs;      // cross: keys of sample b are rows [kofs[b], kofs[b+1]); nullptr: self (rows of q's sample)
+  const int* kspan;     // cross: keys of sample b are rows [kspan[2b], kspan[2b+1]); nullptr: self (rows of q's sample)
   int n_tok;            // queries (tokens) per sample
   int num_heads;
   int num_items;        // samples * heads
@@ -99,9 +99,9 @@ __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t& r0, uint32_t& r1, ui
 }
 
 __device__ __forceinline__ void attn_key_range(const AttnArgs& a, int b, int& k_begin, int& n_keys) {
-  if (a.kofs != nullptr) {
-    k_begin = a.kofs[b];
-    n_keys = a.kofs[b + 1] - k_begin;
+  if (a.kspan != nullptr) {
+    k_begin = a.kspan[2 * b];
+    n_keys = a.kspan[2 * b + 1] - k_begin;
   } else {
     k_begin = b * a.n_tok;
     n_keys = a.n_tok;

@@ -299,6 +299,7 @@ GemmArgs default_args() {
 }
 
 constexpr long long kWsFloats = 16ll << 20;   // split-K partials (64 MB)
+constexpr int kHostChunks = 4;                // sample chunks of the host-buffer entry point
 constexpr int kSmallMaxPhases = 64 * (5 * kSmallMaxLayers + 6);
 constexpr int kCounters = 1 << 16;
 
@@ -360,7 +361,8 @@ struct Profile {
   int B, S, K, bf16;
   GemmOp kv, st1, st2, a1, a2, a3, proj, d1, d2;
   std::vector<GemmOp> q, o, ff1, ff2;
-  cudaGraphExec_t exec = nullptr;
+  cudaGraphExec_t exec = nullptr;        // the whole call
+  cudaGraphExec_t exec_main = nullptr;   // the call after the K/V projection (host-buffer entry point)
   // single-sample profiles run the K-step loop as one persistent kernel
   bool small = false;
   SmallPlan* small_plan = nullptr;   // device copy
@@ -407,7 +409,7 @@ struct gdit_handle {
   __nv_bfloat16 *xp, *kv, *u, *qkv, *o, *f, *xb, *abf, *zbf, *ybf, *rbf, *sb, *s1;
   uint8_t* kflag;           // image flag of each packed backbone token
   float *h, *x, *sfeat, *ws;
-  int *perm, *seg, *vofs, *counters;
+  int *perm, *seg, *vofs, *kspan, *counters;
   int* phase_counters;      // per-phase arrival counters of the single-sample loop
   SmallPhase* phase_table;  // per-phase descriptors of the single-sample loop
   uint8_t* bad;
@@ -421,7 +423,11 @@ struct gdit_handle {
   cudaStream_t cap_stream = nullptr;
   cudaStream_t last_stream = nullptr;
 
-  // host-buffer staging (gdit_get_action_host)
+  // host-buffer staging (gdit_get_action_host): the features are copied in
+  // sample chunks on copy_stream, each chunk packed and projected to K/V as
+  // soon as it has landed
+  cudaStream_t copy_stream = nullptr;
+  cudaEvent_t chunk_ev[kHostChunks] = {};
   void* st_feats = nullptr;
   size_t st_feats_bytes = 0;
   uint8_t* st_mask = nullptr;
@@ -782,6 +788,7 @@ void alloc_workspace(gdit_handle* h) {
   h->perm = h->dalloc<int>((size_t)Bm);
   h->seg = h->dalloc<int>((size_t)h->C + 1);
   h->vofs = h->dalloc<int>((size_t)Bm + 1);
+  h->kspan = h->dalloc<int>((size_t)2 * Bm);
   h->bad = h->dalloc<uint8_t>((size_t)Bm);
   h->status = h->dalloc<unsigned>(1);
   h->io = h->dalloc<IoPtrs>(1);
@@ -1097,7 +1104,7 @@ std::unique_ptr<Profile> build_profile(gdit_handle* h, int B, int S, int K, int 
     sp.max_tok = h->max_tok;
     sp.h = h->h; sp.x = h->x; sp.xb = h->xb;
     sp.abf = h->abf; sp.zbf = h->zbf; sp.qkv = h->qkv; sp.o = h->o; sp.f = h->f; sp.ybf = h->ybf; sp.rbf = h->rbf;
-    sp.sfeat = h->sfeat; sp.seg = h->seg; sp.vofs = h->vofs; sp.kflag = h->kflag;
+    sp.sfeat = h->sfeat; sp.seg = h->seg; sp.vofs = h->vofs; sp.kspan = h->kspan; sp.kflag = h->kflag;
     sp.text_every = h->cfg.attend_text_every_n_blocks;
     sp.ada = t.ada; sp.tw2 = t.tw2;
     sp.wa1t = m.wa1t; sp.wa2at = m.wa2at; sp.wa3t = m.wa3t; sp.wd1t = m.wd1t; sp.wd2t = m.wd2t; sp.proj_w = m.proj_w;
@@ -1151,7 +1158,28 @@ struct Launcher {
   }
 };
 
-void enqueue_forward(gdit_handle* h, Profile& p, cudaStream_t s, Recorder* rec) {
+// Valid backbone tokens of samples [b0, b0 + nb) -> packed rows (caller order).
+void launch_pack(gdit_handle* h, cudaStream_t s, int bf16, int S, int b0, int nb) {
+  launch_k(s, h->pdl, pack_features_kernel, dim3(nb, (S + 31) / 32), dim3(kPackThreads), 0, (const IoPtrs*)h->io,
+           bf16, S, h->Dvl, b0, (const int*)h->vofs, h->xp, h->kflag);
+}
+
+// The vision-language LayerNorm of every packed token (only with its weights).
+void launch_vlln(gdit_handle* h, cudaStream_t s, int B, int S) {
+  const dim3 grid((unsigned)(((long long)B * S + 7) / 8));
+  const int* tot = (const int*)h->vofs + B;
+  const float e = h->cfg.ln_eps;
+  const bool pdl = h->pdl;
+  switch (h->Dvl / 256) {
+    case 1: launch_k(s, pdl, vlln_kernel<1>, grid, dim3(256), 0, h->xp, tot, h->w.vlln_g, h->w.vlln_b, e); break;
+    case 2: launch_k(s, pdl, vlln_kernel<2>, grid, dim3(256), 0, h->xp, tot, h->w.vlln_g, h->w.vlln_b, e); break;
+    case 4: launch_k(s, pdl, vlln_kernel<4>, grid, dim3(256), 0, h->xp, tot, h->w.vlln_g, h->w.vlln_b, e); break;
+    case 8: launch_k(s, pdl, vlln_kernel<8>, grid, dim3(256), 0, h->xp, tot, h->w.vlln_g, h->w.vlln_b, e); break;
+    default: launch_k(s, pdl, vlln_kernel<16>, grid, dim3(256), 0, h->xp, tot, h->w.vlln_g, h->w.vlln_b, e); break;
+  }
+}
+
+void enqueue_forward(gdit_handle* h, Profile& p, cudaStream_t s, Recorder* rec, bool prologue = true) {
   Launcher lx{h, s, rec};
   const int B = p.B, S = p.S, K = p.K;
   const int D = h->D, N = h->N, H = h->H, A = h->A, L = h->L, C = h->C, Dvl = h->Dvl;
@@ -1204,34 +1232,23 @@ void enqueue_forward(gdit_handle* h, Profile& p, cudaStream_t s, Recorder* rec) 
   };
   const bool cross_warp_sched = B * h->cfg.num_heads >= 4 * h->num_sms;
 
-  // routing, packing, gathers
-  lx.timed("route_pack", 0, 0, nullptr, [&] {
-    launch_k(s, pdl, route_kernel, dim3(1), dim3(kRouteThreads), 0, (const IoPtrs*)h->io, B, S, C, h->perm, h->seg,
-             h->vofs, h->bad, h->status);
-  });
-  lx.timed("route_pack", 0, (double)B * S * Dvl * (p.bf16 ? 4 : 6), nullptr, [&] {
-    launch_k(s, pdl, pack_features_kernel, dim3(B, (S + 31) / 32), dim3(kPackThreads), 0, (const IoPtrs*)h->io,
-             p.bf16, S, Dvl, (const int*)h->perm, (const int*)h->vofs, h->xp, h->kflag);
-  });
-  if (h->w.vlln_g != nullptr) {
-    lx.timed("vlln", 0, (double)B * S * Dvl * 4, nullptr, [&] {
-      const dim3 grid((unsigned)(((long long)B * S + 7) / 8));
-      const int* tot = (const int*)h->vofs + B;
-      const float e = h->cfg.ln_eps;
-      switch (Dvl / 256) {
-        case 1: launch_k(s, pdl, vlln_kernel<1>, grid, dim3(256), 0, h->xp, tot, h->w.vlln_g, h->w.vlln_b, e); break;
-        case 2: launch_k(s, pdl, vlln_kernel<2>, grid, dim3(256), 0, h->xp, tot, h->w.vlln_g, h->w.vlln_b, e); break;
-        case 4: launch_k(s, pdl, vlln_kernel<4>, grid, dim3(256), 0, h->xp, tot, h->w.vlln_g, h->w.vlln_b, e); break;
-        case 8: launch_k(s, pdl, vlln_kernel<8>, grid, dim3(256), 0, h->xp, tot, h->w.vlln_g, h->w.vlln_b, e); break;
-        default: launch_k(s, pdl, vlln_kernel<16>, grid, dim3(256), 0, h->xp, tot, h->w.vlln_g, h->w.vlln_b, e); break;
-      }
+  // routing, packing and the K/V projection of the backbone tokens (the
+  // host-buffer entry point runs these itself, overlapped with the copies)
+  if (prologue) {
+    lx.timed("route_pack", 0, 0, nullptr, [&] {
+      launch_k(s, pdl, route_kernel, dim3(1), dim3(kRouteThreads), 0, (const IoPtrs*)h->io, B, S, C, h->perm, h->seg,
+               h->vofs, h->kspan, h->bad, h->status);
     });
+    lx.timed("route_pack", 0, (double)B * S * Dvl * (p.bf16 ? 4 : 6), nullptr,
+             [&] { launch_pack(h, s, p.bf16, S, 0, B); });
+    if (h->w.vlln_g != nullptr)
+      lx.timed("vlln", 0, (double)B * S * Dvl * 4, nullptr, [&] { launch_vlln(h, s, B, S); });
+    lx.gemm("gemm_kv_proj", p.kv);
   }
   lx.timed("route_pack", 0, 0, nullptr, [&] {
     launch_k(s, pdl, gather_inputs_kernel, dim3(B), dim3(128), 0, (const IoPtrs*)h->io, B, H * A, h->Sd,
              (const int*)h->perm, h->x, h->xb, h->sb);
   });
-  lx.gemm("gemm_kv_proj", p.kv);
   lx.gemm("gemm_embodiment", p.st1);
   lx.gemm("gemm_embodiment", p.st2);
 
@@ -1293,7 +1310,7 @@ void enqueue_forward(gdit_handle* h, Profile& p, cudaStream_t s, Recorder* rec) 
         aa.v = h->qkv + 2 * D;
         aa.kv_ld = 3 * D;
         aa.kv_head_stride = h->cfg.head_dim;
-        aa.kofs = nullptr;
+        aa.kspan = nullptr;
         attn("attn_self", aa, true);
       } else {
         const __nv_bfloat16* kvl = h->kv + (size_t)(l / 2) * h->max_tok * 2 * D;
@@ -1302,7 +1319,7 @@ void enqueue_forward(gdit_handle* h, Profile& p, cudaStream_t s, Recorder* rec) 
         aa.v = kvl + (size_t)h->cfg.num_heads * h->max_tok * h->cfg.head_dim;
         aa.kv_ld = h->cfg.head_dim;
         aa.kv_head_stride = h->max_tok * h->cfg.head_dim;
-        aa.kofs = h->vofs;
+        aa.kspan = h->kspan;
         attn("attn_cross", aa, cross_warp_sched);
       }
       lx.gemm("gemm_dit", p.o[l]);
@@ -1331,23 +1348,33 @@ Profile& get_profile(gdit_handle* h, int B, int S, int K, int bf16, bool allow_b
   auto p = build_profile(h, B, S, K, bf16);
   if (h->use_graph) {
     if (h->cap_stream == nullptr) CUDA_TRY(cudaStreamCreateWithFlags(&h->cap_stream, cudaStreamNonBlocking));
-    cudaGraph_t graph = nullptr;
-    CUDA_TRY(cudaStreamBeginCapture(h->cap_stream, cudaStreamCaptureModeThreadLocal));
-    try {
-      enqueue_forward(h, *p, h->cap_stream, nullptr);
-    } catch (...) {
-      cudaStreamEndCapture(h->cap_stream, &graph);
-      if (graph) cudaGraphDestroy(graph);
-      throw;
-    }
-    CUDA_TRY(cudaStreamEndCapture(h->cap_stream, &graph));
-    if (++h->fault.n_graph == h->fault.graph) {
+    // the whole call, and the call after the K/V projection
+    for (int part = 0; part < 2; ++part) {
+      cudaGraph_t graph = nullptr;
+      CUDA_TRY(cudaStreamBeginCapture(h->cap_stream, cudaStreamCaptureModeThreadLocal));
+      try {
+        enqueue_forward(h, *p, h->cap_stream, nullptr, part == 0);
+      } catch (...) {
+        cudaStreamEndCapture(h->cap_stream, &graph);
+        if (graph) cudaGraphDestroy(graph);
+        if (p->exec) cudaGraphExecDestroy(p->exec);
+        throw;
+      }
+      CUDA_TRY(cudaStreamEndCapture(h->cap_stream, &graph));
+      if (++h->fault.n_graph == h->fault.graph) {
+        cudaGraphDestroy(graph);
+        if (p->exec) cudaGraphExecDestroy(p->exec);
+        throw GditError(GDIT_ECUDA, fmt("injected fault: graph instantiation %lld failed", h->fault.n_graph));
+      }
+      cudaGraphExec_t& ex = part == 0 ? p->exec : p->exec_main;
+      cudaError_t e = cudaGraphInstantiate(&ex, graph, 0);
       cudaGraphDestroy(graph);
-      throw GditError(GDIT_ECUDA, fmt("injected fault: graph instantiation %lld failed", h->fault.n_graph));
+      if (e != cudaSuccess && p->exec && part == 1) {
+        cudaGraphExecDestroy(p->exec);
+        p->exec = nullptr;
+      }
+      CUDA_TRY(e);
     }
-    cudaError_t e = cudaGraphInstantiate(&p->exec, graph, 0);
-    cudaGraphDestroy(graph);
-    CUDA_TRY(e);
   }
   Profile& ref = *p;
   h->profiles[key] = std::move(p);
@@ -1407,9 +1434,14 @@ void free_handle(gdit_handle* h) {
   if (!h) return;
   cudaSetDevice(h->cfg.device);
   cudaDeviceSynchronize();
-  for (auto& kv : h->profiles)
+  for (auto& kv : h->profiles) {
     if (kv.second->exec) cudaGraphExecDestroy(kv.second->exec);
+    if (kv.second->exec_main) cudaGraphExecDestroy(kv.second->exec_main);
+  }
   if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
+  if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
+  for (cudaEvent_t e : h->chunk_ev)
+    if (e) cudaEventDestroy(e);
   for (void* p : h->allocs) cudaFree(p);
   delete h;
 }
@@ -1537,20 +1569,58 @@ int gdit_get_action_host(gdit_handle* h, const void* backbone_features, int bb_d
       h->st_noise = h->dalloc<float>(Bm * h->H * h->A);
       h->st_out = h->dalloc<float>(Bm * h->H * h->A);
     }
-    const size_t fbytes = (size_t)batch * seq * h->Dvl * esz;
+    const size_t sample_bytes = (size_t)seq * h->Dvl * esz;
+    const size_t fbytes = (size_t)batch * sample_bytes;
     if (h->st_feats_bytes < fbytes) {
       const size_t cap = Bm * Sm * h->Dvl * esz;
       h->st_feats = h->dalloc<uint8_t>(std::max(cap, fbytes));
       h->st_feats_bytes = std::max(cap, fbytes);
     }
+    if (h->copy_stream == nullptr) {
+      CUDA_TRY(cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking));
+      for (cudaEvent_t& e : h->chunk_ev) CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+    }
+    compute_tables(h, num_steps, s);
+    Profile& p = get_profile(h, batch, seq, num_steps, bb_dtype == GDIT_BF16, !h->strict);
     const size_t ha = (size_t)batch * h->H * h->A;
-    CUDA_TRY(cudaMemcpyAsync(h->st_feats, backbone_features, fbytes, cudaMemcpyHostToDevice, s));
+    // the small inputs first: routing needs the masks and ids
     CUDA_TRY(cudaMemcpyAsync(h->st_mask, vl_mask, (size_t)batch * seq, cudaMemcpyHostToDevice, s));
-    CUDA_TRY(cudaMemcpyAsync(h->st_state, state, (size_t)batch * h->Sd * 4, cudaMemcpyHostToDevice, s));
     CUDA_TRY(cudaMemcpyAsync(h->st_ids, embodiment_id, (size_t)batch * 4, cudaMemcpyHostToDevice, s));
+    CUDA_TRY(cudaMemcpyAsync(h->st_state, state, (size_t)batch * h->Sd * 4, cudaMemcpyHostToDevice, s));
     CUDA_TRY(cudaMemcpyAsync(h->st_noise, init_noise, ha * 4, cudaMemcpyHostToDevice, s));
-    run_call(h, h->st_feats, bb_dtype, h->st_mask, h->st_state, h->st_ids, h->st_noise, num_steps, h->st_out, batch,
-             seq, s);
+    IoPtrs io{h->st_feats, h->st_mask, h->st_state, h->st_ids, h->st_noise, h->st_out, nullptr};
+    set_io_kernel<<<1, 1, 0, s>>>(h->io, io);
+    CUDA_TRY(cudaGetLastError());
+    launch_k(s, h->pdl, route_kernel, dim3(1), dim3(kRouteThreads), 0, (const IoPtrs*)h->io, batch, seq, h->C,
+             h->perm, h->seg, h->vofs, h->kspan, h->bad, h->status);
+    // The features in sample chunks on the copy stream; each chunk is packed
+    // and projected to K/V on the compute stream once it has landed, while
+    // the next chunk is still being copied.  (With vlln weights the whole
+    // batch is one chunk: the LayerNorm runs over all packed rows.)
+    const int nch = h->w.vlln_g != nullptr ? 1 : std::min(kHostChunks, batch);
+    for (int c = 0; c < nch; ++c) {
+      const int b0 = (int)((long long)c * batch / nch), b1 = (int)((long long)(c + 1) * batch / nch);
+      CUDA_TRY(cudaMemcpyAsync(static_cast<uint8_t*>(h->st_feats) + (size_t)b0 * sample_bytes,
+                               static_cast<const uint8_t*>(backbone_features) + (size_t)b0 * sample_bytes,
+                               (size_t)(b1 - b0) * sample_bytes, cudaMemcpyHostToDevice, h->copy_stream));
+      CUDA_TRY(cudaEventRecord(h->chunk_ev[c], h->copy_stream));
+    }
+    for (int c = 0; c < nch; ++c) {
+      const int b0 = (int)((long long)c * batch / nch), b1 = (int)((long long)(c + 1) * batch / nch);
+      CUDA_TRY(cudaStreamWaitEvent(s, h->chunk_ev[c], 0));
+      launch_pack(h, s, bb_dtype == GDIT_BF16, seq, b0, b1 - b0);
+      if (h->w.vlln_g != nullptr) launch_vlln(h, s, batch, seq);
+      GemmArgs kv = p.kv.args;   // packed rows [vofs[b0], vofs[b1])
+      kv.m_begin_dev = h->vofs + b0;
+      kv.m_dev = h->vofs + b1;
+      launch_gemm(p.kv, kv, s, h->pdl);
+    }
+    if (p.exec_main != nullptr)
+      CUDA_TRY(cudaGraphLaunch(p.exec_main, s));
+    else
+      enqueue_forward(h, p, s, nullptr, false);
+    h->last_stream = s;
+    h->last_B = batch;
     CUDA_TRY(cudaMemcpyAsync(out_actions, h->st_out, ha * 4, cudaMemcpyDeviceToHost, s));
     CUDA_TRY(cudaStreamSynchronize(s));
   });

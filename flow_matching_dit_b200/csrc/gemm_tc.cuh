@@ -52,6 +52,7 @@ struct GemmArgs {
   int M;                    // rows of A (dense) or row capacity (grouped)
   int N, K;
   const int* m_dev;         // dense: optional device row count (<= M)
+  const int* m_begin_dev;   // dense with m_dev: optional first row (device): rows [*m_begin_dev, *m_dev)
   int num_groups;           // 0 = dense
   const int* seg;           // grouped: [num_groups + 1] sample offsets (device)
   int rows_per_sample;      // grouped: rows of A per sample
@@ -96,7 +97,8 @@ struct GemmSched {
   int units;          // output tiles (without the split factor)
   int nt;             // column tiles
   int mt;             // dense: row tiles
-  int rows;           // dense: valid rows
+  int rows;           // dense: end of the valid rows
+  int m_begin;        // dense: first row
   int uprefix[kMaxGroups + 1];
   int rstart[kMaxGroups];
   int rend[kMaxGroups];
@@ -121,7 +123,7 @@ __device__ __forceinline__ void gemm_decode(const GemmArgs& a, const GemmSched& 
     m_idx = first_m + r % gm;
     n_idx = r / gm;
     ti.g = 0;
-    ti.m0 = m_idx * kBM;
+    ti.m0 = s.m_begin + m_idx * kBM;
     ti.m_end = s.rows;
   } else {
     int g = 0;
@@ -147,8 +149,10 @@ __device__ __forceinline__ void gemm_build_sched(const GemmArgs& a, GemmSched& s
     int rows = a.M;
     if (a.m_dev != nullptr) rows = min(rows, *a.m_dev);
     rows = max(rows, 0);
+    const int begin = (a.m_dev != nullptr && a.m_begin_dev != nullptr) ? min(max(*a.m_begin_dev, 0), rows) : 0;
     sched.rows = rows;
-    sched.mt = (rows + kBM - 1) / kBM;
+    sched.m_begin = begin;
+    sched.mt = (rows - begin + kBM - 1) / kBM;
     sched.units = sched.mt * sched.nt;
   } else {
     int u = 0;

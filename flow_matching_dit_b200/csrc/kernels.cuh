@@ -30,14 +30,18 @@ __global__ void set_io_kernel(IoPtrs* dst, IoPtrs src) { *dst = src; }
 // contiguous for the grouped GEMMs:
 //   perm[i]  original index of the i-th sample in sorted order
 //   seg[c]   first sorted position of category c (seg[C] = B)
-//   vofs[i]  first packed valid backbone token of sorted sample i (vofs[B] = total)
+//   vofs[b]  first packed valid backbone token of sample b (vofs[B] = total):
+//            the tokens are packed in the caller's sample order, so that the
+//            packing and the K/V projection of a range of samples can start
+//            as soon as those samples' features have arrived
+//   kspan[2i], kspan[2i + 1]  the packed tokens [begin, end) of sorted sample i
 // An id outside [0, C) is routed to category 0 (never read out of bounds),
 // flagged in bad[b], and reported through the status word.
 constexpr int kRouteThreads = 1024;
 constexpr int kMaxBatch = 4096;
 
 __global__ void __launch_bounds__(kRouteThreads)
-    route_kernel(const IoPtrs* io, int B, int S, int C, int* perm, int* seg, int* vofs, uint8_t* bad,
+    route_kernel(const IoPtrs* io, int B, int S, int C, int* perm, int* seg, int* vofs, int* kspan, uint8_t* bad,
                  unsigned* status) {
   __shared__ int s_cnt[kMaxBatch];
   __shared__ int s_cat[kMaxBatch];
@@ -73,35 +77,40 @@ __global__ void __launch_bounds__(kRouteThreads)
     for (int c = 0; c <= C; ++c) seg[c] = s_pos[c];
     for (int b = 0; b < B; ++b) perm[s_pos[s_cat[b]]++] = b;   // stable: ties keep sample order
     int acc = 0;
-    for (int i = 0; i < B; ++i) {
-      vofs[i] = acc;
-      acc += s_cnt[perm[i]];
+    for (int b = 0; b < B; ++b) {
+      vofs[b] = acc;
+      acc += s_cnt[b];
     }
     vofs[B] = acc;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < B; i += kRouteThreads) {
+    const int b = perm[i];
+    kspan[2 * i] = vofs[b];
+    kspan[2 * i + 1] = vofs[b] + s_cnt[b];
   }
 }
 
 // ---------------------------------------------------------------- packing
 //
 // Copies the valid backbone tokens (vl_mask == 1; Isaac-GR00T architecture
-// page, backbone forward: attention_mask == 1) of each sample, in sorted
-// sample order, to a dense bf16 matrix Xp [total_valid, Dvl].  Only these rows
-// enter the K/V projection, so padding costs nothing downstream.
-// grid = (sorted sample, chunk of 32 positions).
+// page, backbone forward: attention_mask == 1) of samples b0, b0 + 1, ... in
+// the caller's sample order to a dense bf16 matrix Xp [total_valid, Dvl].
+// Only these rows enter the K/V projection, so padding costs nothing
+// downstream.  grid = (sample - b0, chunk of 32 positions).
 constexpr int kPackThreads = 256;
 
 __global__ void __launch_bounds__(kPackThreads)
-    pack_features_kernel(const IoPtrs* io, int bb_bf16, int S, int Dvl, const int* perm, const int* vofs,
-                         __nv_bfloat16* xp, uint8_t* kflag) {
+    pack_features_kernel(const IoPtrs* io, int bb_bf16, int S, int Dvl, int b0, const int* vofs, __nv_bfloat16* xp,
+                         uint8_t* kflag) {
   __shared__ int s_red[kPackThreads / 32];
   __shared__ int s_rows[32];
   __shared__ int s_n;
   __shared__ int s_before;
   pdl_wait();
   pdl_launch_dependents();
-  const int i = blockIdx.x;
+  const int b = b0 + blockIdx.x;
   const int j0 = blockIdx.y * 32;
-  const int b = perm[i];
   const uint8_t* mrow = io->mask + (long long)b * S;
   // valid tokens before this chunk
   int c = 0;
@@ -125,7 +134,7 @@ __global__ void __launch_bounds__(kPackThreads)
   }
   __syncthreads();
   const int n = s_n;
-  const long long dst0 = (long long)vofs[i] + s_before;
+  const long long dst0 = (long long)vofs[b] + s_before;
   // image flag of every packed token (the image/text split of the cross layers)
   if ((int)threadIdx.x < n)
     kflag[dst0 + threadIdx.x] =

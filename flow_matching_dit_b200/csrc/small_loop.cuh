@@ -111,6 +111,7 @@ struct SmallPlan {
   const float* sfeat;
   const int* seg;
   const int* vofs;
+  const int* kspan;          // [begin, end) of the sample's packed keys
   const uint8_t* kflag;      // image flag of each packed backbone token
   int text_every;            // attend_text_every_n_blocks (0: no image/text split)
   // per-K tables: AdaLN [K][L+1][2D], timestep term of the action encoder's W2 [K][C][D]
@@ -238,10 +239,10 @@ __device__ __forceinline__ void small_describe(const SmallPlan& P, int c, int k,
         a.ksel = (self || P.text_every <= 0) ? -1 : (l % (2 * P.text_every) == 0 ? 0 : 1);
         if (self) {
           a.q = P.qkv; a.q_ld = 3 * D; a.k = P.qkv + D; a.v = P.qkv + 2 * D; a.kv_ld = 3 * D;
-          a.kv_head_stride = P.dh; a.kofs = nullptr;
+          a.kv_head_stride = P.dh; a.kspan = nullptr;
         } else {
           a.q = P.qkv; a.q_ld = D; a.k = Ly.kv; a.v = Ly.kv + (size_t)P.nh * P.max_tok * P.dh; a.kv_ld = P.dh;
-          a.kv_head_stride = P.max_tok * P.dh; a.kofs = P.vofs;
+          a.kv_head_stride = P.max_tok * P.dh; a.kspan = P.kspan;
           ph.kv_row = (int)((long long)(l / 2) * 2 * P.nh * P.max_tok);
         }
         break;
@@ -376,7 +377,7 @@ __device__ __forceinline__ void small_producer(const SmallCtx& P, int total, uin
       for (int j = 0; j < nu; ++j)
         l2_prefetch_hint(g.W + (size_t)small_unit(j) * kSmallUF * g.K, (uint32_t)(kSmallUF * g.K * 2),
                          stream_policy);
-    } else if (ph.a.kofs != nullptr && (int)blockIdx.x < ph.a.num_heads) {
+    } else if (ph.a.kspan != nullptr && (int)blockIdx.x < ph.a.num_heads) {
       // K and V of this CTA's head: contiguous rows of the head-major cache
       const uint32_t bytes = (uint32_t)P.vofs[1] * (uint32_t)P.dh * 2u;
       if (bytes > 0) {
@@ -500,81 +501,60 @@ __device__ __forceinline__ void small_issue_ln(const SmallGemm& g, const SmallCt
   }
 }
 
-// LN(h rows) -> bf16 X rows, from the rows staged by small_issue_ln.  Thread
-// t owns columns [4t, 4t + 4) of every row: it reads them from shared memory
-// (consecutive threads, consecutive 16 bytes), the CTA reduces each row's sum
-// and sum of squares (warp shuffles, then the 8 warps' totals through shared
-// memory), and the thread writes its columns of every normalised row with the
-// AdaLN ((1 + p0), p1) or affine (p0, p1) modulation.
+// LN(h rows) -> bf16 X rows, from the rows staged by small_issue_ln, one
+// warp per row (rows warp, warp + 8, ...): each lane takes 32 of the row's
+// columns (float4 at column 4 (lane + 32 j)); the row's mean, then the mean of
+// the squared deviations (two passes over the staged row), are warp shuffle
+// reductions; the lane writes its columns of the normalised row with the
+// AdaLN ((1 + p0), p1) or affine (p0, p1) modulation.  A warp owns whole rows,
+// so no statistics cross warps: 10 shuffles per row instead of a CTA-wide
+// reduction of every row (the shuffles' latency bounded the LN here).
 __device__ __forceinline__ void small_ln_rows(const SmallGemm& g, const SmallCtx& P, uint8_t* smem) {
-  constexpr int G = 17;   // rows per round (N = H + 1 = 17 in one)
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int D = g.K, d4 = D / 4, xrow = D + 8;
-  const bool has = tid < d4;
-  static_assert((kSmallWarps * G * 2 + G * 2) * 4 <= kSmLnScratchBytes, "LN scratch");
-  float* part = reinterpret_cast<float*>(smem + kSmLnScratch);   // [warp][row][2]
-  float* stat = part + kSmallWarps * G * 2;                     // [row][2]
+  constexpr int kMaxVec = kSmallMaxD / 128;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int D = g.K, d4 = D / 4, xrow = D + 8, nv = D / 128;
+  const float4* st = reinterpret_cast<const float4*>(smem + small_ln_stage_offset(g.rows, D));
+  const float4* p0 = st + (size_t)g.rows * d4;
+  const float4* p1 = p0 + d4;
   __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(smem);
-  const float4* st = reinterpret_cast<const float4*>(smem + small_ln_stage_offset(g.rows, D)) + tid;
-  const float4 zero = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  float4 a = zero, b = zero;
-  if (has) {
-    a = st[(size_t)g.rows * d4];
-    b = st[(size_t)(g.rows + 1) * d4];
-  }
-  if (g.ln_mode == 0) {
-    a.x += 1.0f; a.y += 1.0f; a.z += 1.0f; a.w += 1.0f;
-  }
-  for (int r0 = 0; r0 < g.rows; r0 += G) {
-    const int nr = min(G, g.rows - r0);
-    float4 v[G];
+  const float inv_d = 1.0f / (float)D;
+  const float add = g.ln_mode == 0 ? 1.0f : 0.0f;
+  for (int r = warp; r < g.rows; r += kSmallWarps) {
+    // three passes over the staged row (shared memory): sum, squared
+    // deviations, normalised output
+    const float4* row = st + (size_t)r * d4 + lane;
+    float sum = 0.0f;
 #pragma unroll
-    for (int i = 0; i < G; ++i) v[i] = (has && i < nr) ? st[(size_t)(r0 + i) * d4] : zero;
-    float sm[G], sq[G];
-#pragma unroll
-    for (int i = 0; i < G; ++i) {
-      sm[i] = (v[i].x + v[i].y) + (v[i].z + v[i].w);
-      sq[i] = fmaf(v[i].x, v[i].x, fmaf(v[i].y, v[i].y, fmaf(v[i].z, v[i].z, v[i].w * v[i].w)));
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-      for (int i = 0; i < G; ++i) {
-        sm[i] += __shfl_xor_sync(0xffffffffu, sm[i], o);
-        sq[i] += __shfl_xor_sync(0xffffffffu, sq[i], o);
+    for (int j = 0; j < kMaxVec; ++j)
+      if (j < nv) {
+        const float4 x = row[32 * j];
+        sum += (x.x + x.y) + (x.z + x.w);
       }
-    if (lane == 0)
 #pragma unroll
-      for (int i = 0; i < G; ++i) {
-        part[(warp * G + i) * 2] = sm[i];
-        part[(warp * G + i) * 2 + 1] = sq[i];
-      }
-    csync();
-    if (tid < nr) {
-      float S = 0.0f, Q = 0.0f;
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    const float mean = sum * inv_d;
+    float q = 0.0f;
 #pragma unroll
-      for (int w = 0; w < kSmallWarps; ++w) {
-        S += part[(w * G + tid) * 2];
-        Q += part[(w * G + tid) * 2 + 1];
+    for (int j = 0; j < kMaxVec; ++j)
+      if (j < nv) {
+        const float4 x = row[32 * j];
+        const float a = x.x - mean, b = x.y - mean, c = x.z - mean, d = x.w - mean;
+        q += (a * a + b * b) + (c * c + d * d);
       }
-      const float mean = S / (float)D;
-      stat[tid * 2] = mean;
-      stat[tid * 2 + 1] = rsqrtf(fmaxf(Q / (float)D - mean * mean, 0.0f) + P.eps);
-    }
-    csync();
-    if (has) {
 #pragma unroll
-      for (int i = 0; i < G; ++i) {
-        if (i < nr) {
-          const float mean = stat[i * 2], rstd = stat[i * 2 + 1];
-          uint2 w;
-          w.x = pack_bf16x2((v[i].x - mean) * rstd * a.x + b.x, (v[i].y - mean) * rstd * a.y + b.y);
-          w.y = pack_bf16x2((v[i].z - mean) * rstd * a.z + b.z, (v[i].w - mean) * rstd * a.w + b.w);
-          *reinterpret_cast<uint2*>(xs + (size_t)(r0 + i) * xrow + 4 * tid) = w;
-        }
+    for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+    const float rstd = rsqrtf(q * inv_d + P.eps);
+#pragma unroll
+    for (int j = 0; j < kMaxVec; ++j)
+      if (j < nv) {
+        const int c4 = lane + 32 * j;
+        const float4 x = row[32 * j];
+        const float4 a = p0[c4], b = p1[c4];
+        uint2 w;
+        w.x = pack_bf16x2((x.x - mean) * rstd * (a.x + add) + b.x, (x.y - mean) * rstd * (a.y + add) + b.y);
+        w.y = pack_bf16x2((x.z - mean) * rstd * (a.z + add) + b.z, (x.w - mean) * rstd * (a.w + add) + b.w);
+        *reinterpret_cast<uint2*>(xs + (size_t)r * xrow + 4 * c4) = w;
       }
-    }
-    csync();   // part / stat are reused by the next round
   }
 }
 
@@ -766,9 +746,8 @@ __device__ __forceinline__ void small_epilogue(const SmallGemm& g, int n, int to
 // Operands of the MMA loop of one GEMM phase on one compute warp.
 struct SmallMmaIn {
   const __nv_bfloat16* xa0;     // token tile 0: this lane's ldmatrix row of the X rows
-  const __nv_bfloat16* xb_lo;   // token tile 1: this lane's fragment rows 16 + gr and 24 + gr
-  const __nv_bfloat16* xb_hi;
-  bool lo1, hi1, two;           // those rows exist; the phase has a second token tile
+  const __nv_bfloat16* xa1;     // token tile 1 (rows past the last token repeat it)
+  bool two;                     // the phase has a second token tile
   int wrow;                     // this lane's ldmatrix offset in a weight slot
   int ks0, ks1;                 // this warp's k-steps (16 wide) of every chunk
   int kc, nch;                  // chunk width (K columns) and chunk count
@@ -808,20 +787,39 @@ __device__ __forceinline__ void small_mma_units(const SmallMmaIn& in, uint8_t* s
     }
     if (!ok) continue;
     const int kx = c * in.kc;
+    // two k-steps at a time: the weight fragments of both in one ldmatrix.x4
+    // (shared-memory instructions, not the MMAs, are what this loop waits on)
 #pragma unroll
-    for (int i = 0; i < kSmallMaxKs; ++i) {
+    for (int i = 0; i < kSmallMaxKs; i += 2) {
       const int s = in.ks0 + i;
-      if (s < in.ks1) {
-        const int k = s * 16;
-        uint32_t a[4], a1[4] = {0u, 0u, 0u, 0u};
-        ldmatrix_x4(a[0], a[1], a[2], a[3], in.xa0 + kx + k);
-        if (in.two) {
-          const int kk = kx + k;
-          a1[0] = in.lo1 ? *reinterpret_cast<const uint32_t*>(in.xb_lo + kk) : 0u;
-          a1[1] = in.hi1 ? *reinterpret_cast<const uint32_t*>(in.xb_hi + kk) : 0u;
-          a1[2] = in.lo1 ? *reinterpret_cast<const uint32_t*>(in.xb_lo + kk + 8) : 0u;
-          a1[3] = in.hi1 ? *reinterpret_cast<const uint32_t*>(in.xb_hi + kk + 8) : 0u;
+      const int k = s * 16;
+      if (s + 1 < in.ks1) {
+        uint32_t b[NU][4];
+        {
+          uint32_t a[4], e[4];   // token tile 0
+          ldmatrix_x4(a[0], a[1], a[2], a[3], in.xa0 + kx + k);
+          ldmatrix_x4(e[0], e[1], e[2], e[3], in.xa0 + kx + k + 16);
+#pragma unroll
+          for (int j = 0; j < NU; ++j) {
+            ldmatrix_x4(b[j][0], b[j][1], b[j][2], b[j][3], wsj[j] + k);
+            mma_bf16_16816(a_s[j][i % NS][0], a[0], a[1], a[2], a[3], b[j][0], b[j][1]);
+            mma_bf16_16816(a_s[j][(i + 1) % NS][0], e[0], e[1], e[2], e[3], b[j][2], b[j][3]);
+          }
         }
+        if (in.two) {
+          uint32_t a[4], e[4];   // token tile 1
+          ldmatrix_x4(a[0], a[1], a[2], a[3], in.xa1 + kx + k);
+          ldmatrix_x4(e[0], e[1], e[2], e[3], in.xa1 + kx + k + 16);
+#pragma unroll
+          for (int j = 0; j < NU; ++j) {
+            mma_bf16_16816(a_s[j][i % NS][1], a[0], a[1], a[2], a[3], b[j][0], b[j][1]);
+            mma_bf16_16816(a_s[j][(i + 1) % NS][1], e[0], e[1], e[2], e[3], b[j][2], b[j][3]);
+          }
+        }
+      } else if (s < in.ks1) {   // an odd last k-step (narrow K)
+        uint32_t a[4], a1[4];
+        ldmatrix_x4(a[0], a[1], a[2], a[3], in.xa0 + kx + k);
+        if (in.two) ldmatrix_x4(a1[0], a1[1], a1[2], a1[3], in.xa1 + kx + k);
 #pragma unroll
         for (int j = 0; j < NU; ++j) {
           uint32_t b0, b1;
@@ -892,19 +890,19 @@ __device__ __forceinline__ bool small_gemm_phase(const SmallGemm& g, const AttnA
   // their products land in accumulator rows that are never stored)
   const int ar0 = min(lane & 15, g.rows - 1);
   const __nv_bfloat16* xa0 = xs + (size_t)ar0 * xrow + (lane >> 4) * 8;
-  // tile 1 (tokens 16-31) usually holds one real token: each lane reads only
-  // the 32-bit words of its fragment rows that exist (16 + gr, 24 + gr)
-  const bool lo1 = 16 + gr < g.rows, hi1 = 24 + gr < g.rows;
-  const __nv_bfloat16* xb_lo = xs + (size_t)(lo1 ? 16 + gr : 0) * xrow + 2 * tig;
-  const __nv_bfloat16* xb_hi = xs + (size_t)(hi1 ? 24 + gr : 0) * xrow + 2 * tig;
-  // weight fragments: ldmatrix.x2 over k, k + 8 (rows lane & 7, k half (lane >> 3) & 1)
+  // tile 1 (tokens 16-31) usually holds one real token; its rows past the
+  // last token repeat it as well
+  const int ar1 = min(16 + (lane & 15), g.rows - 1);
+  const __nv_bfloat16* xa1 = xs + (size_t)ar1 * xrow + (lane >> 4) * 8;
+  // weight fragments: ldmatrix.x4 over k, k + 8, k + 16, k + 24 (two k-steps;
+  // lanes 0-15 also address the x2 form of one k-step)
   const int wrow = (lane & 7) * kSlotRow + (lane >> 3) * 8;
   const uint32_t base = item;
   float acc[kSmallMaxUnits][2][4];
-  SmallMmaIn in{xa0, xb_lo, xb_hi, lo1, hi1, two, wrow, ks0, ks1, kc, nch, base};
+  SmallMmaIn in{xa0, xa1, two, wrow, ks0, ks1, kc, nch, base};
   switch (nu) {
-    case 1: small_mma_units<1, 4>(in, smem, R, P, ok, acc); break;
-    case 2: small_mma_units<2, 4>(in, smem, R, P, ok, acc); break;
+    case 1: small_mma_units<1, 2>(in, smem, R, P, ok, acc); break;
+    case 2: small_mma_units<2, 2>(in, smem, R, P, ok, acc); break;
     case 3: small_mma_units<3, 2>(in, smem, R, P, ok, acc); break;
     default: small_mma_units<4, 2>(in, smem, R, P, ok, acc); break;
   }
@@ -945,6 +943,7 @@ __device__ __forceinline__ bool small_gemm_phase(const SmallGemm& g, const AttnA
     const int n = small_unit(threadIdx.x / kSmallUF) * kSmallUF + threadIdx.x % kSmallUF;
     reinterpret_cast<float*>(g.out)[n] = g.state_row[n];
   }
+
   // One barrier ends the phase: every thread's epilogue stores precede the
   // arrival (thread 0 releases right after it), the X area and the slot of
   // this phase's descriptor may be rewritten after it (every thread waited
