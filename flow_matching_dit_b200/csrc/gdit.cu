@@ -412,6 +412,7 @@ struct gdit_handle {
   int *perm, *seg, *vofs, *kspan, *counters;
   int* phase_counters;      // per-phase arrival counters of the single-sample loop
   SmallPhase* phase_table;  // per-phase descriptors of the single-sample loop
+  float2* ln_part;          // LayerNorm statistics pieces of the single-sample loop
   uint8_t* bad;
   unsigned* status;
   IoPtrs* io;
@@ -796,6 +797,7 @@ void alloc_workspace(gdit_handle* h) {
   h->counters = h->dalloc<int>((size_t)kCounters);
   h->phase_counters = h->dalloc<int>((size_t)kSmallMaxPhases);
   h->phase_table = h->dalloc<SmallPhase>((size_t)kSmallMaxPhases);
+  h->ln_part = h->dalloc<float2>((size_t)kSmallMaxTok * kLnPieces);
   CUDA_TRY(cudaMemset(h->counters, 0, sizeof(int) * kCounters));
   CUDA_TRY(cudaMemset(h->status, 0, sizeof(unsigned)));
   CUDA_TRY(cudaMemset(h->h, 0, sizeof(float) * (size_t)Bm * N * D));
@@ -947,8 +949,8 @@ bool small_loop_fits(const gdit_config& c, int N, int num_sms) {
       (1LL << 31))
     return false;
   if ((long long)N * (D + 8) * 2 > kSmLnScratch) return false;   // LN output rows below the LN scratch
-  // LN: the staged f32 rows and the two modulation vectors, after the output rows
-  if ((long long)small_ln_stage_offset(N, (int)D) + (long long)(N + 2) * D * 4 > kSmLnScratch) return false;
+  // LN: the staged f32 rows and their statistics pieces, after the output rows
+  if ((long long)small_ln_piece_offset(N, (int)D) + (long long)N * kLnPieces * 8 > kSmLnScratch) return false;
   for (long long K : {A, D, F}) {
     if (K % 16 != 0 || (K > kSmallKC && K % kSmallKC != 0)) return false;
     if ((long long)N * (K + 8) * 2 > kSmXBytes) return false;
@@ -1119,6 +1121,7 @@ std::unique_ptr<Profile> build_profile(gdit_handle* h, int B, int S, int K, int 
                              kSmallAttnKB);
     sp.counters = h->phase_counters;
     sp.phases = h->phase_table;
+    sp.ln_part = h->ln_part;
     sp.err = h->status;
     p->small_phases = small_phases_per_step(L) * K;
     if (p->small_phases > kSmallMaxPhases) throw GditError(GDIT_EINVAL, "too many phases for the single-sample loop");

@@ -56,8 +56,11 @@ constexpr int kSlotBytes = kSmallUF * kSlotRow * 2;
 
 // dynamic shared memory (bytes)
 constexpr int kSmXBytes = 140800;                        // X rows / LN / attention / QKV rows / reduction
-constexpr int kSmLnScratchBytes = 4096;                  // LN row sums across warps, at the end of the X area
+constexpr int kSmLnScratchBytes = 4096;                  // LN (mean, rstd) of each row, at the end of the X area
 constexpr int kSmLnScratch = kSmXBytes - kSmLnScratchBytes;
+constexpr int kLnPieces = kSmallMaxD / 8;                // LayerNorm statistics pieces of a row: one per 8 columns
+static_assert(kSmallMaxTok * 8 <= kSmLnScratchBytes, "(mean, rstd) of every row fits the LN scratch");
+static_assert(kSmallMaxD / 4 <= kSmallCompute, "one float4 column group per compute thread");
 constexpr int kSmRing = kSmXBytes;                       // weight slots
 constexpr int kSmHold = kSmRing + kSmallSlots * kSlotBytes;                       // [unit][tok][8] f32 old values
 constexpr int kSmBias = kSmHold + kSmallMaxUnits * kSmallMaxTok * kSmallUF * 4;  // [unit][8] f32
@@ -123,6 +126,10 @@ struct SmallPlan {
   SmallLayer layers[kSmallMaxLayers];
   int* counters;             // one arrival counter per phase, zero at launch
   struct SmallPhase* phases; // descriptor of every phase, written by small_describe_kernel
+  // LayerNorm statistics of the residual rows h, in pieces: the phase that
+  // writes h stores, for every row and every 8 columns of it, their (mean,
+  // M2) ([kSmallMaxTok][kLnPieces]); a LayerNorm phase combines them
+  float2* ln_part;
   unsigned* err;
 };
 
@@ -296,6 +303,7 @@ struct SmallCtx {
   int nh;
   long long max_tok;
   const CUtensorMap* kv_map;
+  float2* ln_part;
 };
 
 // Thread 0 waits (acquire) until `target` CTAs have arrived on `phase`; the
@@ -471,16 +479,20 @@ __device__ __forceinline__ void small_issue_side(const SmallGemm& g, int nu, uin
 }
 
 // Shared-memory offset of the f32 rows staged for LayerNorm (after the bf16
-// output rows); the two modulation vectors follow them.
+// output rows).
 __device__ __host__ __forceinline__ int small_ln_stage_offset(int rows, int D) {
   return (rows * (D + 8) * 2 + 127) & ~127;
 }
+// ... and of the rows' statistics pieces, after the staged rows
+__device__ __host__ __forceinline__ int small_ln_piece_offset(int rows, int D) {
+  return small_ln_stage_offset(rows, D) + rows * D * 4;
+}
 
-// Warp 0: the f32 residual rows that the phase normalises and its two
-// modulation vectors, by bulk copies into shared memory on `xbar`.  The
-// copy engine keeps the whole 70 KB in flight at once; loads through the
-// threads' registers are limited by the SM's outstanding-miss capacity and
-// took several L2 round trips.
+// Warp 0: the f32 residual rows that the phase normalises and their
+// statistics pieces, by bulk copies into shared memory on `xbar`.  The copy
+// engine keeps the whole 90 KB in flight at once; loads through the threads'
+// registers are limited by the SM's outstanding-miss capacity and took
+// several L2 round trips.
 __device__ __forceinline__ void small_issue_ln(const SmallGemm& g, const SmallCtx& P, uint8_t* smem,
                                                uint64_t* xbar) {
   const int lane = threadIdx.x & 31;
@@ -490,72 +502,108 @@ __device__ __forceinline__ void small_issue_ln(const SmallGemm& g, const SmallCt
   if (lane == 0) {
     fence_proxy_async_global();
     fence_proxy_async_smem();
-    mbar_arrive_expect_tx(xbar, (uint32_t)(g.rows + 2) * row_bytes);
+    const uint32_t piece_bytes = (uint32_t)(g.rows * kLnPieces * 8);
+    mbar_arrive_expect_tx(xbar, (uint32_t)g.rows * row_bytes + piece_bytes);
+    bulk_g2s(smem + small_ln_piece_offset(g.rows, D), P.ln_part + (size_t)g.h_row_off * kLnPieces, piece_bytes,
+             xbar);
   }
   __syncwarp();
   uint8_t* st = smem + small_ln_stage_offset(g.rows, D);
   const float* h0 = P.h + (size_t)g.h_row_off * D;
-  for (int r = lane; r < g.rows + 2; r += 32) {
-    const float* src = r < g.rows ? h0 + (size_t)r * D : (r == g.rows ? g.p0 : g.p1);
-    bulk_g2s(st + (size_t)r * row_bytes, src, row_bytes, xbar);
+  for (int r = lane; r < g.rows; r += 32)
+    bulk_g2s(st + (size_t)r * row_bytes, h0 + (size_t)r * D, row_bytes, xbar);
+}
+
+// Mean and 1/std of the rows a LayerNorm phase normalises, from the pieces
+// staged with them: piece i of a row is the mean m_i and the sum of squared
+// deviations M2_i of its columns 8i .. 8i + 7, so the row's mean is the mean
+// of the m_i and its M2 is sum(M2_i + 8 (m_i - mean)^2) (the pairwise update
+// of Chan, Golub and LeVeque, applied to all pieces at once).  A warp per row
+// (rows warp, warp + 8, ...), a lane per piece (and pieces 32, 64, 96 after
+// it); the reductions of a warp's rows are interleaved, one shuffle level
+// for all of them at a time, so their latencies overlap.
+constexpr int kLnRowsPerWarp = kSmallMaxTok / kSmallWarps;
+constexpr int kLnPiecesPerLane = kLnPieces / 32;
+__device__ __forceinline__ void small_ln_stats(const SmallGemm& g, const SmallCtx& P, const uint8_t* smem,
+                                               float2* stat) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int D = g.K, U = D / kSmallUF;
+  const float2* pcs = reinterpret_cast<const float2*>(smem + small_ln_piece_offset(g.rows, D));
+  float2 pc[kLnRowsPerWarp][kLnPiecesPerLane];
+  float s[kLnRowsPerWarp], q[kLnRowsPerWarp], mean[kLnRowsPerWarp];
+#pragma unroll
+  for (int t = 0; t < kLnRowsPerWarp; ++t) {
+    const int r = warp + t * kSmallWarps;
+    s[t] = 0.0f;
+#pragma unroll
+    for (int k = 0; k < kLnPiecesPerLane; ++k) {
+      const int i = lane + 32 * k;
+      pc[t][k] = (r < g.rows && i < U) ? pcs[r * kLnPieces + i] : make_float2(0.0f, 0.0f);
+      s[t] += pc[t][k].x;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+    for (int t = 0; t < kLnRowsPerWarp; ++t) s[t] += __shfl_xor_sync(0xffffffffu, s[t], o);
+#pragma unroll
+  for (int t = 0; t < kLnRowsPerWarp; ++t) {
+    mean[t] = s[t] / (float)U;
+    q[t] = 0.0f;
+#pragma unroll
+    for (int k = 0; k < kLnPiecesPerLane; ++k) {
+      const float w = lane + 32 * k < U ? (float)kSmallUF : 0.0f;
+      const float d = pc[t][k].x - mean[t];
+      q[t] += pc[t][k].y + w * d * d;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+    for (int t = 0; t < kLnRowsPerWarp; ++t) q[t] += __shfl_xor_sync(0xffffffffu, q[t], o);
+  if (lane == 0) {
+#pragma unroll
+    for (int t = 0; t < kLnRowsPerWarp; ++t) {
+      const int r = warp + t * kSmallWarps;
+      if (r < g.rows) stat[r] = make_float2(mean[t], rsqrtf(q[t] / (float)D + P.eps));
+    }
   }
 }
 
-// LN(h rows) -> bf16 X rows, from the rows staged by small_issue_ln, one
-// warp per row (rows warp, warp + 8, ...): each lane takes 32 of the row's
-// columns (float4 at column 4 (lane + 32 j)); the row's mean, then the mean of
-// the squared deviations (two passes over the staged row), are warp shuffle
-// reductions; the lane writes its columns of the normalised row with the
-// AdaLN ((1 + p0), p1) or affine (p0, p1) modulation.  A warp owns whole rows,
-// so no statistics cross warps: 10 shuffles per row instead of a CTA-wide
-// reduction of every row (the shuffles' latency bounded the LN here).
-__device__ __forceinline__ void small_ln_rows(const SmallGemm& g, const SmallCtx& P, uint8_t* smem) {
-  constexpr int kMaxVec = kSmallMaxD / 128;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int D = g.K, d4 = D / 4, xrow = D + 8, nv = D / 128;
-  const float4* st = reinterpret_cast<const float4*>(smem + small_ln_stage_offset(g.rows, D));
-  const float4* p0 = st + (size_t)g.rows * d4;
-  const float4* p1 = p0 + d4;
-  __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(smem);
-  const float inv_d = 1.0f / (float)D;
-  const float add = g.ln_mode == 0 ? 1.0f : 0.0f;
-  for (int r = warp; r < g.rows; r += kSmallWarps) {
-    // three passes over the staged row (shared memory): sum, squared
-    // deviations, normalised output
-    const float4* row = st + (size_t)r * d4 + lane;
-    float sum = 0.0f;
-#pragma unroll
-    for (int j = 0; j < kMaxVec; ++j)
-      if (j < nv) {
-        const float4 x = row[32 * j];
-        sum += (x.x + x.y) + (x.z + x.w);
-      }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    const float mean = sum * inv_d;
-    float q = 0.0f;
-#pragma unroll
-    for (int j = 0; j < kMaxVec; ++j)
-      if (j < nv) {
-        const float4 x = row[32 * j];
-        const float a = x.x - mean, b = x.y - mean, c = x.z - mean, d = x.w - mean;
-        q += (a * a + b * b) + (c * c + d * d);
-      }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
-    const float rstd = rsqrtf(q * inv_d + P.eps);
-#pragma unroll
-    for (int j = 0; j < kMaxVec; ++j)
-      if (j < nv) {
-        const int c4 = lane + 32 * j;
-        const float4 x = row[32 * j];
-        const float4 a = p0[c4], b = p1[c4];
-        uint2 w;
-        w.x = pack_bf16x2((x.x - mean) * rstd * (a.x + add) + b.x, (x.y - mean) * rstd * (a.y + add) + b.y);
-        w.y = pack_bf16x2((x.z - mean) * rstd * (a.z + add) + b.z, (x.w - mean) * rstd * (a.w + add) + b.w);
-        *reinterpret_cast<uint2*>(xs + (size_t)r * xrow + 4 * c4) = w;
-      }
+// LN(h rows) -> bf16 X rows, from the rows staged by small_issue_ln and the
+// (mean, rstd) of small_ln_stats: thread t owns columns 4t .. 4t + 3 of every
+// row, so its AdaLN ((1 + p0), p1) or affine (p0, p1) modulation is loaded
+// once, from global memory, before the rows land.
+__device__ __forceinline__ void small_ln_apply(const SmallGemm& g, const uint8_t* smem, uint8_t* xout,
+                                               const float2* stat, float4 m0, float4 m1) {
+  const int D = g.K, d4 = D / 4, xrow = D + 8, c4 = threadIdx.x;
+  if (c4 >= d4) return;
+  const float4* st = reinterpret_cast<const float4*>(smem + small_ln_stage_offset(g.rows, D)) + c4;
+  __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(xout) + 4 * c4;
+#pragma unroll 4
+  for (int r = 0; r < g.rows; ++r) {
+    const float4 x = st[(size_t)r * d4];
+    const float2 ms = stat[r];
+    uint2 w;
+    w.x = pack_bf16x2((x.x - ms.x) * ms.y * m0.x + m1.x, (x.y - ms.x) * ms.y * m0.y + m1.y);
+    w.y = pack_bf16x2((x.z - ms.x) * ms.y * m0.z + m1.z, (x.w - ms.x) * ms.y * m0.w + m1.w);
+    *reinterpret_cast<uint2*>(xs + (size_t)r * xrow) = w;
   }
+}
+
+// The statistics piece of 8 columns of one row, from the 8 adjacent lanes
+// that hold them (lanes 8i .. 8i + 7 of a warp): their mean, then the sum of
+// their squared deviations from it.  Every lane of the warp takes part.
+__device__ __forceinline__ float2 small_piece8(float v) {
+  float s = v;
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  const float m = s * 0.125f;
+  const float d = v - m;
+  float q = d * d;
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+  return make_float2(m, q);
 }
 
 // Self-attention of all heads from the phase's own copy of the QKV rows, for
@@ -710,8 +758,9 @@ __device__ __forceinline__ void small_self_attention(const AttnArgs& a, int D, u
     small_self_attention_dh<32>(a, D, smem);
 }
 
-__device__ __forceinline__ void small_epilogue(const SmallGemm& g, int n, int tok, float v, float bias,
-                                               float hold) {
+// Returns the value stored (the f32 one for the residual outputs).
+__device__ __forceinline__ float small_epilogue(const SmallGemm& g, int n, int tok, float v, float bias,
+                                                float hold) {
   if (g.epi == EPI_SWISH_VEC_BF16) {
     v = swish_f(v + bias);
   } else {
@@ -733,14 +782,16 @@ __device__ __forceinline__ void small_epilogue(const SmallGemm& g, int n, int to
       reinterpret_cast<float*>(g.out)[idx] = v;
       break;
     case EPI_RESID_F32:
-      reinterpret_cast<float*>(g.out)[idx] = hold + v;
+      v += hold;
+      reinterpret_cast<float*>(g.out)[idx] = v;
       break;
     default: {   // EPI_EULER
-      const float xn = hold + g.alpha * v;
-      reinterpret_cast<float*>(g.out)[idx] = xn;
-      g.out2[(size_t)tok * g.ldo + n] = __float2bfloat16_rn(xn);
+      v = hold + g.alpha * v;
+      reinterpret_cast<float*>(g.out)[idx] = v;
+      g.out2[(size_t)tok * g.ldo + n] = __float2bfloat16_rn(v);
     }
   }
+  return v;
 }
 
 // Operands of the MMA loop of one GEMM phase on one compute warp.
@@ -868,11 +919,20 @@ __device__ __forceinline__ bool small_gemm_phase(const SmallGemm& g, const AttnA
     ++xuse;
   } else if (g.x_mode == 1) {
     small_issue_ln(g, P, smem, xbar);
+    float4 m0 = make_float4(0.0f, 0.0f, 0.0f, 0.0f), m1 = m0;
+    if ((int)threadIdx.x < g.K / 4) {
+      const float add = g.ln_mode == 0 ? 1.0f : 0.0f;
+      m0 = __ldg(reinterpret_cast<const float4*>(g.p0) + threadIdx.x);
+      m1 = __ldg(reinterpret_cast<const float4*>(g.p1) + threadIdx.x);
+      m0.x += add; m0.y += add; m0.z += add; m0.w += add;
+    }
+    float2* stat = reinterpret_cast<float2*>(smem + kSmLnScratch);
     if (!mbar_wait(xbar, xuse & 1u, P.err)) *fail = 1;
     ++xuse;
-    csync();                       // a failed wait is seen by every thread
+    small_ln_stats(g, P, smem, stat);   // every lane (shuffles); unused after a failed wait
+    csync();                       // a failed wait is seen by every thread; stat complete
     ok = *fail == 0;
-    if (ok) small_ln_rows(g, P, smem);
+    if (ok) small_ln_apply(g, smem, smem, stat, m0, m1);
     csync();
   } else {
     small_issue_qkv(att, g.K, smem, xbar);
@@ -929,21 +989,39 @@ __device__ __forceinline__ bool small_gemm_phase(const SmallGemm& g, const AttnA
   const bool has_bias = (g.epi == EPI_SWISH_VEC_BF16 ? g.vec : g.bias) != nullptr;
   const float* biases = reinterpret_cast<const float*>(smem + kSmBias);
   const float* holds = reinterpret_cast<const float*>(smem + kSmHold);
-  const int per_unit = g.rows * kSmallUF;
-  for (int idx = threadIdx.x; idx < nu * per_unit; idx += kSmallCompute) {
-    const int j = idx / per_unit, rem = idx - j * per_unit;
+  // a phase that writes h also leaves the LayerNorm statistics piece of every
+  // (row, unit) it wrote: the 8 lanes 8i .. 8i + 7 hold one (unit, row), as
+  // the CTA's outputs are walked unit by unit, row by row, column by column
+  const bool pieces = g.epi == EPI_F32 || g.epi == EPI_RESID_F32;
+  const int per_unit = g.rows * kSmallUF, n_out = nu * per_unit;
+  for (int base = 0; base < n_out; base += kSmallCompute) {   // the same trip count in every thread
+    const int idx = base + (int)threadIdx.x;
+    const bool mine = idx < n_out;
+    const int j = mine ? idx / per_unit : 0, rem = idx - j * per_unit;
     const int tok = rem / kSmallUF, fi = rem - tok * kSmallUF;
-    float v = 0.0f;
+    float r = 0.0f;
+    if (mine) {
+      float v = 0.0f;
 #pragma unroll
-    for (int w = 0; w < kSmallWarps; ++w) v += red[((w * kSmallMaxUnits + j) * kSmallMaxTok + tok) * kSmallUF + fi];
-    small_epilogue(g, small_unit(j) * kSmallUF + fi, tok, v, has_bias ? biases[j * kSmallUF + fi] : 0.0f,
-                   holds[(j * kSmallMaxTok + tok) * kSmallUF + fi]);
+      for (int w = 0; w < kSmallWarps; ++w) v += red[((w * kSmallMaxUnits + j) * kSmallMaxTok + tok) * kSmallUF + fi];
+      r = small_epilogue(g, small_unit(j) * kSmallUF + fi, tok, v, has_bias ? biases[j * kSmallUF + fi] : 0.0f,
+                         holds[(j * kSmallMaxTok + tok) * kSmallUF + fi]);
+    }
+    if (pieces) {
+      const float2 pc = small_piece8(r);
+      if (mine && fi == 0 && ok) P.ln_part[(size_t)(g.out_row_off + tok) * kLnPieces + small_unit(j)] = pc;
+    }
   }
-  if (g.state_row != nullptr && threadIdx.x < nu * kSmallUF) {
-    const int n = small_unit(threadIdx.x / kSmallUF) * kSmallUF + threadIdx.x % kSmallUF;
-    reinterpret_cast<float*>(g.out)[n] = g.state_row[n];
+  // the action encoder's output row 0 is the state row, copied (its pieces too)
+  if (g.state_row != nullptr && (int)threadIdx.x < 32 * ((nu * kSmallUF + 31) / 32)) {
+    const int t = threadIdx.x;
+    const bool mine = t < nu * kSmallUF;
+    const int n = small_unit(t / kSmallUF) * kSmallUF + t % kSmallUF;
+    const float v = mine ? g.state_row[n] : 0.0f;
+    if (mine) reinterpret_cast<float*>(g.out)[n] = v;
+    const float2 pc = small_piece8(v);
+    if (mine && t % kSmallUF == 0 && ok) P.ln_part[small_unit(t / kSmallUF)] = pc;
   }
-
   // One barrier ends the phase: every thread's epilogue stores precede the
   // arrival (thread 0 releases right after it), the X area and the slot of
   // this phase's descriptor may be rewritten after it (every thread waited
@@ -1148,7 +1226,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1) small_loop_kernel(const Smal
   __shared__ int s_ok;
   __shared__ int s_fail;
   const SmallCtx P = {plan->err,  plan->counters, plan->h,  plan->eps,     plan->phases,
-                      plan->vofs, plan->dh,       plan->nh, plan->max_tok, &plan->kv_map};
+                      plan->vofs, plan->dh,       plan->nh, plan->max_tok, &plan->kv_map, plan->ln_part};
   const int total = small_phases_per_step(plan->L) * plan->K;
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSmallSlots; ++i) {
