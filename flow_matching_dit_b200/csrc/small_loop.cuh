@@ -1071,22 +1071,29 @@ __device__ __forceinline__ bool small_cross_attention(const SmallPhase& ph, cons
   attn_key_range(a, 0, k_begin, n_keys);
   const int krow = ph.kv_row + head * (int)P.max_tok + k_begin;
   const int vrow = ph.kv_row + (P.nh + head) * (int)P.max_tok + k_begin;
+  const int nblk = (n_keys + kSmallAttnKB - 1) / kSmallAttnKB;
+  // K/V boxes of pass b0 (thread 0), on xbar
+  auto issue_kv = [&](int b0) {
+    if (threadIdx.x != 0) return;
+    const int nb = min(kSmallAttnBlocks, nblk - b0);
+    fence_proxy_async_smem();   // earlier reads of the area precede the copies
+    mbar_arrive_expect_tx(xbar, (uint32_t)(2 * nb * BOX));
+    for (int b = 0; b < nb; ++b) {
+      tma_load_2d(sK + b * BOX, P.kv_map, xbar, 0, krow + (b0 + b) * kSmallAttnKB);
+      tma_load_2d(sV + b * BOX, P.kv_map, xbar, 0, vrow + (b0 + b) * kSmallAttnKB);
+    }
+  };
+  // the first pass's keys are requested before the queries are loaded: the
+  // query loads (an L2 round trip) then overlap the K/V copies
+  if (nblk > 0) issue_kv(0);
   attn_load_q<2, DH>(a, 0, head, sQ, threadIdx.x, kSmallCompute);
   float o[2][DH / 8][4];
   float mrow[2][2], lrow[2][2];
   attn_init<2, DH>(o, mrow, lrow);
-  const int nblk = (n_keys + kSmallAttnKB - 1) / kSmallAttnKB;
   bool ok = true;
   for (int b0 = 0; b0 < nblk; b0 += kSmallAttnBlocks) {
     const int nb = min(kSmallAttnBlocks, nblk - b0);
-    if (threadIdx.x == 0) {
-      fence_proxy_async_smem();   // earlier reads of the area precede the copies
-      mbar_arrive_expect_tx(xbar, (uint32_t)(2 * nb * BOX));
-      for (int b = 0; b < nb; ++b) {
-        tma_load_2d(sK + b * BOX, P.kv_map, xbar, 0, krow + (b0 + b) * kSmallAttnKB);
-        tma_load_2d(sV + b * BOX, P.kv_map, xbar, 0, vrow + (b0 + b) * kSmallAttnKB);
-      }
-    }
+    if (b0 > 0) issue_kv(b0);
     if (!mbar_wait(xbar, xuse & 1u, P.err)) *fail = 1;
     ++xuse;
     // rows past the last key (in the last box) hold other tokens or nothing
