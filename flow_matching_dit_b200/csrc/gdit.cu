@@ -142,6 +142,24 @@ CUtensorMap make_kv_tmap(const void* ptr, long long rows, int head_dim, int box_
   return m;
 }
 
+// Output map of the head-major K/V cache for the TMA-store epilogue: a 3-D
+// bf16 tensor [blocks][rows][64] (one (layer, K|V, head) block of head_dim 64
+// per index of the outer dimension), boxes of 64 columns x 32 rows x 1 block,
+// 128-byte swizzle like the 2-D output boxes.
+CUtensorMap make_kv_out_tmap(const void* ptr, long long blocks, long long rows) {
+  REQUIRE(((uintptr_t)ptr & 15u) == 0, "TMA base pointer not 16-byte aligned");
+  CUtensorMap m;
+  cuuint64_t dims[3] = {64u, (cuuint64_t)std::max<long long>(rows, 1), (cuuint64_t)std::max<long long>(blocks, 1)};
+  cuuint64_t strides[2] = {64u * 2u, (cuuint64_t)rows * 64u * 2u};
+  cuuint32_t box[3] = {64u, 32u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = encode_fn()(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) throw GditError(GDIT_ECUDA, fmt("cuTensorMapEncodeTiled (K/V output) failed (%d)", (int)r));
+  return m;
+}
+
 // Output map for the TMA-store epilogue: [rows, cols] with row pitch `pitch`
 // elements, 32-row boxes of 128 bytes (bf16: 64 columns, f32: 32), 128-byte swizzle.
 CUtensorMap make_out_tmap(const void* ptr, bool f32, long long rows, long long cols, long long pitch) {
@@ -907,6 +925,35 @@ void compute_tables(gdit_handle* h, int K, cudaStream_t s) {
 
 // ------------------------------------------------------------------ planning
 
+// The cross-attention K/V projection on the CTA-pair kernel.  Its output, the
+// head-major cache [layer][K | V][head][token][head_dim], is the 3-D tensor
+// [Lc * 2 * heads][max_tok][head_dim]: with head_dim 64 every 64-column
+// epilogue box is one head block, written by a 3-D TMA store.  Its rows are
+// the packed token range the router wrote, read by the kernel after its
+// dependency wait.  The last row tile also writes rows past that range
+// (projections of stale packed rows): no reader looks past a sample's keys
+// (the attention kernels zero-fill those rows), and a later chunk of the same
+// call rewrites its own rows.
+void enable_pair_kv(GemmOp& op, const gdit_handle* h, const void* A, const void* W) {
+  GemmArgs& a = op.args;
+  if (h->cfg.head_dim != 64 || a.splits != 1 || (op.bn != 256 && op.bn != 128) || a.N % op.bn != 0 ||
+      a.N % 64 != 0 || a.num_groups != 0)
+    return;
+  const long long nt = a.N / op.bn;
+  const long long pair_tiles = ((a.M + kPairBM - 1) / kPairBM) * nt;
+  const long long one_tiles = ((a.M + kBM - 1) / kBM) * nt;
+  const long long pair_sms = std::min<long long>(2 * pair_tiles, h->num_sms - h->num_sms % 2);
+  const long long one_sms = std::min<long long>(one_tiles, h->num_sms);
+  if (10 * pair_sms < 9 * one_sms) return;
+  op.to = make_kv_out_tmap(a.out, a.N / 64, h->max_tok);
+  a.tma_out = 1;
+  a.out3d = 1;
+  op.pair = true;
+  op.ta = make_tmap(A, a.M, a.K, a.K, 128);
+  op.tb = make_tmap(W, a.N, a.K, a.K, op.bn / 2);
+  op.grid = (int)(2 * std::min<long long>(pair_tiles, h->num_sms / 2));
+}
+
 GemmOp plan_gemm(gdit_handle* h, const void* A, long long a_rows, int K, const void* Bw, long long b_rows, int N,
                  int epi, long long rows_est, int groups, int rows_per_sample, int groups_est) {
   GemmOp op;
@@ -992,6 +1039,7 @@ std::unique_ptr<Profile> build_profile(gdit_handle* h, int B, int S, int K, int 
   p->kv.args.head_stride = h->max_tok * h->cfg.head_dim;
   p->kv.rows_kind = 1;
   p->kv.weight_bytes = (long long)h->Lc * 2 * D * Dvl * 2;
+  if ((h->cfg.flags & GDIT_FLAG_NO_PAIR) == 0) enable_pair_kv(p->kv, h, h->xp, m.wkv);
 
   // state encoder (CategorySpecificMLP, ReLU)
   p->st1 = plan_gemm(h, h->sb, B, Sd, m.ws1t, (long long)C * D, D, EPI_RELU_BF16, B, C, 1, gest);

@@ -77,6 +77,7 @@ struct GemmArgs {
   long long head_stride;    //   stored [rows][head_cols] at block + (c / head_cols) * head_stride
 
   int tma_out;              // 1: output through the TMA map (dense, one split, plain [M, N] layout)
+  int out3d;                // with tma_out: the map is 3-D [N / 64][rows][64] (head-major K/V cache; bf16)
   unsigned* err;
 
 };
@@ -371,6 +372,8 @@ __device__ __forceinline__ void gemm_epilogue_tma(const GemmArgs& a, const CUten
     if (lane == 0) {
       if (a.epi == EPI_RESID_F32)
         tma_reduce_add_2d(tmO, box, n, ym);
+      else if (a.out3d)
+        tma_store_3d(tmO, box, 0, ym, n >> 6);   // 64 columns: one head block
       else
         tma_store_2d(tmO, box, n, ym);
       bulk_commit();
@@ -735,17 +738,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t full_l = mapa_shared(&full[0], 0);       // the even CTA's stage barriers
   const uint32_t tempty_l = mapa_shared(&tempty[0], 0);   // the even CTA's accumulator-free barriers
 
-  const int mt = (a.M + kPairBM - 1) / kPairBM;
+  int mt = (a.M + kPairBM - 1) / kPairBM;
   const int nt = (a.N + BN - 1) / BN;
-  const int total = mt * nt;
+  int total = mt * nt;
   const int cid = blockIdx.x >> 1;
   const int ncl = gridDim.x >> 1;
   const int nkb = (a.K + kBK - 1) / kBK;
 
   // The weights depend on no earlier kernel: the first tile's B stages are
-  // requested before the dependency wait.
+  // requested before the dependency wait (with host-side rows only: a
+  // device-side row range is known after it).
   int pre = 0;
-  if (warp == 0 && lane == 0 && cid < total) {
+  if (warp == 0 && lane == 0 && cid < total && a.m_dev == nullptr) {
     int m0, n_idx;
     gemm_pair_decode(cid, mt, nt, m0, n_idx);
     pre = min(nkb, STAGES);
@@ -758,6 +762,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   pdl_wait();
   pdl_launch_dependents();
   __syncthreads();
+  // rows [mb, me): all M, or the device-side range an earlier kernel wrote
+  int mb = 0;
+  if (a.m_dev != nullptr) {
+    const int me = min(__ldcg(a.m_dev), a.M);
+    mb = a.m_begin_dev != nullptr ? max(__ldcg(a.m_begin_dev), 0) : 0;
+    mt = me > mb ? (me - mb + kPairBM - 1) / kPairBM : 0;
+    total = mt * nt;
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
@@ -769,6 +781,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int t = cid; t < total && ok; t += ncl) {
         int m0, n_idx;
         gemm_pair_decode(t, mt, nt, m0, n_idx);
+        m0 += mb;
         const int arow = m0 + (int)rank * 128;
         const int brow = n_idx * BN + (int)rank * (BN / 2);
         for (int kb = 0; kb < nkb; ++kb) {
@@ -832,6 +845,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int t = cid; t < total; t += ncl, ++it) {
       int m0, n_idx;
       gemm_pair_decode(t, mt, nt, m0, n_idx);
+      m0 += mb;
       const int buf = it & 1;
       const uint32_t aphase = (it >> 1) & 1;
       int ready = 0;

@@ -344,6 +344,22 @@ def test_tma_store_epilogue_is_bitwise_equal_to_thread_stores(full_weights):
     np.testing.assert_array_equal(x, y)
 
 
+def test_host_entry_point_matches_device_entry_point_at_full_size(head_full):
+    """The host-buffer entry point packs and projects the features in four
+    sample chunks (the K/V projection of each chunk starts at a device-side
+    row); the device entry point projects all packed rows at once.  With
+    ragged key counts the chunk boundaries fall inside row tiles.  Every
+    output element is accumulated in the same order either way: equal bit
+    for bit."""
+    w = synth.WORKLOADS["batched"]
+    inp = synth.make_inputs(w, seed=53)
+    dev, st = run_gpu(head_full, inp, w.num_steps)
+    assert st == 0
+    host = head_full.get_action_host(inp["backbone_features"], inp["vl_mask"], inp["state"],
+                                     inp["embodiment_id"], inp["init_noise"], w.num_steps)
+    np.testing.assert_array_equal(dev, host)
+
+
 def test_pair_gemms_match_single_cta_gemms(head_full, full_weights):
     """At B = 256 the DiT GEMMs run on CTA pairs (cta_group::2, 256-row tiles);
     with GDIT_FLAG_NO_PAIR they run on single CTAs.  Both sum the same bf16
