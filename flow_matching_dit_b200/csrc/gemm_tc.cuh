@@ -192,6 +192,59 @@ __device__ __forceinline__ float erf_as(float x) {
 
 // exact (erf) GELU: x * Phi(x)
 __device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.0f + erf_as(x * 0.70710678118654752f)); }
+
+// Packed pairs of f32 (sm_100 f32x2 arithmetic: one instruction for both
+// lanes, each rounded to nearest like its scalar form).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_splat(float c) { return f2_pack(c, c); }
+
+// gelu_erf of two values at once: the same operations in the same order as
+// gelu_erf (so the same results, bit for bit), the multiply-adds and
+// multiplies as f32x2 instructions, about half the instructions per value.
+__device__ __forceinline__ void gelu_erf2(float& x0, float& x1) {
+  const uint64_t x = f2_pack(x0, x1);
+  float u0, u1;
+  f2_unpack(f2_mul(x, f2_splat(0.70710678118654752f)), u0, u1);
+  const uint64_t z = f2_pack(fminf(fabsf(u0), 4.0f), fminf(fabsf(u1), 4.0f));
+  uint64_t p = f2_fma(f2_splat(4.30638e-5f), z, f2_splat(2.765672e-4f));
+  p = f2_fma(p, z, f2_splat(1.520143e-4f));
+  p = f2_fma(p, z, f2_splat(9.2705272e-3f));
+  p = f2_fma(p, z, f2_splat(4.22820123e-2f));
+  p = f2_fma(p, z, f2_splat(7.05230784e-2f));
+  p = f2_fma(p, z, f2_splat(1.0f));
+  p = f2_mul(p, p);
+  p = f2_mul(p, p);
+  p = f2_mul(p, p);
+  p = f2_mul(p, p);
+  float p0, p1;
+  f2_unpack(p, p0, p1);
+  const float e0 = copysignf(1.0f - __fdividef(1.0f, p0), u0);
+  const float e1 = copysignf(1.0f - __fdividef(1.0f, p1), u1);
+  const uint64_t r = f2_mul(f2_mul(f2_splat(0.5f), x), f2_add(f2_splat(1.0f), f2_pack(e0, e1)));
+  f2_unpack(r, x0, x1);
+}
 __device__ __forceinline__ float swish_f(float x) { return x / (1.0f + __expf(-x)); }
 
 // Epilogue of 32 consecutive columns [n, n + 32) of row m (group g).
@@ -334,7 +387,8 @@ __device__ __forceinline__ void gemm_epilogue_tma(const GemmArgs& a, const CUten
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const float4 b = __ldg(bp + j);
-          v[4 * j] += b.x; v[4 * j + 1] += b.y; v[4 * j + 2] += b.z; v[4 * j + 3] += b.w;
+          f2_unpack(f2_add(f2_pack(v[4 * j], v[4 * j + 1]), f2_pack(b.x, b.y)), v[4 * j], v[4 * j + 1]);
+          f2_unpack(f2_add(f2_pack(v[4 * j + 2], v[4 * j + 3]), f2_pack(b.z, b.w)), v[4 * j + 2], v[4 * j + 3]);
         }
       }
 #pragma unroll
@@ -347,12 +401,13 @@ __device__ __forceinline__ void gemm_epilogue_tma(const GemmArgs& a, const CUten
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const float4 b = __ldg(bp + j);
-          v[4 * j] += b.x; v[4 * j + 1] += b.y; v[4 * j + 2] += b.z; v[4 * j + 3] += b.w;
+          f2_unpack(f2_add(f2_pack(v[4 * j], v[4 * j + 1]), f2_pack(b.x, b.y)), v[4 * j], v[4 * j + 1]);
+          f2_unpack(f2_add(f2_pack(v[4 * j + 2], v[4 * j + 3]), f2_pack(b.z, b.w)), v[4 * j + 2], v[4 * j + 3]);
         }
       }
       if (a.epi == EPI_GELU_BF16) {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) v[j] = gelu_erf(v[j]);
+        for (int j = 0; j < 64; j += 2) gelu_erf2(v[j], v[j + 1]);
       } else if (a.epi == EPI_RELU_BF16) {
 #pragma unroll
         for (int j = 0; j < 64; ++j) v[j] = fmaxf(v[j], 0.0f);
