@@ -72,7 +72,8 @@ extern "C" {
 #define GDIT_FLAG_NO_SMALL 4u         /* never use the single-sample persistent loop (batch 1 then runs the
                                          same per-layer kernels as larger batches) */
 #define GDIT_FLAG_NO_TMA_STORE 8u     /* DiT GEMMs store their outputs thread by thread instead of by TMA */
-#define GDIT_FLAG_NO_PAIR 16u         /* DiT GEMMs never run on CTA pairs (cta_group::2, 256-row tiles) */
+#define GDIT_FLAG_NO_PAIR 16u         /* the DiT GEMMs and the cross K/V projection never run on CTA pairs
+                                         (cta_group::2, 256-row tiles) */
 
 /* ------------------------------------------------------------------ config
  * Model geometry and capacity.  Every size is explicit.  Defaults of the
@@ -138,7 +139,16 @@ typedef struct gdit_handle gdit_handle;
  * allocates the workspace for max_batch x max_backbone_seq.  The host weight
  * buffers are read before the call returns and are not retained.
  * On success *out owns all device memory of the model.  On failure *out is
- * NULL and gdit_last_error(NULL) holds the reason (e.g. the missing weight). */
+ * NULL and gdit_last_error(NULL) holds the reason (e.g. the missing weight);
+ * everything allocated before the failure has been freed.
+ * Host-side fault injection (for testing callers' error paths): the
+ * environment variable GDIT_FAULT, read here, is a comma-separated list of
+ * kind:N items.  alloc:N makes the handle's N-th device allocation fail
+ * (GDIT_ENOMEM), upload:N its N-th weight or table upload (GDIT_ECUDA), and
+ * graph:N its N-th CUDA-graph instantiation, at the first call of a profile
+ * or in gdit_prepare (GDIT_ECUDA); N counts from 1.  Only the host-side call
+ * is made to fail: nothing runs on the device for it.  A malformed value
+ * makes gdit_create return GDIT_EINVAL. */
 int gdit_create(const gdit_config* cfg, const gdit_tensor* weights, int n_weights, gdit_handle** out);
 
 /* Frees graphs, weights and workspace.  Waits for the handle's outstanding work.
