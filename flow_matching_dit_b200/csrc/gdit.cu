@@ -332,6 +332,9 @@ void choose_tiling(long long rows_est, int groups_est, int N, int K, int num_sms
     bn = 256;
   else if (rows_est >= 512 && N % 128 == 0)
     bn = 128;
+  else if (N >= 16384 && N % 256 == 0)
+    bn = 256;   // few rows, very wide N (the K/V projection of a few hundred tokens): each column tile
+                // re-reads all the rows of A, so wide tiles read A 4x less often than 64-wide ones
   else
     bn = 64;
   const long long mt = (rows_est + kBM - 1) / kBM + std::max(groups_est - 1, 0);
