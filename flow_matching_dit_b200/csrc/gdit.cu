@@ -449,6 +449,7 @@ struct gdit_handle {
   // sample chunks on copy_stream, each chunk packed and projected to K/V as
   // soon as it has landed
   cudaStream_t copy_stream = nullptr;
+  cudaEvent_t small_ev = nullptr;           // the small inputs have landed
   cudaEvent_t chunk_ev[kHostChunks] = {};
   void* st_feats = nullptr;
   size_t st_feats_bytes = 0;
@@ -1496,6 +1497,7 @@ void free_handle(gdit_handle* h) {
   if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
   for (cudaEvent_t e : h->chunk_ev)
     if (e) cudaEventDestroy(e);
+  if (h->small_ev) cudaEventDestroy(h->small_ev);
   for (void* p : h->allocs) cudaFree(p);
   delete h;
 }
@@ -1633,15 +1635,25 @@ int gdit_get_action_host(gdit_handle* h, const void* backbone_features, int bb_d
     if (h->copy_stream == nullptr) {
       CUDA_TRY(cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking));
       for (cudaEvent_t& e : h->chunk_ev) CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+      CUDA_TRY(cudaEventCreateWithFlags(&h->small_ev, cudaEventDisableTiming));
     }
     compute_tables(h, num_steps, s);
     Profile& p = get_profile(h, batch, seq, num_steps, bb_dtype == GDIT_BF16, !h->strict);
     const size_t ha = (size_t)batch * h->H * h->A;
-    // the small inputs first: routing needs the masks and ids
-    CUDA_TRY(cudaMemcpyAsync(h->st_mask, vl_mask, (size_t)batch * seq, cudaMemcpyHostToDevice, s));
-    CUDA_TRY(cudaMemcpyAsync(h->st_ids, embodiment_id, (size_t)batch * 4, cudaMemcpyHostToDevice, s));
-    CUDA_TRY(cudaMemcpyAsync(h->st_state, state, (size_t)batch * h->Sd * 4, cudaMemcpyHostToDevice, s));
-    CUDA_TRY(cudaMemcpyAsync(h->st_noise, init_noise, ha * 4, cudaMemcpyHostToDevice, s));
+    // The small inputs first, on the copy stream ahead of the features:
+    // routing needs the masks and ids.  Host-to-device copies of both streams
+    // go through the same copy engine, so a small copy queued on the compute
+    // stream could land only after every feature chunk, holding the routing
+    // (and so every chunk's projection) until the whole upload had finished.
+    // Every earlier use of the staging buffers ended with the previous call's
+    // synchronize.
+    CUDA_TRY(cudaMemcpyAsync(h->st_mask, vl_mask, (size_t)batch * seq, cudaMemcpyHostToDevice, h->copy_stream));
+    CUDA_TRY(cudaMemcpyAsync(h->st_ids, embodiment_id, (size_t)batch * 4, cudaMemcpyHostToDevice, h->copy_stream));
+    CUDA_TRY(cudaMemcpyAsync(h->st_state, state, (size_t)batch * h->Sd * 4, cudaMemcpyHostToDevice,
+                             h->copy_stream));
+    CUDA_TRY(cudaMemcpyAsync(h->st_noise, init_noise, ha * 4, cudaMemcpyHostToDevice, h->copy_stream));
+    CUDA_TRY(cudaEventRecord(h->small_ev, h->copy_stream));
+    CUDA_TRY(cudaStreamWaitEvent(s, h->small_ev, 0));
     IoPtrs io{h->st_feats, h->st_mask, h->st_state, h->st_ids, h->st_noise, h->st_out, nullptr};
     set_io_kernel<<<1, 1, 0, s>>>(h->io, io);
     CUDA_TRY(cudaGetLastError());
