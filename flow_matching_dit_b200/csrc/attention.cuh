@@ -23,6 +23,7 @@
 namespace gdit {
 
 constexpr int kAttnThreads = 128;
+constexpr bool kKvEvictFirst = true;   // L2 priority of the streamed cross K/V (see attn_stream_chunks)
 
 struct AttnArgs {
   const __nv_bfloat16* q;
@@ -62,6 +63,13 @@ struct AttnSmem {
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid) {
   const uint32_t n = valid ? 16u : 0u;
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem)), "l"(gmem), "r"(n) : "memory");
+}
+// Same, with an L2 eviction-priority hint (a createpolicy value).
+__device__ __forceinline__ void cp_async16_hint(void* smem, const void* gmem, bool valid, uint64_t policy) {
+  const uint32_t n = valid ? 16u : 0u;
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(smem_u32(smem)), "l"(gmem),
+               "r"(n), "l"(policy)
+               : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
@@ -284,6 +292,11 @@ __device__ __forceinline__ void attn_stream_chunks(const AttnArgs& a, int h, int
   // validity test
   constexpr int RSTEP = 32 / PIECES;
   const int r0 = lane / PIECES, c = (lane % PIECES) * 8;
+  // The cross layers' K/V cache is read once per step and is larger than L2
+  // at large batch: its lines go first, so that the activations the next
+  // GEMMs read (and the outputs they write) stay in L2.  Self-attention
+  // reads activation rows: normal priority.
+  const uint64_t kv_policy = a.kspan != nullptr && kKvEvictFirst ? policy_evict_first() : policy_evict_normal();
   auto issue = [&](int chunk, int slot) {
     __nv_bfloat16* dk = ring + slot * 2 * SM::CHUNK_ELEMS;
     __nv_bfloat16* dv = dk + SM::CHUNK_ELEMS;
@@ -292,8 +305,8 @@ __device__ __forceinline__ void attn_stream_chunks(const AttnArgs& a, int h, int
       const long long step = (long long)RSTEP * a.kv_ld;
 #pragma unroll
       for (int i = 0; i < DH / 16; ++i) {
-        cp_async16(dk + (r0 + i * RSTEP) * ROW + c, kbase + off + i * step, true);
-        cp_async16(dv + (r0 + i * RSTEP) * ROW + c, vbase + off + i * step, true);
+        cp_async16_hint(dk + (r0 + i * RSTEP) * ROW + c, kbase + off + i * step, true, kv_policy);
+        cp_async16_hint(dv + (r0 + i * RSTEP) * ROW + c, vbase + off + i * step, true, kv_policy);
       }
     } else {
 #pragma unroll
@@ -302,8 +315,8 @@ __device__ __forceinline__ void attn_stream_chunks(const AttnArgs& a, int h, int
         const int key = chunk * 16 + r;
         const bool valid = key < n_keys;
         const long long row = (long long)(k_begin + (valid ? key : 0));
-        cp_async16(dk + r * ROW + c, kbase + row * a.kv_ld + c, valid);
-        cp_async16(dv + r * ROW + c, vbase + row * a.kv_ld + c, valid);
+        cp_async16_hint(dk + r * ROW + c, kbase + row * a.kv_ld + c, valid, kv_policy);
+        cp_async16_hint(dv + r * ROW + c, vbase + row * a.kv_ld + c, valid, kv_policy);
       }
     }
   };
