@@ -25,8 +25,13 @@ from ._lib import (GDIT_BF16, GDIT_F32, GDIT_FLAG_NO_GRAPH, GDIT_FLAG_NO_PAIR, G
                    GditError, check, lib)
 from .build import build  # noqa: F401
 
-__all__ = ["ActionHead", "GditError", "lib", "build", "check_io_shapes", "GDIT_BF16", "GDIT_F32",
+__all__ = ["ActionHead", "GditError", "lib", "build", "check_io_shapes", "is_checked", "GDIT_BF16", "GDIT_F32",
            "GDIT_FLAG_NO_GRAPH", "GDIT_FLAG_NO_SMALL", "GDIT_FLAG_STRICT_PROFILES"]
+
+
+def is_checked() -> bool:
+    """Whether the loaded library is the range-checked build (GDIT_CHECKED=1)."""
+    return bool(_lib.gdit_is_checked())
 
 
 def _ptr(t) -> int:
@@ -169,6 +174,19 @@ class ActionHead:
     def sync_status(self) -> int:
         """0, or the (negative) device status code of the last call."""
         return _lib.gdit_sync_status(self.h)
+
+    def check_canaries(self) -> int:
+        """Range-checked build only: the number of guard bytes of this handle's
+        device allocations that were overwritten (0 when nothing wrote past a
+        buffer).  Synchronizes the device."""
+        n = ctypes.c_longlong()
+        check(_lib.gdit_check_canaries(self.h, ctypes.byref(n)), self.h)
+        return n.value
+
+    def debug_poke_guard(self, which: int = 0):
+        """Range-checked build only (test hook): overwrite the first guard byte
+        after allocation `which`, as a one-element overrun would."""
+        check(_lib.gdit_debug_poke_guard(self.h, which), self.h)
 
     def routing(self, batch: int):
         perm = np.zeros(batch, np.int32)

@@ -1,8 +1,10 @@
 """ctypes binding of include/gdit.h: argument marshalling only.
 
 Every function here forwards to the entry point of the same name in
-``libgdit.so``.  There is no fallback: if the library is missing or cannot be
-loaded, ``lib()`` raises.
+``libgdit.so`` (or, with the environment variable ``GDIT_CHECKED=1`` set
+before the first call, in the range-checked build ``libgdit_checked.so``).
+There is no fallback: if the library is missing or cannot be loaded, ``lib()``
+raises.
 """
 
 from __future__ import annotations
@@ -11,7 +13,7 @@ import ctypes
 import os
 import threading
 
-from .build import LIB
+from .build import LIB, LIB_CHECKED
 
 GDIT_OK = 0
 GDIT_EINVAL = -1
@@ -69,17 +71,25 @@ _SIGS = {
     "gdit_gemm_static_scratch": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "gdit_debug_wait_expiry": (_I, [_I, ctypes.c_ulonglong]),
     "gdit_get_action_vl": (_I, [_P, _P, _I, _P, _P, _P, _P, _P, _I, _P, _I, _I, _P]),
+    "gdit_is_checked": (_I, []),
+    "gdit_check_canaries": (_I, [_P, ctypes.POINTER(ctypes.c_longlong)]),
+    "gdit_debug_poke_guard": (_I, [_P, _I]),
 }
 
 _lock = threading.Lock()
 _lib = None
 
 
-def lib(path: str = LIB) -> ctypes.CDLL:
+def default_path() -> str:
+    return LIB_CHECKED if os.environ.get("GDIT_CHECKED") == "1" else LIB
+
+
+def lib(path: str = None) -> ctypes.CDLL:
     """The loaded library (raises if it is missing: build it first)."""
     global _lib
     with _lock:
         if _lib is None:
+            path = path or default_path()
             if not os.path.exists(path):
                 raise RuntimeError(f"{path} not found: run flow_matching_dit_b200.build.build() first")
             L = ctypes.CDLL(path)
@@ -172,3 +182,15 @@ def gdit_gemm_static_scratch(*a):
 
 def gdit_debug_wait_expiry(device, limit_ns):
     return lib().gdit_debug_wait_expiry(device, limit_ns)
+
+
+def gdit_is_checked():
+    return lib().gdit_is_checked()
+
+
+def gdit_check_canaries(h, out):
+    return lib().gdit_check_canaries(h, out)
+
+
+def gdit_debug_poke_guard(h, which):
+    return lib().gdit_debug_poke_guard(h, which)

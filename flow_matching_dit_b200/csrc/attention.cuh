@@ -41,6 +41,8 @@ struct AttnArgs {
   float scale_log2;     // log2(e) / sqrt(head_dim)
   const uint8_t* kflag; // cross: image flag of each packed key (used when ksel >= 0)
   int ksel;             // -1: every key; 0: keys with flag 0 (text); 1: flag 1 (image)
+  long long kv_rows;    // cross: rows of a head's block of the K/V cache (the key spans must lie inside)
+  unsigned* status;     // range-checked builds: where a key span outside the block is recorded
 };
 
 // MT: 16-row query tiles (queries padded to 16 * MT); DH: head dim (32 or 64).
@@ -110,6 +112,13 @@ __device__ __forceinline__ void attn_key_range(const AttnArgs& a, int b, int& k_
   if (a.kspan != nullptr) {
     k_begin = a.kspan[2 * b];
     n_keys = a.kspan[2 * b + 1] - k_begin;
+    if constexpr (GDIT_CHECKED) {   // a span outside the block is not followed: no keys
+      if (!checked_in_range(n_keys, 0, a.kv_rows + 1, a.status) ||
+          !checked_in_range(k_begin, 0, a.kv_rows - n_keys + 1, a.status)) {
+        k_begin = 0;
+        n_keys = 0;
+      }
+    }
   } else {
     k_begin = b * a.n_tok;
     n_keys = a.n_tok;

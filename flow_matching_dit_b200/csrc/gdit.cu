@@ -317,6 +317,10 @@ GemmArgs default_args() {
 }
 
 constexpr long long kWsFloats = 16ll << 20;   // split-K partials (64 MB)
+// guard bands of the range-checked build (a multiple of 256 bytes: the
+// buffers keep cudaMalloc's alignment)
+constexpr size_t kGuardBytes = GDIT_CHECKED ? 4096 : 0;
+constexpr uint8_t kGuardByte = 0xA5;
 constexpr int kHostChunks = 4;                // sample chunks of the host-buffer entry point
 constexpr int kSmallMaxPhases = 64 * (5 * kSmallMaxLayers + 6);
 constexpr int kCounters = 1 << 16;
@@ -469,14 +473,30 @@ struct gdit_handle {
     long long n_alloc = 0, n_graph = 0, n_upload = 0;
   } fault;
 
+  // Range-checked builds put a guard band of kGuardBytes before and after
+  // every allocation, filled with kGuardByte; gdit_check_canaries counts the
+  // guard bytes that changed (a write past either end of a buffer).
+  struct Guarded {
+    uint8_t* base;      // start of the front band
+    size_t bytes;       // the buffer between the bands
+  };
+  std::vector<Guarded> guarded_allocs;
+
   template <typename T>
   T* dalloc(size_t count) {
     if (++fault.n_alloc == fault.alloc)
       throw GditError(GDIT_ENOMEM, fmt("injected fault: device allocation %lld failed", fault.n_alloc));
     void* p = nullptr;
-    CUDA_TRY(cudaMalloc(&p, std::max<size_t>(count * sizeof(T), 256)));
+    const size_t bytes = std::max<size_t>(count * sizeof(T), 256);
+    CUDA_TRY(cudaMalloc(&p, bytes + 2 * kGuardBytes));
     allocs.push_back(p);
-    return static_cast<T*>(p);
+    if (kGuardBytes > 0) {
+      uint8_t* b = static_cast<uint8_t*>(p);
+      CUDA_TRY(cudaMemset(b, kGuardByte, kGuardBytes));
+      CUDA_TRY(cudaMemset(b + kGuardBytes + bytes, kGuardByte, kGuardBytes));
+      guarded_allocs.push_back({b, bytes});
+    }
+    return reinterpret_cast<T*>(static_cast<uint8_t*>(p) + kGuardBytes);
   }
 
   // host -> device copy of weight data (synchronous)
@@ -1216,7 +1236,7 @@ struct Launcher {
 // Valid backbone tokens of samples [b0, b0 + nb) -> packed rows (caller order).
 void launch_pack(gdit_handle* h, cudaStream_t s, int bf16, int S, int b0, int nb) {
   launch_k(s, h->pdl, pack_features_kernel, dim3(nb, (S + 31) / 32), dim3(kPackThreads), 0, (const IoPtrs*)h->io,
-           bf16, S, h->Dvl, b0, (const int*)h->vofs, h->xp, h->kflag);
+           bf16, S, h->Dvl, b0, (const int*)h->vofs, h->xp, h->kflag, (long long)h->max_tok, h->status);
 }
 
 // The vision-language LayerNorm of every packed token (only with its weights).
@@ -1302,7 +1322,7 @@ void enqueue_forward(gdit_handle* h, Profile& p, cudaStream_t s, Recorder* rec, 
   }
   lx.timed("route_pack", 0, 0, nullptr, [&] {
     launch_k(s, pdl, gather_inputs_kernel, dim3(B), dim3(128), 0, (const IoPtrs*)h->io, B, H * A, h->Sd,
-             (const int*)h->perm, h->x, h->xb, h->sb);
+             (const int*)h->perm, h->x, h->xb, h->sb, h->status);
   });
   lx.gemm("gemm_embodiment", p.st1);
   lx.gemm("gemm_embodiment", p.st2);
@@ -1332,7 +1352,7 @@ void enqueue_forward(gdit_handle* h, Profile& p, cudaStream_t s, Recorder* rec, 
     });
     lx.timed("route_pack", 0, 0, nullptr, [&] {
       launch_k(s, pdl, scatter_out_kernel, dim3(B), dim3(128), 0, (const IoPtrs*)h->io, H * A, (const int*)h->perm,
-               (const uint8_t*)h->bad, (const float*)h->x);
+               (const uint8_t*)h->bad, (const float*)h->x, h->status);
     });
     return;
   }
@@ -1350,6 +1370,8 @@ void enqueue_forward(gdit_handle* h, Profile& p, cudaStream_t s, Recorder* rec, 
       ln(ada, ada + D, 0, l == 0 ? h->sfeat : nullptr);
       lx.gemm("gemm_dit", p.q[l]);
       AttnArgs aa;
+      aa.kv_rows = h->max_tok;
+      aa.status = h->status;
       aa.q = h->qkv;
       aa.n_tok = N;
       aa.num_heads = h->cfg.num_heads;
@@ -1390,7 +1412,7 @@ void enqueue_forward(gdit_handle* h, Profile& p, cudaStream_t s, Recorder* rec, 
   }
   lx.timed("route_pack", 0, 0, nullptr, [&] {
     launch_k(s, pdl, scatter_out_kernel, dim3(B), dim3(128), 0, (const IoPtrs*)h->io, H * A, (const int*)h->perm,
-             (const uint8_t*)h->bad, (const float*)h->x);
+             (const uint8_t*)h->bad, (const float*)h->x, h->status);
   });
 }
 
@@ -1724,7 +1746,45 @@ int gdit_sync_status(gdit_handle* h) {
     h->last_error = "embodiment_id out of range (those samples are NaN)";
     return GDIT_EDEVICE;
   }
+  if (st & DEV_ERR_INDEX) {
+    h->last_error = "range-checked build: an index derived from the inputs was out of range (the access was skipped)";
+    return GDIT_EDEVICE;
+  }
   return GDIT_OK;
+}
+
+int gdit_is_checked(void) { return GDIT_CHECKED ? 1 : 0; }
+
+int gdit_check_canaries(gdit_handle* h, long long* corrupted_bytes) {
+  if (!h) return GDIT_EINVAL;
+  return guarded(h, [&] {
+    REQUIRE(corrupted_bytes != nullptr, "NULL corrupted_bytes");
+    REQUIRE(GDIT_CHECKED, "not a range-checked build (libgdit_checked.so has the guard bands)");
+    CUDA_TRY(cudaSetDevice(h->cfg.device));
+    CUDA_TRY(cudaDeviceSynchronize());
+    std::vector<uint8_t> band(kGuardBytes);
+    long long bad = 0;
+    for (const gdit_handle::Guarded& g : h->guarded_allocs) {
+      for (const uint8_t* src : {g.base, g.base + kGuardBytes + g.bytes}) {
+        CUDA_TRY(cudaMemcpy(band.data(), src, kGuardBytes, cudaMemcpyDeviceToHost));
+        for (uint8_t v : band) bad += v != kGuardByte;
+      }
+    }
+    *corrupted_bytes = bad;
+  });
+}
+
+int gdit_debug_poke_guard(gdit_handle* h, int which) {
+  if (!h) return GDIT_EINVAL;
+  return guarded(h, [&] {
+    REQUIRE(GDIT_CHECKED, "not a range-checked build");
+    REQUIRE(which >= 0 && which < (int)h->guarded_allocs.size(), "allocation %d of %d", which,
+            (int)h->guarded_allocs.size());
+    CUDA_TRY(cudaSetDevice(h->cfg.device));
+    const gdit_handle::Guarded& g = h->guarded_allocs[(size_t)which];
+    // the first byte after the buffer: what a one-element overrun would write
+    CUDA_TRY(cudaMemset(g.base + kGuardBytes + g.bytes, (int)(uint8_t)~kGuardByte, 1));
+  });
 }
 
 int gdit_debug_routing(gdit_handle* h, int32_t* perm, int32_t* seg, int32_t* vofs) {

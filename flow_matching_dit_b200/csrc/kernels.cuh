@@ -102,7 +102,7 @@ constexpr int kPackThreads = 256;
 
 __global__ void __launch_bounds__(kPackThreads)
     pack_features_kernel(const IoPtrs* io, int bb_bf16, int S, int Dvl, int b0, const int* vofs, __nv_bfloat16* xp,
-                         uint8_t* kflag) {
+                         uint8_t* kflag, long long xp_rows, unsigned* status) {
   __shared__ int s_red[kPackThreads / 32];
   __shared__ int s_rows[32];
   __shared__ int s_n;
@@ -135,6 +135,7 @@ __global__ void __launch_bounds__(kPackThreads)
   __syncthreads();
   const int n = s_n;
   const long long dst0 = (long long)vofs[b] + s_before;
+  if (!checked_in_range(dst0, 0, xp_rows - n + 1, status)) return;   // rows dst0 .. dst0 + n - 1 inside xp
   // image flag of every packed token (the image/text split of the cross layers)
   if ((int)threadIdx.x < n)
     kflag[dst0 + threadIdx.x] =
@@ -161,11 +162,12 @@ __global__ void __launch_bounds__(kPackThreads)
 
 // x (f32) and its bf16 copy from init_noise, bf16 state rows, all in sorted order.
 __global__ void gather_inputs_kernel(const IoPtrs* io, int B, int HA, int Sd, const int* perm, float* x,
-                                     __nv_bfloat16* xb, __nv_bfloat16* sb) {
+                                     __nv_bfloat16* xb, __nv_bfloat16* sb, unsigned* status) {
   pdl_wait();
   pdl_launch_dependents();
   const int i = blockIdx.x;
   const int b = perm[i];
+  if (!checked_in_range(b, 0, B, status)) return;
   for (int e = threadIdx.x; e < HA; e += blockDim.x) {
     const float v = io->noise[(long long)b * HA + e];
     x[(long long)i * HA + e] = v;
@@ -176,11 +178,13 @@ __global__ void gather_inputs_kernel(const IoPtrs* io, int B, int HA, int Sd, co
 }
 
 // out_actions[perm[i]] = x[i]; NaN for a sample whose embodiment id was invalid.
-__global__ void scatter_out_kernel(const IoPtrs* io, int HA, const int* perm, const uint8_t* bad, const float* x) {
+__global__ void scatter_out_kernel(const IoPtrs* io, int HA, const int* perm, const uint8_t* bad, const float* x,
+                                   unsigned* status) {
   pdl_wait();
   pdl_launch_dependents();
   const int i = blockIdx.x;
   const int b = perm[i];
+  if (!checked_in_range(b, 0, (long long)gridDim.x, status)) return;
   const bool nan_out = bad[b] != 0;
   for (int e = threadIdx.x; e < HA; e += blockDim.x)
     io->out[(long long)b * HA + e] = nan_out ? __int_as_float(0x7fc00000) : x[(long long)i * HA + e];

@@ -8,13 +8,35 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+// Range-checked builds (libgdit_checked.so) define GDIT_CHECKED=1: the
+// kernels then check the indices they derive from the caller's inputs (packed
+// token offsets, key spans, the sample permutation) before following them,
+// and the handle's device allocations carry guard bands.  Regular builds
+// compile the checks away.
+#ifndef GDIT_CHECKED
+#define GDIT_CHECKED 0
+#endif
+
 namespace gdit {
 
 // Device status bits (OR-ed into the handle's status word).
 enum : unsigned {
   DEV_ERR_TIMEOUT = 1u,      // a bounded wait expired
   DEV_ERR_BAD_ID = 2u,       // embodiment id out of range
+  DEV_ERR_INDEX = 4u,        // range-checked build: a derived index was out of range (the access was skipped)
 };
+
+// Range-checked builds: whether lo <= i < hi; if not, DEV_ERR_INDEX is recorded
+// in *status and the caller skips the access.  Always true in regular builds.
+__device__ __forceinline__ bool checked_in_range(long long i, long long lo, long long hi, unsigned* status) {
+  if constexpr (GDIT_CHECKED) {
+    if (i < lo || i >= hi) {
+      if (status != nullptr) atomicOr(status, DEV_ERR_INDEX);
+      return false;
+    }
+  }
+  return true;
+}
 
 // A wait that has not completed after this long is treated as a fault: the
 // waiting thread records DEV_ERR_TIMEOUT and gives up.  The whole call takes

@@ -250,6 +250,7 @@ __device__ __forceinline__ void small_describe(const SmallPlan& P, int c, int k,
         } else {
           a.q = P.qkv; a.q_ld = D; a.k = Ly.kv; a.v = Ly.kv + (size_t)P.nh * P.max_tok * P.dh; a.kv_ld = P.dh;
           a.kv_head_stride = P.max_tok * P.dh; a.kspan = P.kspan;
+          a.kv_rows = P.max_tok; a.status = P.err;
           ph.kv_row = (int)((long long)(l / 2) * 2 * P.nh * P.max_tok);
         }
         break;

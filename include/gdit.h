@@ -247,6 +247,29 @@ int gdit_debug_kv(gdit_handle* h, int layer, float* k_out, float* v_out, int* to
  * Allocates and frees one status word on the device; synchronous. */
 int gdit_debug_wait_expiry(int device, unsigned long long limit_ns);
 
+/* Range-checked build.  libgdit_checked.so is the same library compiled with
+ * GDIT_CHECKED=1 (same entry points, same results):
+ *   - every device allocation of a handle sits between two 4 KiB guard bands
+ *     filled with 0xA5 when allocated;
+ *   - the kernels check the indices they derive from the caller's inputs
+ *     before following them: the packed-token rows each sample writes (inside
+ *     the packed buffer), the key spans of the cross attention (inside a
+ *     head's block of the K/V cache) and the sample permutation (inside the
+ *     batch).  An index out of range is not followed: the access is skipped
+ *     and gdit_sync_status returns GDIT_EDEVICE.
+ * gdit_is_checked returns 1 in that build and 0 in libgdit.so.
+ * gdit_check_canaries synchronizes the device and writes to *corrupted_bytes
+ * the number of guard bytes of h's allocations that no longer hold 0xA5 (0
+ * unless something wrote past the end or before the start of a buffer);
+ * GDIT_EINVAL in a regular build.
+ * gdit_debug_poke_guard (test hook) overwrites the first guard byte after
+ * allocation `which` (0-based, in allocation order) from the host, as a
+ * one-element overrun would; GDIT_EINVAL in a regular build or for a bad
+ * index. */
+int gdit_is_checked(void);
+int gdit_check_canaries(gdit_handle* h, long long* corrupted_bytes);
+int gdit_debug_poke_guard(gdit_handle* h, int which);
+
 /* Per-kernel-class timing of one eager (graph-free) run of gdit_get_action
  * with the given device inputs, each launch bracketed by CUDA events on
  * cuda_stream.  Fills up to max_stats entries; returns the count (>= 0) or an

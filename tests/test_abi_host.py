@@ -39,6 +39,23 @@ def test_library_exports_every_declared_symbol(L):
     assert set(declared_functions()) == set(_lib.exported_names())
 
 
+def test_range_checked_build_exports_the_same_symbols_and_says_so(L):
+    """libgdit_checked.so (GDIT_CHECKED=1: guard bands, index checks) has the
+    same entry points; gdit_is_checked tells the two builds apart.  Neither
+    call touches a GPU."""
+    path = build(checked=True)
+    C = ctypes.CDLL(path)
+    for name in declared_functions():
+        assert hasattr(C, name), name
+    C.gdit_is_checked.restype = ctypes.c_int
+    assert C.gdit_is_checked() == 1
+    L.gdit_is_checked.restype = ctypes.c_int
+    assert L.gdit_is_checked() == 0
+    # a regular-build handle has no guard bands: the canary check refuses a NULL handle either way
+    assert L.gdit_check_canaries(None, None) == _lib.GDIT_EINVAL
+    assert L.gdit_debug_poke_guard(None, 0) == _lib.GDIT_EINVAL
+
+
 def test_strings(L):
     assert L.gdit_version().startswith(b"gdit")
     assert L.gdit_strerror(_lib.GDIT_EINVAL) == b"invalid argument"
