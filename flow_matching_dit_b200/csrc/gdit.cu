@@ -325,11 +325,20 @@ constexpr int kHostChunks = 4;                // sample chunks of the host-buffe
 constexpr int kSmallMaxPhases = 64 * (5 * kSmallMaxLayers + 6);
 constexpr int kCounters = 1 << 16;
 
-// Picks the tile width and split-K factor.  Large row counts use wide tiles;
-// small ones (weight streaming) use narrow tiles and split K so that about
-// one CTA per SM streams a slice of the weights.
+// Picks the tile width and split-K factor.  Large row counts use wide tiles,
+// small ones narrow tiles.  The planned GEMMs never split K: measured on the
+// workloads from B = 1 to 256, a split (partials written, a tile counter, the
+// last CTA of a tile reducing them) cost more than the SMs it filled, and it
+// rules out the TMA-store and CTA-pair epilogues (no split: sweep8 11.4 ->
+// 9.3 ms, sweep32 17.3 -> 11.9, sweep128 27.2 -> 17.4, batched 18.3 -> 12.9,
+// B = 256 unchanged).  The split-K kernel path serves the GEMM entry points
+// that take an explicit split count.
 void choose_tiling(long long rows_est, int groups_est, int N, int K, int num_sms, long long ws_rows, int& bn,
                    int& splits) {
+  (void)groups_est;
+  (void)K;
+  (void)num_sms;
+  (void)ws_rows;
   if (N <= 32)
     bn = 32;
   else if (rows_est >= 2048 && N % 256 == 0)
@@ -341,17 +350,7 @@ void choose_tiling(long long rows_est, int groups_est, int N, int K, int num_sms
                 // re-reads all the rows of A, so wide tiles read A 4x less often than 64-wide ones
   else
     bn = 64;
-  const long long mt = (rows_est + kBM - 1) / kBM + std::max(groups_est - 1, 0);
-  const long long nt = (N + bn - 1) / bn;
-  const long long units = std::max<long long>(mt * nt, 1);
-  const int nkb = (K + kBK - 1) / kBK;
   splits = 1;
-  if (units < num_sms) {
-    long long s = num_sms / units;
-    s = std::min<long long>(s, std::max(nkb / 2, 1));
-    while (s > 1 && s * ws_rows * (long long)N > kWsFloats) --s;
-    splits = (int)std::max<long long>(s, 1);
-  }
 }
 
 // ------------------------------------------------------------------ weights
