@@ -339,15 +339,17 @@ void choose_tiling(long long rows_est, int groups_est, int N, int K, int num_sms
   (void)K;
   (void)num_sms;
   (void)ws_rows;
+  // (measured: 256 from 512 rows; 128 from 256 rows, e.g. long_chunk's 408,
+  // 7 % faster there than 64; 64 below, e.g. 136 rows at B = 8)
   if (N <= 32)
     bn = 32;
-  else if (rows_est >= 2048 && N % 256 == 0)
+  else if (rows_est >= 512 && N % 256 == 0)
     bn = 256;
-  else if (rows_est >= 512 && N % 128 == 0)
-    bn = 128;
   else if (N >= 16384 && N % 256 == 0)
     bn = 256;   // few rows, very wide N (the K/V projection of a few hundred tokens): each column tile
                 // re-reads all the rows of A, so wide tiles read A 4x less often than 64-wide ones
+  else if (rows_est >= 256 && N % 128 == 0)
+    bn = 128;
   else
     bn = 64;
   splits = 1;
