@@ -308,7 +308,8 @@ def run_reference(args, rank):
 # ------------------------------------------------------------------ our arm
 
 # every workload of the task, timed one call after the other (inputs resident in HBM)
-WORKLOAD_TABLE = ("latency", "sweep1", "sweep8", "sweep32", "sweep128", "sweep256", "batched", "long_chunk")
+WORKLOAD_TABLE = ("latency", "sweep1", "sweep2", "sweep4", "sweep8", "sweep32", "sweep128", "sweep256", "batched",
+                  "long_chunk")
 
 
 def time_calls(head, d, K, out, stream, calls: int, warmup: int):

@@ -391,8 +391,11 @@ struct Profile {
   cudaGraphExec_t exec_main = nullptr;   // the call after the K/V projection (host-buffer entry point)
   // single-sample profiles run the K-step loop as one persistent kernel
   bool small = false;
-  SmallPlan* small_plan = nullptr;   // device copy
-  int small_phases = 0;
+  SmallPlan* small_plan = nullptr;   // device copies, one per sample
+  int small_phases = 0;              // per sample
+  int small_groups = 0;              // samples (CTA groups) of the loop
+  int small_gsize = 0;               // CTAs per group
+  bool small_grouped = false;        // several groups, or more than kSmallMaxUnits units of a CTA in some linear
 };
 
 struct KStat {
@@ -840,7 +843,7 @@ void alloc_workspace(gdit_handle* h) {
   h->counters = h->dalloc<int>((size_t)kCounters);
   h->phase_counters = h->dalloc<int>((size_t)kSmallMaxPhases);
   h->phase_table = h->dalloc<SmallPhase>((size_t)kSmallMaxPhases);
-  h->ln_part = h->dalloc<float2>((size_t)kSmallMaxTok * kLnPieces);
+  h->ln_part = h->dalloc<float2>((size_t)kSmallMaxGroups * kSmallMaxTok * kLnPieces);
   CUDA_TRY(cudaMemset(h->counters, 0, sizeof(int) * kCounters));
   CUDA_TRY(cudaMemset(h->status, 0, sizeof(unsigned)));
   CUDA_TRY(cudaMemset(h->h, 0, sizeof(float) * (size_t)Bm * N * D));
@@ -896,13 +899,19 @@ void set_kernel_attrs() {
   set_gemm_pair_attr<256>();
   max_shared_carveout(gemm_tc_pair_kernel<128>);
   max_shared_carveout(gemm_tc_pair_kernel<256>);
-  CUDA_TRY(cudaFuncSetAttribute(small_loop_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  CUDA_TRY(cudaFuncSetAttribute(small_loop_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 SmallSmem<64>::TOTAL));
-  CUDA_TRY(cudaFuncSetAttribute(small_loop_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  CUDA_TRY(cudaFuncSetAttribute(small_loop_kernel<32, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 SmallSmem<32>::TOTAL));
-  max_shared_carveout(small_loop_kernel<64>);
+  CUDA_TRY(cudaFuncSetAttribute(small_loop_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                SmallSmem<64>::TOTAL));
+  CUDA_TRY(cudaFuncSetAttribute(small_loop_kernel<32, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                SmallSmem<32>::TOTAL));
+  max_shared_carveout(small_loop_kernel<64, false>);
+  max_shared_carveout(small_loop_kernel<32, false>);
+  max_shared_carveout(small_loop_kernel<64, true>);
+  max_shared_carveout(small_loop_kernel<32, true>);
   max_shared_carveout(small_describe_kernel);
-  max_shared_carveout(small_loop_kernel<32>);
   set_attn_attrs<2, 64>();
   set_attn_attrs<4, 64>();
   set_attn_attrs<2, 32>();
@@ -1010,12 +1019,14 @@ GemmOp plan_gemm(gdit_handle* h, const void* A, long long a_rows, int K, const v
   return op;
 }
 
-// Whether one sample of N tokens fits the single-sample loop: its shared
-// buffers, its weight chunking (K <= 1024 or a multiple of 1024) and at most
-// kSmallMaxUnits units of 8 features per CTA in every linear.
-bool small_loop_fits(const gdit_config& c, int N, int num_sms) {
+// Whether one sample of N tokens fits the single-sample loop run by `ctas`
+// CTAs: its shared buffers, its weight chunking (K <= 1024 or a multiple of
+// 1024), one CTA per head, and, where a CTA has more than kSmallMaxUnits units
+// of 8 features in a linear (it takes them in passes), room for the
+// reduction area after the normalised / attention rows, which are read again.
+bool small_loop_fits(const gdit_config& c, int N, int ctas) {
   const long long D = c.hidden, F = c.mlp_hidden, A = c.action_dim;
-  if (N > kSmallMaxTok || D > kSmallMaxD || c.num_layers > kSmallMaxLayers || c.num_heads > num_sms) return false;
+  if (N > kSmallMaxTok || D > kSmallMaxD || c.num_layers > kSmallMaxLayers || c.num_heads > ctas) return false;
   // the K/V cache rows (with one box of slack) are addressed by 32-bit TMA coordinates
   if ((long long)(c.num_layers / 2) * 2 * c.num_heads * ((long long)c.max_batch * c.max_backbone_seq + kSmallAttnKB) >=
       (1LL << 31))
@@ -1029,10 +1040,12 @@ bool small_loop_fits(const gdit_config& c, int N, int num_sms) {
   }
   // self layers: the attention output rows and the QKV rows share the X area
   if ((((long long)N * (D + 8) * 2 + 127) & ~127LL) + (long long)N * (3 * D + 8) * 2 > kSmXBytes) return false;
+  bool passes = false;
   for (long long n_out : {A, D, 3 * D, F}) {
     if (n_out % kSmallUF != 0) return false;
-    if ((n_out / kSmallUF + num_sms - 1) / num_sms > kSmallMaxUnits) return false;
+    if ((n_out / kSmallUF + ctas - 1) / ctas > kSmallMaxUnits) passes = true;
   }
+  if (passes && (long long)small_ln_stage_offset(N, (int)D) + kSmRedBytes > kSmLnScratch) return false;
   return true;
 }
 
@@ -1166,8 +1179,11 @@ std::unique_ptr<Profile> build_profile(gdit_handle* h, int B, int S, int K, int 
   for (GemmOp* g : {&p->st1, &p->st2, &p->a1, &p->a2, &p->a3, &p->d1, &p->d2})
     g->weight_bytes = (long long)g->args.N * g->args.K * 2;   // per category used
 
-  // one sample: the K-step loop as one persistent kernel
-  p->small = B == 1 && small_loop_fits(h->cfg, N, h->num_sms) && (h->cfg.flags & GDIT_FLAG_NO_SMALL) == 0;
+  // one sample, or up to kSmallMaxGroups: the K-step loop as one persistent
+  // kernel whose CTAs form one group per sample
+  const int gsize = B >= 1 ? h->num_sms / B : 0;
+  p->small = B >= 1 && B <= kSmallMaxGroups && (h->cfg.flags & GDIT_FLAG_NO_SMALL) == 0 &&
+             (long long)B * small_phases_per_step(L) * K <= kSmallMaxPhases && small_loop_fits(h->cfg, N, gsize);
   if (p->small) {
     const Tables& t = h->tables.at(K);
     SmallPlan sp;
@@ -1192,14 +1208,38 @@ std::unique_ptr<Profile> build_profile(gdit_handle* h, int B, int S, int K, int 
     }
     sp.kv_map = make_kv_tmap(h->kv, (long long)h->Lc * 2 * h->cfg.num_heads * h->max_tok, h->cfg.head_dim,
                              kSmallAttnKB);
-    sp.counters = h->phase_counters;
-    sp.phases = h->phase_table;
-    sp.ln_part = h->ln_part;
     sp.err = h->status;
+    sp.groups = B;
     p->small_phases = small_phases_per_step(L) * K;
-    if (p->small_phases > kSmallMaxPhases) throw GditError(GDIT_EINVAL, "too many phases for the single-sample loop");
-    p->small_plan = h->dalloc<SmallPlan>(1);
-    CUDA_TRY(cudaMemcpy(p->small_plan, &sp, sizeof(sp), cudaMemcpyHostToDevice));
+    p->small_groups = B;
+    p->small_gsize = gsize;
+    p->small_grouped = B > 1;
+    for (long long n_out : {(long long)A, (long long)D, 3LL * D, (long long)F})
+      if ((n_out / kSmallUF + gsize - 1) / gsize > kSmallMaxUnits) p->small_grouped = true;
+    // sample b (embodiment-sorted position) works on its own rows of the
+    // batch buffers and on its own counters, descriptors and statistics
+    std::vector<SmallPlan> plans((size_t)B, sp);
+    for (int b = 0; b < B; ++b) {
+      SmallPlan& q = plans[(size_t)b];
+      q.sample = b;
+      q.h = h->h + (size_t)b * N * D;
+      q.x = h->x + (size_t)b * H * A;
+      q.xb = h->xb + (size_t)b * H * A;
+      q.abf = h->abf + (size_t)b * H * D;
+      q.zbf = h->zbf + (size_t)b * H * D;
+      q.ybf = h->ybf + (size_t)b * H * D;
+      q.rbf = h->rbf + (size_t)b * H * D;
+      q.qkv = h->qkv + (size_t)b * N * 3 * D;
+      q.o = h->o + (size_t)b * N * D;
+      q.f = h->f + (size_t)b * N * F;
+      q.sfeat = h->sfeat + (size_t)b * D;
+      q.kspan = h->kspan + 2 * b;
+      q.counters = h->phase_counters + (size_t)b * p->small_phases;
+      q.phases = h->phase_table + (size_t)b * p->small_phases;
+      q.ln_part = h->ln_part + (size_t)b * kSmallMaxTok * kLnPieces;
+    }
+    p->small_plan = h->dalloc<SmallPlan>((size_t)B);
+    CUDA_TRY(cudaMemcpy(p->small_plan, plans.data(), sizeof(SmallPlan) * (size_t)B, cudaMemcpyHostToDevice));
   }
   return p;
 }
@@ -1330,11 +1370,12 @@ void enqueue_forward(gdit_handle* h, Profile& p, cudaStream_t s, Recorder* rec, 
 
   if (p.small) {
     lx.timed("small_loop", 0, 0, nullptr, [&] {
-      launch_k(s, pdl, small_describe_kernel, dim3((p.small_phases + 127) / 128), dim3(128), 0,
+      const int n_desc = p.small_groups * p.small_phases;
+      launch_k(s, pdl, small_describe_kernel, dim3((n_desc + 127) / 128), dim3(128), 0,
                (const SmallPlan*)p.small_plan);
-      CUDA_TRY(cudaMemsetAsync(h->phase_counters, 0, sizeof(int) * (size_t)p.small_phases, s));
+      CUDA_TRY(cudaMemsetAsync(h->phase_counters, 0, sizeof(int) * (size_t)n_desc, s));
       cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(h->num_sms);
+      cfg.gridDim = dim3((unsigned)(p.small_groups * p.small_gsize));
       cfg.blockDim = dim3(kSmallThreads);
       cfg.stream = s;
       cudaLaunchAttribute attr[1];
@@ -1343,13 +1384,15 @@ void enqueue_forward(gdit_handle* h, Profile& p, cudaStream_t s, Recorder* rec, 
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       const SmallPlan* sp = p.small_plan;
-      if (h->cfg.head_dim == 64) {
-        cfg.dynamicSmemBytes = SmallSmem<64>::TOTAL;
-        CUDA_TRY(cudaLaunchKernelEx(&cfg, small_loop_kernel<64>, sp));
-      } else {
-        cfg.dynamicSmemBytes = SmallSmem<32>::TOTAL;
-        CUDA_TRY(cudaLaunchKernelEx(&cfg, small_loop_kernel<32>, sp));
-      }
+      cfg.dynamicSmemBytes = h->cfg.head_dim == 64 ? SmallSmem<64>::TOTAL : SmallSmem<32>::TOTAL;
+      if (h->cfg.head_dim == 64 && p.small_grouped)
+        CUDA_TRY(cudaLaunchKernelEx(&cfg, small_loop_kernel<64, true>, sp));
+      else if (h->cfg.head_dim == 64)
+        CUDA_TRY(cudaLaunchKernelEx(&cfg, small_loop_kernel<64, false>, sp));
+      else if (p.small_grouped)
+        CUDA_TRY(cudaLaunchKernelEx(&cfg, small_loop_kernel<32, true>, sp));
+      else
+        CUDA_TRY(cudaLaunchKernelEx(&cfg, small_loop_kernel<32, false>, sp));
     });
     lx.timed("route_pack", 0, 0, nullptr, [&] {
       launch_k(s, pdl, scatter_out_kernel, dim3(B), dim3(128), 0, (const IoPtrs*)h->io, H * A, (const int*)h->perm,

@@ -9,8 +9,8 @@
 //
 //   * a phase is a GEMM (out = epilogue(X W^T)) or an attention;
 //   * a GEMM's output features are cut into units of 8 (N / 8 units, unit u on
-//     CTA u mod grid), so a 1024-wide linear keeps 128 CTAs busy and the
-//     4096-wide FF1 all of them;
+//     CTA u mod grid), so at B = 1 a 1024-wide linear keeps 128 CTAs busy and
+//     the 4096-wide FF1 all of them;
 //   * one producer warp per CTA walks the phase table ahead of the compute
 //     warps and streams this CTA's weight chunks (8 rows x up to 1024 columns,
 //     one bulk copy per row into padded rows) into a ring of shared-memory
@@ -26,6 +26,16 @@
 //     the attention kernels, keys split over the 8 warps); self-attention (17
 //     keys) is computed inside the self layer's O phase by every CTA of it,
 //     from its own copy of the QKV rows, so that phase needs no X load.
+//
+// A batch of 2-4 samples runs the same loop with the grid cut into one group
+// of CTAs per sample (148 / B each): each group has its own phase table,
+// counters and rows, and streams all the weights itself (the groups read the
+// same weights, mostly from L2).  A CTA then has up to 4 x B units of 8
+// features in a linear and takes them in passes of up to four.  At B = 2 a
+// call takes 5.3 ms against 8.8 ms for the per-layer kernels; from B = 5 on
+// the per-layer kernels are faster (9.1 against 9.0 ms at B = 5, 12.4 against
+// 9.3 ms at B = 8: a CTA's weight stream, not the shared phase cost, then sets
+// the time).
 //
 // Phases are ordered by arrival counters in global memory: the CTAs that work
 // in phase p wait until every CTA that worked in phase p-1 has arrived (each
@@ -48,7 +58,8 @@ constexpr int kSmallMaxD = 1024;
 constexpr int kSmallMaxLayers = 64;
 constexpr int kSmallKC = 1024;                           // widest weight chunk (K columns)
 constexpr int kSmallUF = 8;                              // output features per unit
-constexpr int kSmallMaxUnits = 4;                        // units of one CTA in one phase
+constexpr int kSmallMaxUnits = 4;                        // units of one CTA in one pass of a phase
+constexpr int kSmallMaxGroups = 4;                       // samples run at once (one CTA group each)
 constexpr int kSmallSlots = 5;                           // weight chunks resident at once
 constexpr int kSmallPairPhases = 9;                      // phases of a (cross, self) layer pair
 constexpr int kSlotRow = kSmallKC + 8;                   // padded slot row (elements): conflict-free ldmatrix
@@ -131,6 +142,8 @@ struct SmallPlan {
   // M2) ([kSmallMaxTok][kLnPieces]); a LayerNorm phase combines them
   float2* ln_part;
   unsigned* err;
+  int groups;                // samples run at once: one plan per sample, plan[0].groups of them
+  int sample;                // this plan's sample (position in the embodiment-sorted batch)
 };
 
 struct SmallGemm {
@@ -305,6 +318,8 @@ struct SmallCtx {
   long long max_tok;
   const CUtensorMap* kv_map;
   float2* ln_part;
+  int rank;                  // this CTA's index in its group (the CTAs that run one sample's loop)
+  int gsize;                 // CTAs in the group
 };
 
 // Thread 0 waits (acquire) until `target` CTAs have arrived on `phase`; the
@@ -345,17 +360,18 @@ __device__ __forceinline__ void small_arrive(const SmallCtx& P, int phase) {
 // ---------------------------------------------------------------- units and chunks
 
 __device__ __forceinline__ int gemm_units(const SmallGemm& g) { return g.N / kSmallUF; }
-__device__ __forceinline__ int workers(int units) { return units < (int)gridDim.x ? units : (int)gridDim.x; }
-__device__ __forceinline__ int small_my_units(const SmallGemm& g) {
+__device__ __forceinline__ int workers(const SmallCtx& P, int units) { return units < P.gsize ? units : P.gsize; }
+__device__ __forceinline__ int small_my_units(const SmallCtx& P, const SmallGemm& g) {
   const int u = gemm_units(g);
-  return (int)blockIdx.x < u ? (u - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+  return P.rank < u ? (u - P.rank + P.gsize - 1) / P.gsize : 0;
 }
 __device__ __forceinline__ int small_kc(const SmallGemm& g) { return g.K < kSmallKC ? g.K : kSmallKC; }
 __device__ __forceinline__ int small_nchunks(const SmallGemm& g) { return g.K / small_kc(g); }
-__device__ __forceinline__ int small_unit(int j) { return (int)blockIdx.x + j * (int)gridDim.x; }
+// unit j of this CTA (units go round robin over the group's CTAs)
+__device__ __forceinline__ int small_unit(const SmallCtx& P, int j) { return P.rank + j * P.gsize; }
 
-__device__ __forceinline__ int small_phase_workers(const SmallPhase& ph) {
-  return ph.kind == 1 ? ph.a.num_heads : workers(gemm_units(ph.g));
+__device__ __forceinline__ int small_phase_workers(const SmallCtx& P, const SmallPhase& ph) {
+  return ph.kind == 1 ? ph.a.num_heads : workers(P, gemm_units(ph.g));
 }
 
 // ---------------------------------------------------------------- weight producer (warp 8)
@@ -367,8 +383,12 @@ struct SmallRing {
 
 // Streams this CTA's weight chunks of every GEMM phase, in the order the
 // compute warps consume them, into the slot ring; runs ahead as far as free
-// slots allow.  Lanes 0..7 each copy one weight row per chunk.
-__device__ __forceinline__ void small_producer(const SmallCtx& P, int total, uint8_t* smem, SmallRing& R) {
+// slots allow.  Lanes 0..7 each copy one weight row per chunk.  GROUPS: the
+// grid may hold several groups, and a CTA more than kSmallMaxUnits units of
+// a phase (else one group, one pass).  [k0, k1): the sample's packed keys.
+template <bool GROUPS>
+__device__ __forceinline__ void small_producer(const SmallCtx& P, int total, int k0, int k1, uint8_t* smem,
+                                               SmallRing& R) {
   const int lane = threadIdx.x & 31;
   uint32_t item = 0;
   bool ok = true;
@@ -382,16 +402,16 @@ __device__ __forceinline__ void small_producer(const SmallCtx& P, int total, uin
     const SmallPhase& ph = P.phases[gp];
     if (ph.kind == 0) {
       const SmallGemm& g = ph.g;
-      const int nu = small_my_units(g);
+      const int nu = small_my_units(P, g);
       for (int j = 0; j < nu; ++j)
-        l2_prefetch_hint(g.W + (size_t)small_unit(j) * kSmallUF * g.K, (uint32_t)(kSmallUF * g.K * 2),
+        l2_prefetch_hint(g.W + (size_t)small_unit(P, j) * kSmallUF * g.K, (uint32_t)(kSmallUF * g.K * 2),
                          stream_policy);
-    } else if (ph.a.kspan != nullptr && (int)blockIdx.x < ph.a.num_heads) {
-      // K and V of this CTA's head: contiguous rows of the head-major cache
-      const uint32_t bytes = (uint32_t)P.vofs[1] * (uint32_t)P.dh * 2u;
+    } else if (ph.a.kspan != nullptr && P.rank < ph.a.num_heads) {
+      // K and V of this CTA's head: the sample's contiguous rows of the head-major cache
+      const uint32_t bytes = (uint32_t)(k1 - k0) * (uint32_t)P.dh * 2u;
       if (bytes > 0) {
-        l2_prefetch(ph.a.k + (size_t)blockIdx.x * ph.a.kv_head_stride, bytes);
-        l2_prefetch(ph.a.v + (size_t)blockIdx.x * ph.a.kv_head_stride, bytes);
+        l2_prefetch(ph.a.k + (size_t)P.rank * ph.a.kv_head_stride + (size_t)k0 * P.dh, bytes);
+        l2_prefetch(ph.a.v + (size_t)P.rank * ph.a.kv_head_stride + (size_t)k0 * P.dh, bytes);
       }
     }
   };
@@ -402,7 +422,11 @@ __device__ __forceinline__ void small_producer(const SmallCtx& P, int total, uin
     const SmallPhase& ph = P.phases[gp];
     if (ph.kind != 0) continue;
     const SmallGemm& g = ph.g;
-    const int nu = small_my_units(g), nch = small_nchunks(g), kc = small_kc(g);
+    const int nu_all = small_my_units(P, g), nch = small_nchunks(g), kc = small_kc(g);
+    // the compute warps take the units in passes of up to kSmallMaxUnits,
+    // each pass chunk by chunk: the same order here
+    for (int u0 = 0; u0 < nu_all && ok; u0 += kSmallMaxUnits) {
+    const int nu = GROUPS ? min(kSmallMaxUnits, nu_all - u0) : nu_all;
     for (int c = 0; c < nch && ok; ++c) {
       for (int j = 0; j < nu; ++j, ++item) {
         const int slot = (int)(item % kSmallSlots);
@@ -416,10 +440,13 @@ __device__ __forceinline__ void small_producer(const SmallCtx& P, int total, uin
         if (!good) { ok = false; break; }
         if (lane < kSmallUF) {
           uint8_t* dst = smem + kSmRing + slot * kSlotBytes + lane * kSlotRow * 2;
-          const __nv_bfloat16* src = g.W + ((size_t)small_unit(j) * kSmallUF + lane) * g.K + (size_t)c * kc;
+          const __nv_bfloat16* src =
+              g.W + ((size_t)small_unit(P, u0 + j) * kSmallUF + lane) * g.K + (size_t)c * kc;
           bulk_g2s_hint(dst, src, (uint32_t)kc * 2u, &R.full[slot], stream_policy);
         }
       }
+    }
+    if (!GROUPS) break;
     }
   }
   // Let every copy issued land before the CTA can exit: wait for the last
@@ -458,13 +485,14 @@ __device__ __forceinline__ void small_issue_x(const SmallGemm& g, uint8_t* smem,
 
 // Bias and, for the residual and Euler epilogues, the old output values of
 // this CTA's units: one cp.async group, waited for before the epilogue.
-__device__ __forceinline__ void small_issue_side(const SmallGemm& g, int nu, uint8_t* smem) {
+__device__ __forceinline__ void small_issue_side(const SmallGemm& g, const SmallCtx& P, int u0, int nu,
+                                                 uint8_t* smem) {
   const int tid = threadIdx.x;
   const float* bsrc = g.epi == EPI_SWISH_VEC_BF16 ? g.vec : g.bias;
   if (bsrc != nullptr && tid < 2 * nu) {
     const int j = tid >> 1, q = tid & 1;
     cp_async16(reinterpret_cast<float*>(smem + kSmBias) + j * kSmallUF + q * 4,
-               bsrc + small_unit(j) * kSmallUF + q * 4, true);
+               bsrc + small_unit(P, u0 + j) * kSmallUF + q * 4, true);
   }
   if (g.epi == EPI_RESID_F32 || g.epi == EPI_EULER) {
     float* hold = reinterpret_cast<float*>(smem + kSmHold);
@@ -472,7 +500,7 @@ __device__ __forceinline__ void small_issue_side(const SmallGemm& g, int nu, uin
       const int j = i / (g.rows * 2), rem = i - j * g.rows * 2, r = rem >> 1, q = rem & 1;
       cp_async16(hold + (j * kSmallMaxTok + r) * kSmallUF + q * 4,
                  reinterpret_cast<const float*>(g.out) + (size_t)(g.out_row_off + r) * g.ldo +
-                     small_unit(j) * kSmallUF + q * 4,
+                     small_unit(P, u0 + j) * kSmallUF + q * 4,
                  true);
     }
   }
@@ -905,13 +933,14 @@ __device__ __forceinline__ void small_mma_units(const SmallMmaIn& in, uint8_t* s
 // count sits in slot item % kSmallSlots, filled for the (item / kSmallSlots)-th
 // time; a phase's items go chunk by chunk (every unit's K-chunk 0, then 1 ...)
 // and every warp releases a slot after its last read of it.
+template <bool GROUPS>
 __device__ __forceinline__ bool small_gemm_phase(const SmallGemm& g, const AttnArgs& att, const SmallCtx& P,
                                                  uint8_t* smem, SmallRing& R, uint32_t& item, uint64_t* xbar,
                                                  uint32_t& xuse, int* fail) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gr = lane >> 2, tig = lane & 3;
-  const int nu = small_my_units(g), nch = small_nchunks(g), kc = small_kc(g);
-  small_issue_side(g, nu, smem);
+  const int nu_all = small_my_units(P, g), nch = small_nchunks(g), kc = small_kc(g);
+  small_issue_side(g, P, 0, GROUPS ? min(kSmallMaxUnits, nu_all) : nu_all, smem);
   bool ok = true;
   if (g.x_mode == 0) {
     small_issue_x(g, smem, xbar);
@@ -958,70 +987,108 @@ __device__ __forceinline__ bool small_gemm_phase(const SmallGemm& g, const AttnA
   // weight fragments: ldmatrix.x4 over k, k + 8, k + 16, k + 24 (two k-steps;
   // lanes 0-15 also address the x2 form of one k-step)
   const int wrow = (lane & 7) * kSlotRow + (lane >> 3) * 8;
-  const uint32_t base = item;
-  float acc[kSmallMaxUnits][2][4];
-  SmallMmaIn in{xa0, xa1, two, wrow, ks0, ks1, kc, nch, base};
-  switch (nu) {
-    case 1: small_mma_units<1, 2>(in, smem, R, P, ok, acc); break;
-    case 2: small_mma_units<2, 2>(in, smem, R, P, ok, acc); break;
-    case 3: small_mma_units<3, 2>(in, smem, R, P, ok, acc); break;
-    default: small_mma_units<4, 2>(in, smem, R, P, ok, acc); break;
-  }
-  item = base + (uint32_t)(nch * nu);
-  // all warps stay together from here on, also on a timeout
-  cp_async_wait<0>();   // bias / old values
-  csync();
-  float* red = reinterpret_cast<float*>(smem);   // over the X area, no longer read
+  // One pass over units u0 .. u0 + nu - 1 of this CTA (nu <= kSmallMaxUnits):
+  // MMAs, the cross-warp reduction through `red`, the epilogue.
+  auto pass = [&](int u0, int nu, float* red) {
+    const uint32_t base = item;
+    float acc[kSmallMaxUnits][2][4];
+    SmallMmaIn in{xa0, xa1, two, wrow, ks0, ks1, kc, nch, base};
+    switch (nu) {
+      case 1: small_mma_units<1, 2>(in, smem, R, P, ok, acc); break;
+      case 2: small_mma_units<2, 2>(in, smem, R, P, ok, acc); break;
+      case 3: small_mma_units<3, 2>(in, smem, R, P, ok, acc); break;
+      default: small_mma_units<4, 2>(in, smem, R, P, ok, acc); break;
+    }
+    item = base + (uint32_t)(nch * nu);
+    // all warps stay together from here on, also on a timeout
+    cp_async_wait<0>();   // bias / old values
+    csync();
 #pragma unroll
-  for (int j = 0; j < kSmallMaxUnits; ++j) {
-    if (j < nu) {
-      float* rw = red + ((warp * kSmallMaxUnits + j) * kSmallMaxTok) * kSmallUF;
+    for (int j = 0; j < kSmallMaxUnits; ++j) {
+      if (j < nu) {
+        float* rw = red + ((warp * kSmallMaxUnits + j) * kSmallMaxTok) * kSmallUF;
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const int tok = t * 16 + gr;
-        rw[tok * kSmallUF + 2 * tig] = acc[j][t][0];
-        rw[tok * kSmallUF + 2 * tig + 1] = acc[j][t][1];
-        rw[(tok + 8) * kSmallUF + 2 * tig] = acc[j][t][2];
-        rw[(tok + 8) * kSmallUF + 2 * tig + 1] = acc[j][t][3];
+        for (int t = 0; t < 2; ++t) {
+          const int tok = t * 16 + gr;
+          rw[tok * kSmallUF + 2 * tig] = acc[j][t][0];
+          rw[tok * kSmallUF + 2 * tig + 1] = acc[j][t][1];
+          rw[(tok + 8) * kSmallUF + 2 * tig] = acc[j][t][2];
+          rw[(tok + 8) * kSmallUF + 2 * tig + 1] = acc[j][t][3];
+        }
       }
     }
-  }
-  csync();
-  const bool has_bias = (g.epi == EPI_SWISH_VEC_BF16 ? g.vec : g.bias) != nullptr;
-  const float* biases = reinterpret_cast<const float*>(smem + kSmBias);
-  const float* holds = reinterpret_cast<const float*>(smem + kSmHold);
-  // a phase that writes h also leaves the LayerNorm statistics piece of every
-  // (row, unit) it wrote: the 8 lanes 8i .. 8i + 7 hold one (unit, row), as
-  // the CTA's outputs are walked unit by unit, row by row, column by column
-  const bool pieces = g.epi == EPI_F32 || g.epi == EPI_RESID_F32;
-  const int per_unit = g.rows * kSmallUF, n_out = nu * per_unit;
-  for (int base = 0; base < n_out; base += kSmallCompute) {   // the same trip count in every thread
-    const int idx = base + (int)threadIdx.x;
-    const bool mine = idx < n_out;
-    const int j = mine ? idx / per_unit : 0, rem = idx - j * per_unit;
-    const int tok = rem / kSmallUF, fi = rem - tok * kSmallUF;
-    float r = 0.0f;
-    if (mine) {
-      float v = 0.0f;
+    csync();
+    const bool has_bias = (g.epi == EPI_SWISH_VEC_BF16 ? g.vec : g.bias) != nullptr;
+    const float* biases = reinterpret_cast<const float*>(smem + kSmBias);
+    const float* holds = reinterpret_cast<const float*>(smem + kSmHold);
+    // a phase that writes h also leaves the LayerNorm statistics piece of
+    // every (row, unit) it wrote: the 8 lanes 8i .. 8i + 7 hold one (unit,
+    // row), as the CTA's outputs are walked unit by unit, row by row, column
+    // by column
+    const bool pieces = g.epi == EPI_F32 || g.epi == EPI_RESID_F32;
+    const int per_unit = g.rows * kSmallUF, n_out = nu * per_unit;
+    for (int b0 = 0; b0 < n_out; b0 += kSmallCompute) {   // the same trip count in every thread
+      const int idx = b0 + (int)threadIdx.x;
+      const bool mine = idx < n_out;
+      const int j = mine ? idx / per_unit : 0, rem = idx - j * per_unit;
+      const int tok = rem / kSmallUF, fi = rem - tok * kSmallUF;
+      float r = 0.0f;
+      if (mine) {
+        float v = 0.0f;
 #pragma unroll
-      for (int w = 0; w < kSmallWarps; ++w) v += red[((w * kSmallMaxUnits + j) * kSmallMaxTok + tok) * kSmallUF + fi];
-      r = small_epilogue(g, small_unit(j) * kSmallUF + fi, tok, v, has_bias ? biases[j * kSmallUF + fi] : 0.0f,
-                         holds[(j * kSmallMaxTok + tok) * kSmallUF + fi]);
+        for (int w = 0; w < kSmallWarps; ++w)
+          v += red[((w * kSmallMaxUnits + j) * kSmallMaxTok + tok) * kSmallUF + fi];
+        r = small_epilogue(g, small_unit(P, u0 + j) * kSmallUF + fi, tok, v,
+                           has_bias ? biases[j * kSmallUF + fi] : 0.0f, holds[(j * kSmallMaxTok + tok) * kSmallUF + fi]);
+      }
+      if (pieces) {
+        const float2 pc = small_piece8(r);
+        if (mine && fi == 0 && ok)
+          P.ln_part[(size_t)(g.out_row_off + tok) * kLnPieces + small_unit(P, u0 + j)] = pc;
+      }
     }
-    if (pieces) {
-      const float2 pc = small_piece8(r);
-      if (mine && fi == 0 && ok) P.ln_part[(size_t)(g.out_row_off + tok) * kLnPieces + small_unit(j)] = pc;
+    // the action encoder's output row 0 is the state row, copied (its pieces too)
+    if (g.state_row != nullptr && (int)threadIdx.x < 32 * ((nu * kSmallUF + 31) / 32)) {
+      const int t = threadIdx.x;
+      const bool mine = t < nu * kSmallUF;
+      const int n = small_unit(P, u0 + t / kSmallUF) * kSmallUF + t % kSmallUF;
+      const float v = mine ? g.state_row[n] : 0.0f;
+      if (mine) reinterpret_cast<float*>(g.out)[n] = v;
+      const float2 pc = small_piece8(v);
+      if (mine && t % kSmallUF == 0 && ok) P.ln_part[small_unit(P, u0 + t / kSmallUF)] = pc;
     }
-  }
-  // the action encoder's output row 0 is the state row, copied (its pieces too)
-  if (g.state_row != nullptr && (int)threadIdx.x < 32 * ((nu * kSmallUF + 31) / 32)) {
-    const int t = threadIdx.x;
-    const bool mine = t < nu * kSmallUF;
-    const int n = small_unit(t / kSmallUF) * kSmallUF + t % kSmallUF;
-    const float v = mine ? g.state_row[n] : 0.0f;
-    if (mine) reinterpret_cast<float*>(g.out)[n] = v;
-    const float2 pc = small_piece8(v);
-    if (mine && t % kSmallUF == 0 && ok) P.ln_part[small_unit(t / kSmallUF)] = pc;
+  };
+  if constexpr (!GROUPS) {
+    pass(0, nu_all, reinterpret_cast<float*>(smem));   // the reduction over the X area, no longer read
+  } else {
+    // More than kSmallMaxUnits units: several passes.  The reduction goes
+    // after the activation rows (they are read again), or, when the rows
+    // fill the area (the FF2 input), over them, and they are copied in again
+    // for each later pass.
+    int red_off = 0;
+    bool reload = false;
+    if (nu_all > kSmallMaxUnits) {
+      const int off = small_ln_stage_offset(g.rows, g.K);
+      if (off + kSmRedBytes <= kSmLnScratch) red_off = off;
+      else reload = true;
+      if (reload && g.x_mode != 0) ok = false;   // computed rows cannot be copied in again (the host rules it out)
+    }
+    for (int u0 = 0; u0 < nu_all; u0 += kSmallMaxUnits) {
+      const int nu = min(kSmallMaxUnits, nu_all - u0);
+      if (u0 > 0) {   // the previous pass ended with a barrier: side area and rows are free
+        small_issue_side(g, P, u0, nu, smem);
+        if (reload) {
+          small_issue_x(g, smem, xbar);
+          if (!mbar_wait(xbar, xuse & 1u, P.err)) ok = false;
+          ++xuse;
+        }
+      }
+      pass(u0, nu, reinterpret_cast<float*>(smem + red_off));
+      if (u0 + kSmallMaxUnits < nu_all) {   // another pass: its side loads and rows may overwrite these
+        cp_async_wait<0>();
+        csync();
+      }
+    }
   }
   // One barrier ends the phase: every thread's epilogue stores precede the
   // arrival (thread 0 releases right after it), the X area and the slot of
@@ -1193,21 +1260,22 @@ struct SmallSmem {
 };
 
 __device__ __forceinline__ int small_category(const SmallPlan& P) {
-  int c = 0;   // category of the single sample (an out-of-range id was routed to 0)
+  int c = 0;   // category of the plan's sample (an out-of-range id was routed to 0)
   for (int i = 0; i < P.C; ++i)
-    if (P.seg[i] == 0 && P.seg[i + 1] == 1) c = i;
+    if (P.seg[i] <= P.sample && P.sample < P.seg[i + 1]) c = i;
   return c;
 }
 
-// One thread per phase: the descriptor table of the whole loop.
+// One thread per (sample, phase): the descriptor tables of the whole loop.
 __global__ void small_describe_kernel(const SmallPlan* __restrict__ plan) {
-  const SmallPlan& P = *plan;
   pdl_wait();
   pdl_launch_dependents();
-  const int per_step = small_phases_per_step(P.L);
-  const int total = per_step * P.K;
-  const int gp = blockIdx.x * blockDim.x + threadIdx.x;
-  if (gp >= total) return;
+  const int per_step = small_phases_per_step(plan->L);
+  const int total = per_step * plan->K;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= total * plan->groups) return;
+  const SmallPlan& P = plan[i / total];
+  const int gp = i % total;
   small_describe(P, small_category(P), gp / per_step, gp % per_step, P.phases[gp]);
 }
 
@@ -1223,7 +1291,7 @@ __device__ __forceinline__ void small_fetch_phase(const SmallPhase* phases, int 
   cp_async_commit();
 }
 
-template <int DH>
+template <int DH, bool GROUPS>
 __global__ void __launch_bounds__(kSmallThreads, 1) small_loop_kernel(const SmallPlan* __restrict__ plan) {
   extern __shared__ __align__(16) uint8_t smem[];
   // phase descriptors: slot gp % 3 holds the current phase; the one two ahead
@@ -1233,9 +1301,17 @@ __global__ void __launch_bounds__(kSmallThreads, 1) small_loop_kernel(const Smal
   __shared__ __align__(8) uint64_t s_xbar;
   __shared__ int s_ok;
   __shared__ int s_fail;
-  const SmallCtx P = {plan->err,  plan->counters, plan->h,  plan->eps,     plan->phases,
-                      plan->vofs, plan->dh,       plan->nh, plan->max_tok, &plan->kv_map, plan->ln_part};
-  const int total = small_phases_per_step(plan->L) * plan->K;
+  // the grid is cut into plan->groups equal groups of CTAs, one per sample:
+  // group q runs the loop of sample q on its own plan, counters and tables
+  // (without GROUPS there is one group: the whole grid, one pass per phase)
+  const int gsize = GROUPS ? (int)gridDim.x / plan->groups : (int)gridDim.x;
+  const int group = GROUPS ? (int)blockIdx.x / gsize : 0;
+  if (group >= plan->groups) return;   // (the host launches groups x gsize CTAs)
+  const SmallPlan* gpl = plan + group;
+  const SmallCtx P = {gpl->err,  gpl->counters, gpl->h,  gpl->eps,     gpl->phases,
+                      gpl->vofs, gpl->dh,       gpl->nh, gpl->max_tok, &gpl->kv_map, gpl->ln_part,
+                      (int)blockIdx.x - group * gsize, gsize};
+  const int total = small_phases_per_step(gpl->L) * gpl->K;
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSmallSlots; ++i) {
       mbar_init(&s_ring.full[i], 1);
@@ -1247,7 +1323,8 @@ __global__ void __launch_bounds__(kSmallThreads, 1) small_loop_kernel(const Smal
   }
   __syncthreads();
   if (threadIdx.x >= kSmallCompute) {
-    small_producer(P, total, smem, s_ring);
+    // the key span was written by an earlier kernel: read once, for the L2 requests
+    small_producer<GROUPS>(P, total, gpl->kspan[0], gpl->kspan[1], smem, s_ring);
     return;
   }
   small_fetch_phase(P.phases, 0, &s_ph[0]);
@@ -1261,15 +1338,15 @@ __global__ void __launch_bounds__(kSmallThreads, 1) small_loop_kernel(const Smal
   for (int gp = 0; gp < total; ++gp) {
     const SmallPhase& cur = s_ph[slot];
     if (gp + 2 < total) small_fetch_phase(P.phases, gp + 2, &s_ph[slot == 0 ? 2 : slot - 1]);
-    const int w = small_phase_workers(cur);
+    const int w = small_phase_workers(P, cur);
     bool ok = true;
-    if ((int)blockIdx.x < w) {
+    if (P.rank < w) {
       ok = small_wait(P, gp - 1, prev_workers, &s_ok);
       if (ok) {
         if (cur.kind == 0)
-          ok = small_gemm_phase(cur.g, cur.a, P, smem, s_ring, item, &s_xbar, xuse, &s_fail);
+          ok = small_gemm_phase<GROUPS>(cur.g, cur.a, P, smem, s_ring, item, &s_xbar, xuse, &s_fail);
         else
-          ok = small_cross_attention<DH>(cur, P, blockIdx.x, smem, &s_xbar, xuse, &s_fail);
+          ok = small_cross_attention<DH>(cur, P, P.rank, smem, &s_xbar, xuse, &s_fail);
         if (ok) small_arrive(P, gp);
       }
     }
@@ -1284,7 +1361,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1) small_loop_kernel(const Smal
       return;
     }
     prev_workers = w;
-    if ((int)blockIdx.x >= w) {
+    if (P.rank >= w) {
       // an idle CTA: the next descriptor has landed, and every compute thread
       // is done with this one before its slot is refilled (a working CTA's
       // phase ended with that barrier)

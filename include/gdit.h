@@ -69,8 +69,9 @@ extern "C" {
 /* flags for gdit_config.flags */
 #define GDIT_FLAG_STRICT_PROFILES 1u  /* unprepared (batch, seq, steps) -> GDIT_EPROFILE, never a capture */
 #define GDIT_FLAG_NO_GRAPH 2u         /* run eagerly (no CUDA graph); same kernels, for debugging */
-#define GDIT_FLAG_NO_SMALL 4u         /* never use the single-sample persistent loop (batch 1 then runs the
-                                         same per-layer kernels as larger batches) */
+#define GDIT_FLAG_NO_SMALL 4u         /* never use the persistent loop of batches 1-4 (one CTA group per
+                                         sample); they then run the same per-layer kernels as larger
+                                         batches */
 #define GDIT_FLAG_NO_TMA_STORE 8u     /* DiT GEMMs store their outputs thread by thread instead of by TMA */
 #define GDIT_FLAG_NO_PAIR 16u         /* the DiT GEMMs and the cross K/V projection never run on CTA pairs
                                          (cta_group::2, 256-row tiles) */

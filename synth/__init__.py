@@ -212,7 +212,7 @@ WORKLOADS: Dict[str, Workload] = {
     "sweep256": Workload("sweep256", GEOM_FULL, batch=256, seq=256, num_steps=4, id_low=0, id_high=31,
                          description="B=256, S=256 all valid, ids~U{0..31}, K=4"),
 }
-for _b in (1, 8, 32, 128):
+for _b in (1, 2, 4, 8, 32, 128):
     WORKLOADS[f"sweep{_b}"] = Workload(
         f"sweep{_b}", GEOM_FULL, batch=_b, seq=256, num_steps=4, id_low=0, id_high=31,
         fixed_ids=(0,) if _b == 1 else None,

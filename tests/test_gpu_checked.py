@@ -26,11 +26,13 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def _cases():
-    """A ragged tiny batch (general path), one tiny sample (the single-sample
-    loop) and the full-size batched workload (ragged keys, 32 embodiments)."""
+    """Ragged tiny batches of 3 (the persistent loop, one CTA group per
+    sample) and 6 (the per-layer path), one tiny sample (the loop, one group)
+    and the full-size batched workload (ragged keys, 32 embodiments)."""
     tiny = synth.workload("tiny", batch=3, fixed_ids=(1, 0, 1), valid_min=1)
     tiny_w = synth.make_weights(tiny.geom)
     return [("tiny", tiny, tiny_w, 5),
+            ("tiny6", synth.workload("tiny", batch=6, fixed_ids=(1, 0), valid_min=1), tiny_w, 8),
             ("tiny_b1", synth.workload("tiny", batch=1, fixed_ids=(1,), valid_min=1), tiny_w, 6),
             ("batched", synth.WORKLOADS["batched"], synth.make_weights(synth.GEOM_FULL), 7)]
 

@@ -309,6 +309,64 @@ def test_single_sample_loop_eager_equals_graph(tiny_weights):
     np.testing.assert_array_equal(b, c)
 
 
+def test_grouped_loop_matches_general_path_and_oracle(full_weights, full_model, head_full):
+    """2 <= B <= 4 run the same persistent loop with one group of CTAs per
+    sample (each CTA takes its units of a linear in several passes).  At
+    full size, mixed embodiments and ragged valid lengths, it must agree with
+    the per-layer path (GDIT_FLAG_NO_SMALL) and, on sampled rows, the oracle."""
+    from flow_matching_dit_b200 import GDIT_FLAG_NO_SMALL, ActionHead
+    for B, seed in ((2, 61), (4, 62)):
+        w = synth.workload("sweep8", batch=B, valid_min=40, id_low=0, id_high=31)
+        inp = synth.make_inputs(w, seed=seed)
+        grouped, st = run_gpu(head_full, inp, w.num_steps)
+        assert st == 0
+        with ActionHead(w.geom, full_weights, max_batch=B, max_seq=w.seq, flags=GDIT_FLAG_NO_SMALL) as general:
+            gen, st2 = run_gpu(general, inp, w.num_steps)
+        assert st2 == 0
+        assert_parity(grouped, gen, inp["init_noise"], f"grouped loop vs general path, B={B}")
+        rows = [0, B - 1]
+        ref = run_oracle(full_weights, w.geom, inp, w.num_steps, samples=rows, model=full_model)
+        assert_parity(grouped[rows], ref, inp["init_noise"][rows], f"grouped loop vs oracle, B={B}")
+
+
+@pytest.mark.parametrize("B", [2, 3, 4, 5, 6, 7, 8])
+def test_grouped_loop_every_batch_size(head_tiny, tiny_weights, B):
+    """Every group count of the loop (B <= 4) and the per-layer path just
+    above it, on the tiny DiT: both embodiments, ragged (and one empty) key
+    lists, one out-of-range id (its row NaN, the others unaffected), every
+    row against the oracle."""
+    from flow_matching_dit_b200._lib import GDIT_EDEVICE
+    w = synth.workload("tiny", batch=B, valid_min=1, fixed_ids=None, id_low=0, id_high=1)
+    inp = synth.make_inputs(w, seed=70 + B)
+    inp["vl_mask"][B - 1] = 0                          # a sample with no valid key
+    bad = B // 2 if B >= 3 else None
+    if bad is not None:
+        inp["embodiment_id"][bad] = 9
+    gpu, st = run_gpu(head_tiny, inp, 4)
+    assert st == (GDIT_EDEVICE if bad is not None else 0)
+    rows = [b for b in range(B) if b != bad]
+    if bad is not None:
+        assert np.isnan(gpu[bad]).all()
+    ok = {k: v[rows] for k, v in inp.items()}
+    ref = run_oracle(tiny_weights, w.geom, ok, 4)
+    assert_parity(gpu[rows], ref, ok["init_noise"], f"grouped loop B={B}")
+    assert head_tiny.sync_status() == 0
+
+
+def test_grouped_loop_eager_equals_graph(tiny_weights):
+    require_gpu()
+    from flow_matching_dit_b200 import GDIT_FLAG_NO_GRAPH, ActionHead
+    w = synth.workload("tiny", batch=6, fixed_ids=None, id_low=0, id_high=1, valid_min=10)
+    inp = synth.make_inputs(w, seed=23)
+    with ActionHead(synth.GEOM_TINY, tiny_weights, max_batch=6, max_seq=64, flags=GDIT_FLAG_NO_GRAPH) as eager:
+        a, _ = run_gpu(eager, inp, 4)
+    with ActionHead(synth.GEOM_TINY, tiny_weights, max_batch=6, max_seq=64) as graph:
+        b, _ = run_gpu(graph, inp, 4)
+        c, _ = run_gpu(graph, inp, 4)
+    np.testing.assert_array_equal(a, b)
+    np.testing.assert_array_equal(b, c)
+
+
 @pytest.mark.parametrize("case", ["empty", "one_token", "bad_id"])
 def test_single_sample_loop_edge_cases(head_tiny, tiny_weights, case):
     from flow_matching_dit_b200._lib import GDIT_EDEVICE
@@ -409,9 +467,9 @@ def test_bounded_wait_expiry_is_reported_and_the_device_stays_usable(head_tiny, 
 # ---------------------------------------------------------------- image/text split of the cross layers
 
 @pytest.mark.parametrize("n", [1, 2])
-# 1: the persistent single-sample loop; 3: per-layer kernels, split attention schedule;
-# 160 (x 4 heads >= 4 x SMs): per-layer kernels, warp attention schedule (rows sampled)
-@pytest.mark.parametrize("batch", [1, 3, 160])
+# 1, 3: the persistent loop (one and three CTA groups); 12: per-layer kernels, split attention
+# schedule; 160 (x 4 heads >= 4 x SMs): per-layer kernels, warp attention schedule (rows sampled)
+@pytest.mark.parametrize("batch", [1, 3, 12, 160])
 def test_image_text_split_matches_oracle(n, batch):
     """AlternateVLDiT with attend_text_every_n_blocks = n on a 4-layer tiny DiT
     (cross blocks 0 and 2): ragged valid lengths and seeded image masks; the
@@ -431,7 +489,7 @@ def test_image_text_split_matches_oracle(n, batch):
         gpu = out.cpu().numpy()
         plain = head.get_action(*to_dev(inp), num_steps=4).cpu().numpy()   # no image mask: no image token
     assert st == 0
-    rows = list(range(batch)) if batch <= 3 else [0, 77, batch - 1]
+    rows = list(range(batch)) if batch <= 3 else [0, batch // 2, batch - 1]
     ref = oracle.get_action(W, g, inp["backbone_features"], inp["vl_mask"], inp["state"], inp["embodiment_id"],
                             inp["init_noise"], 4, image_mask=img, samples=rows)
     assert_parity(gpu[rows], ref, inp["init_noise"][rows], f"image/text split n={n} B={batch}")
