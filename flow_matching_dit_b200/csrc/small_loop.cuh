@@ -393,10 +393,13 @@ __device__ __forceinline__ void small_producer(const SmallCtx& P, int total, int
   uint32_t item = 0;
   bool ok = true;
   // The weights are read once per Euler step and 0.75 GB of them pass
-  // through L2 per step: they are marked first to evict, so that the
-  // activations, the per-step tables and the K/V cache (read every step)
-  // stay in L2.
-  const uint64_t stream_policy = policy_evict_first();
+  // through L2 per step: with one group they are marked first to evict, so
+  // that the activations, the per-step tables and the K/V cache (read every
+  // step) stay in L2.  With several groups every group reads every weight
+  // line within a few microseconds of the others: evict-first lines were
+  // read from DRAM again (4.7 GB per call at B = 2 against 2.95 GB), so they
+  // keep the normal policy (B = 4: 7.39 ms per call against 7.61 ms).
+  const uint64_t stream_policy = GROUPS ? policy_evict_normal() : policy_evict_first();
   auto l2_ahead = [&](int gp) {   // the chunks of phase gp (if any) towards L2
     if (lane != 0 || gp >= total) return;
     const SmallPhase& ph = P.phases[gp];
