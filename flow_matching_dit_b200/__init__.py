@@ -20,8 +20,8 @@ from typing import Dict, List, Optional
 import numpy as np
 
 from . import _lib
-from ._lib import (GDIT_BF16, GDIT_F32, GDIT_FLAG_NO_GRAPH, GDIT_FLAG_NO_PAIR, GDIT_FLAG_NO_SMALL,  # noqa: F401
-                   GDIT_FLAG_NO_TMA_STORE, GDIT_FLAG_STRICT_PROFILES,
+from ._lib import (GDIT_BF16, GDIT_F32, GDIT_FLAG_NO_GRAPH, GDIT_FLAG_NO_PAIR, GDIT_FLAG_NO_SKINNY,  # noqa: F401
+                   GDIT_FLAG_NO_SMALL, GDIT_FLAG_NO_TMA_STORE, GDIT_FLAG_STRICT_PROFILES,
                    GditError, check, lib)
 from .build import build  # noqa: F401
 

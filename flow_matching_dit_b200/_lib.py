@@ -30,6 +30,7 @@ GDIT_FLAG_NO_GRAPH = 2
 GDIT_FLAG_NO_SMALL = 4
 GDIT_FLAG_NO_TMA_STORE = 8
 GDIT_FLAG_NO_PAIR = 16
+GDIT_FLAG_NO_SKINNY = 32
 
 
 class gdit_config(ctypes.Structure):

@@ -28,6 +28,7 @@
 
 #include "gdit.h"
 #include "attention.cuh"
+#include "gemm_skinny.cuh"
 #include "gemm_tc.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
@@ -211,7 +212,69 @@ struct GemmOp {
   int rows_kind = 0;   // 0 fixed M, 1 = total valid tokens, 2 = all rows (grouped)
   long long weight_bytes = 0;
   int out_bytes = 2;
+  const void* a_ptr = nullptr;   // the operands (the skinny-M kernel takes plain pointers)
+  const void* b_ptr = nullptr;
+  int sk_mt = 0;                 // > 0: the skinny-M kernel, row blocks of 16 sk_mt rows
+  int sk_nu = 0;                 // its units of 8 features per item
+  int sk_stages = 0;             // its ring depth
 };
+
+// Few rows (a batch of a few samples) use the skinny-M kernel: all SMs stream
+// the weights instead of a handful of 128-row tensor-core tiles.
+constexpr long long kSkinnyMaxRows = 160;
+// per-item cost beyond its bytes (pipeline fill, reduction, epilogue), in
+// bytes of streaming
+constexpr double kSkinnyItemBytes = 64.0 * 1024;
+
+// Row block (16 mt rows) and units per item for an [M, K] x [N, K]^T GEMM:
+// the least bytes streamed by the busiest CTA (items go round robin over the
+// SMs), with a ring of at least 3 stages.  False if none fits.
+bool plan_skinny(long long M, int N, int K, int num_sms, int& mt, int& nu, int& stages) {
+  double best = 0.0;
+  bool found = false;
+  const long long units = N / 8;
+  for (int m : {1, 2, 3, 5}) {
+    const long long rows = 16LL * m, nrb = (M + rows - 1) / rows;
+    for (int u = 1; u <= sk_max_units(m); ++u) {
+      const long long items = nrb * ((units + u - 1) / u);
+      const long long rounds = (items + num_sms - 1) / num_sms;
+      const int st = std::min(8, (kSkSmemMax - 1024 - sk_red_bytes(m, u) - 64) / sk_stage_bytes(m, u));
+      if (st < 3) continue;
+      const double cost = (double)rounds * ((double)(std::min(rows, M) + 8LL * u) * K * 2.0 + kSkinnyItemBytes);
+      if (!found || cost < best) {
+        found = true;
+        best = cost;
+        mt = m;
+        nu = u;
+        stages = st;
+      }
+    }
+  }
+  return found;
+}
+
+// Switch a planned dense GEMM with few rows to the skinny-M kernel (plain
+// [M, K] x [N, K]^T layout, one output row per input row, no split).
+void enable_skinny(GemmOp& op, int num_sms) {
+  GemmArgs& a = op.args;
+  const bool epi_ok = a.epi == EPI_BF16 || a.epi == EPI_GELU_BF16 || a.epi == EPI_RELU_BF16 || a.epi == EPI_F32 ||
+                      a.epi == EPI_RESID_F32;
+  const bool aligned = ((uintptr_t)op.a_ptr % 16) == 0 && ((uintptr_t)op.b_ptr % 16) == 0;
+  if (a.M > kSkinnyMaxRows || a.M < 1 || a.splits != 1 || a.num_groups != 0 || a.m_dev != nullptr || a.nblk != 0 ||
+      a.in_group != 0x7fffffff || a.out_off != 0 || !epi_ok || a.N % 8 != 0 || a.K % 64 != 0 || !aligned)
+    return;
+  int mt, nu, stages;
+  if (!plan_skinny(a.M, a.N, a.K, num_sms, mt, nu, stages)) return;
+  op.sk_mt = mt;
+  op.sk_nu = nu;
+  op.sk_stages = stages;
+  op.ta = make_tmap(op.a_ptr, a.M, a.K, a.K, 16 * mt);
+  op.tb = make_tmap(op.b_ptr, a.N, a.K, a.K, 8 * nu);
+  const long long items = ((a.M + 16LL * mt - 1) / (16LL * mt)) * ((a.N / 8 + nu - 1) / nu);
+  op.grid = (int)std::min<long long>(items, num_sms);
+  op.pair = false;
+  a.tma_out = 0;
+}
 
 // Switch a planned dense GEMM to the TMA-store epilogue when its output is a
 // plain [M, N] matrix (no split-K, no row remap, no column blocking).
@@ -277,7 +340,35 @@ void launch_gemm_pair(const GemmOp& op, const GemmArgs& a, cudaStream_t s, bool 
   CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_tc_pair_kernel<BN>, op.ta, op.tb, op.to, a));
 }
 
+void launch_gemm_skinny(const GemmOp& op, const GemmArgs& a, cudaStream_t s, bool pdl) {
+  SkinnyArgs k;
+  k.W = static_cast<const __nv_bfloat16*>(op.b_ptr);
+  k.bias = a.bias;
+  k.out = a.out;
+  k.ldo = a.ldo;
+  k.M = a.M;
+  k.N = a.N;
+  k.K = a.K;
+  k.epi = a.epi;
+  k.nu = op.sk_nu;
+  k.stages = op.sk_stages;
+  k.err = a.err;
+  const int smem = sk_smem_bytes(op.sk_mt, op.sk_nu, op.sk_stages);
+  const dim3 grid(op.grid), block(kSkThreads);
+  switch (op.sk_mt) {
+    case 1: launch_k(s, pdl, gemm_skinny_kernel<1>, grid, block, smem, op.ta, op.tb, k); break;
+    case 2: launch_k(s, pdl, gemm_skinny_kernel<2>, grid, block, smem, op.ta, op.tb, k); break;
+    case 3: launch_k(s, pdl, gemm_skinny_kernel<3>, grid, block, smem, op.ta, op.tb, k); break;
+    case 5: launch_k(s, pdl, gemm_skinny_kernel<5>, grid, block, smem, op.ta, op.tb, k); break;
+    default: throw GditError(GDIT_EINVAL, fmt("bad skinny row block %d", op.sk_mt));
+  }
+}
+
 void launch_gemm(const GemmOp& op, const GemmArgs& a, cudaStream_t s, bool pdl) {
+  if (op.sk_mt > 0) {
+    launch_gemm_skinny(op, a, s, pdl);
+    return;
+  }
   if (op.pair) {
     if (op.bn == 256)
       launch_gemm_pair<256>(op, a, s, pdl);
@@ -912,6 +1003,11 @@ void set_kernel_attrs() {
   max_shared_carveout(small_loop_kernel<64, true>);
   max_shared_carveout(small_loop_kernel<32, true>);
   max_shared_carveout(small_describe_kernel);
+  for (const void* f : {(const void*)gemm_skinny_kernel<1>, (const void*)gemm_skinny_kernel<2>,
+                        (const void*)gemm_skinny_kernel<3>, (const void*)gemm_skinny_kernel<5>}) {
+    CUDA_TRY(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kSkSmemMax));
+    CUDA_TRY(cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
+  }
   set_attn_attrs<2, 64>();
   set_attn_attrs<4, 64>();
   set_attn_attrs<2, 32>();
@@ -1010,6 +1106,8 @@ GemmOp plan_gemm(gdit_handle* h, const void* A, long long a_rows, int K, const v
   a.splits = splits;
   op.ta = make_tmap(A, a_rows, K, K, kBM);
   op.tb = make_tmap(Bw, b_rows, K, K, bn);
+  op.a_ptr = A;
+  op.b_ptr = Bw;
   op.to = op.ta;   // placeholder unless the TMA-store epilogue is enabled
   const long long nt = (N + bn - 1) / bn;
   long long max_units = ((a_rows + kBM - 1) / kBM + (groups ? std::min<long long>(groups, a_rows) : 0)) * nt;
@@ -1150,6 +1248,8 @@ std::unique_ptr<Profile> build_profile(gdit_handle* h, int B, int S, int K, int 
       enable_pair(p->ff1[l], h->u, m.wff1[l], h->num_sms);
       enable_pair(p->ff2[l], h->f, m.wff2[l], h->num_sms);
     }
+    if ((h->cfg.flags & GDIT_FLAG_NO_SKINNY) == 0)
+      for (GemmOp* g : {&p->q[l], &p->o[l], &p->ff1[l], &p->ff2[l]}) enable_skinny(*g, h->num_sms);
   }
   // norm_out + proj_out on every token; only the H action rows are kept (compact)
   p->proj = plan_gemm(h, h->u, rows, D, m.proj_w, D, D, EPI_BF16, rows, 0, 0, 1);

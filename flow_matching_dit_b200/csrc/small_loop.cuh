@@ -168,21 +168,6 @@ struct SmallGemm {
   const float* state_row;    // EPI_F32 into h: also write h row 0 from this vector
 };
 
-__device__ __forceinline__ void ldmatrix_x2(uint32_t& r0, uint32_t& r1, const void* p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
-               : "=r"(r0), "=r"(r1)
-               : "r"(smem_u32(p)));
-}
-
-__device__ __forceinline__ void l2_prefetch(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
-__device__ __forceinline__ void l2_prefetch_hint(const void* p, uint32_t bytes, uint64_t policy) {
-  asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], %1, %2;" ::"l"(p), "r"(bytes), "l"(policy)
-               : "memory");
-}
-
 // barrier of the 8 compute warps (the producer warp never joins it)
 __device__ __forceinline__ void csync() { named_bar_sync(1, kSmallCompute); }
 

@@ -75,6 +75,9 @@ extern "C" {
 #define GDIT_FLAG_NO_TMA_STORE 8u     /* DiT GEMMs store their outputs thread by thread instead of by TMA */
 #define GDIT_FLAG_NO_PAIR 16u         /* the DiT GEMMs and the cross K/V projection never run on CTA pairs
                                          (cta_group::2, 256-row tiles) */
+#define GDIT_FLAG_NO_SKINNY 32u       /* the DiT GEMMs of few rows (batches of up to 9 samples on the
+                                         per-layer path) run on the tensor-core GEMM instead of the
+                                         skinny-M kernel */
 
 /* ------------------------------------------------------------------ config
  * Model geometry and capacity.  Every size is explicit.  Defaults of the

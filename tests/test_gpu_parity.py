@@ -353,6 +353,27 @@ def test_grouped_loop_every_batch_size(head_tiny, tiny_weights, B):
     assert head_tiny.sync_status() == 0
 
 
+def test_skinny_gemms_match_tensor_core_gemms_and_oracle(full_weights, full_model):
+    """The per-layer path at a few samples (B = 6, 102 rows) runs its DiT
+    linears on the skinny-M kernel; against the same path on the tensor-core
+    GEMM (GDIT_FLAG_NO_SKINNY) and, on sampled rows, the oracle."""
+    require_gpu()
+    from flow_matching_dit_b200 import GDIT_FLAG_NO_SKINNY, GDIT_FLAG_NO_SMALL, ActionHead
+    w = synth.workload("sweep8", batch=6, valid_min=40, id_low=0, id_high=31)
+    inp = synth.make_inputs(w, seed=63)
+    with ActionHead(w.geom, full_weights, max_batch=6, max_seq=w.seq, flags=GDIT_FLAG_NO_SMALL) as sk:
+        a, st = run_gpu(sk, inp, w.num_steps)
+    assert st == 0
+    with ActionHead(w.geom, full_weights, max_batch=6, max_seq=w.seq,
+                    flags=GDIT_FLAG_NO_SMALL | GDIT_FLAG_NO_SKINNY) as tc:
+        b, st2 = run_gpu(tc, inp, w.num_steps)
+    assert st2 == 0
+    assert_parity(a, b, inp["init_noise"], "skinny-M GEMMs vs tensor-core GEMMs, B=6")
+    rows = [0, 5]
+    ref = run_oracle(full_weights, w.geom, inp, w.num_steps, samples=rows, model=full_model)
+    assert_parity(a[rows], ref, inp["init_noise"][rows], "skinny-M GEMMs vs oracle, B=6")
+
+
 def test_grouped_loop_eager_equals_graph(tiny_weights):
     require_gpu()
     from flow_matching_dit_b200 import GDIT_FLAG_NO_GRAPH, ActionHead
