@@ -2088,6 +2088,9 @@ int gdit_test_gemm(const void* A, const void* B, const float* bias, float* C, in
                    void* cuda_stream) {
   const bool tma_out = getenv("GDIT_TEST_TMA_OUT") != nullptr;   // unit-test knob: exercise the TMA-store epilogue
   const bool pair = getenv("GDIT_TEST_PAIR") != nullptr;         // unit-test knob: the CTA-pair kernel (with TMA store)
+  // unit-test knob: the skinny-M kernel, "mt,nu" (a forced plan, items may
+  // exceed the SMs) or "0,0" (the planner's choice)
+  const char* skinny = getenv("GDIT_TEST_SKINNY");
   g_create_error.clear();
   return guarded(nullptr, [&] {
     REQUIRE(A && B && C, "NULL matrix");
@@ -2139,6 +2142,30 @@ int gdit_test_gemm(const void* A, const void* B, const float* bias, float* C, in
         op.tb = make_tmap(B, N, K, K, bn / 2);
         const long long pt = ((M + kPairBM - 1) / kPairBM) * nt;
         op.grid = (int)(2 * std::min<long long>(pt, sms / 2));
+      }
+    }
+    if (skinny != nullptr) {
+      REQUIRE(splits == 1, "the skinny-M kernel does not split K");
+      op.a_ptr = A;
+      op.b_ptr = B;
+      int mt = 0, nu = 0;
+      REQUIRE(std::sscanf(skinny, "%d,%d", &mt, &nu) == 2, "GDIT_TEST_SKINNY is \"mt,nu\"");
+      if (mt == 0) {
+        enable_skinny(op, sms);
+        REQUIRE(op.sk_mt > 0, "no skinny-M plan for M %d, N %d, K %d", M, N, K);
+      } else {
+        REQUIRE(mt == 1 || mt == 2 || mt == 3 || mt == 5, "mt must be 1, 2, 3 or 5");
+        REQUIRE(nu >= 1 && nu <= sk_max_units(mt), "nu must be in [1, %d]", sk_max_units(mt));
+        REQUIRE(N % 8 == 0 && K % 64 == 0, "the skinny-M kernel needs N %% 8 == 0 and K %% 64 == 0");
+        const int st = std::min(8, (kSkSmemMax - 1024 - sk_red_bytes(mt, nu) - 64) / sk_stage_bytes(mt, nu));
+        REQUIRE(st >= 2, "mt %d, nu %d do not fit shared memory", mt, nu);
+        op.sk_mt = mt;
+        op.sk_nu = nu;
+        op.sk_stages = st;
+        op.ta = make_tmap(A, M, K, K, 16 * mt);
+        op.tb = make_tmap(B, N, K, K, 8 * nu);
+        const long long items = ((M + 16LL * mt - 1) / (16LL * mt)) * ((N / 8 + nu - 1) / nu);
+        op.grid = (int)std::min<long long>(items, sms);
       }
     }
     launch_gemm(op, op.args, s, false);

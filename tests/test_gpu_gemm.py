@@ -63,6 +63,32 @@ def test_pair_gemm_matches_float64(M, N, K, bn, monkeypatch):
     np.testing.assert_allclose(C, ref, rtol=1e-5, atol=2e-5 * np.sqrt(K))
 
 
+@pytest.mark.parametrize("M,N,K,plan", [
+    (17, 1024, 1024, "2,1"),       # one sample's rows, one unit per item
+    (136, 1024, 1024, "2,5"),      # eight samples: 32-row blocks, ragged last block (8 rows)
+    (136, 4096, 1024, "3,6"),      # 258 items: CTAs take several items (pipeline across items)
+    (34, 384, 128, "1,16"),        # K of half a chunk (boxes past K read zeros)
+    (85, 96, 320, "5,5"),          # ragged unit block (12 units by 5), K tail of 64 columns
+    (160, 1024, 4096, "5,7"),      # long K (16 chunks), two 80-row blocks
+    (150, 64, 64, "3,2"),          # K of one box
+    (136, 3072, 1024, "0,0"),      # the planner's choice
+])
+def test_skinny_gemm_matches_float64(M, N, K, plan, monkeypatch):
+    """The skinny-M kernel (row blocks x 8-feature units over all SMs, TMA
+    boxes, mma.sync, fixed-order cross-warp sums) against float64 products."""
+    require_gpu()
+    monkeypatch.setenv("GDIT_TEST_SKINNY", plan)
+    import torch
+    from flow_matching_dit_b200 import test_gemm
+    g = torch.Generator().manual_seed(M * 3 + N + K)
+    A = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    B = torch.randn(N, K, generator=g).to(torch.bfloat16)
+    bias = torch.randn(N, generator=g)
+    C = test_gemm(A.cuda(), B.cuda(), bias.cuda(), bn=64, splits=1).cpu().double().numpy()
+    ref = A.double().numpy() @ B.double().numpy().T + bias.double().numpy()
+    np.testing.assert_allclose(C, ref, rtol=1e-5, atol=2e-5 * np.sqrt(K))
+
+
 def test_gemm_rejects_bad_shapes():
     require_gpu()
     import torch
