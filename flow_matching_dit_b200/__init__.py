@@ -258,6 +258,17 @@ def gemm_static_scratch(A, B, bias, C=None, bn: int = 64, splits: int = 1, strea
     return C
 
 
+def debug_skinny_plan(M: int, N: int, K: int, num_sms: int = 148):
+    """The skinny-M GEMM's plan for an [M, K] x [N, K]^T product
+    (gdit_debug_skinny_plan): dict(mt, nu, stages, ctas, smem_bytes), or None
+    when the shape runs on the tensor-core GEMM."""
+    out = [ctypes.c_int() for _ in range(5)]
+    rc = _lib.gdit_debug_skinny_plan(int(M), int(N), int(K), int(num_sms), *[ctypes.byref(o) for o in out])
+    if rc != 0:
+        return None
+    return dict(zip(("mt", "nu", "stages", "ctas", "smem_bytes"), (o.value for o in out)))
+
+
 def debug_wait_expiry(device: int = 0, limit_ns: int = 1_000_000) -> int:
     """Status of one bounded wait on an mbarrier that nothing arrives at
     (gdit_debug_wait_expiry): GDIT_ETIMEOUT is the expected result."""

@@ -254,6 +254,12 @@ bool plan_skinny(long long M, int N, int K, int num_sms, int& mt, int& nu, int& 
   return found;
 }
 
+// Shapes the skinny-M kernel takes: few rows, whole units of 8 features,
+// K in 64-column boxes.
+bool skinny_shape_ok(long long M, int N, int K) {
+  return M >= 1 && M <= kSkinnyMaxRows && N >= 8 && N % 8 == 0 && K >= 64 && K % 64 == 0;
+}
+
 // Switch a planned dense GEMM with few rows to the skinny-M kernel (plain
 // [M, K] x [N, K]^T layout, one output row per input row, no split).
 void enable_skinny(GemmOp& op, int num_sms) {
@@ -261,8 +267,8 @@ void enable_skinny(GemmOp& op, int num_sms) {
   const bool epi_ok = a.epi == EPI_BF16 || a.epi == EPI_GELU_BF16 || a.epi == EPI_RELU_BF16 || a.epi == EPI_F32 ||
                       a.epi == EPI_RESID_F32;
   const bool aligned = ((uintptr_t)op.a_ptr % 16) == 0 && ((uintptr_t)op.b_ptr % 16) == 0;
-  if (a.M > kSkinnyMaxRows || a.M < 1 || a.splits != 1 || a.num_groups != 0 || a.m_dev != nullptr || a.nblk != 0 ||
-      a.in_group != 0x7fffffff || a.out_off != 0 || !epi_ok || a.N % 8 != 0 || a.K % 64 != 0 || !aligned)
+  if (!skinny_shape_ok(a.M, a.N, a.K) || a.splits != 1 || a.num_groups != 0 || a.m_dev != nullptr || a.nblk != 0 ||
+      a.in_group != 0x7fffffff || a.out_off != 0 || !epi_ok || !aligned)
     return;
   int mt, nu, stages;
   if (!plan_skinny(a.M, a.N, a.K, num_sms, mt, nu, stages)) return;
@@ -1953,6 +1959,24 @@ __global__ void wait_expiry_kernel(unsigned* status, unsigned long long limit_ns
   mbar_init(&bar, 1);
   fence_mbar_init();
   mbar_wait(&bar, 0, status, limit_ns);
+}
+
+int gdit_debug_skinny_plan(long long M, int N, int K, int num_sms, int* mt, int* nu, int* stages, int* ctas,
+                           int* smem_bytes) {
+  g_create_error.clear();
+  return guarded(nullptr, [&] {
+    REQUIRE(mt && nu && stages && ctas && smem_bytes, "NULL output");
+    REQUIRE(num_sms >= 1, "num_sms %d", num_sms);
+    REQUIRE(skinny_shape_ok(M, N, K), "M %lld, N %d, K %d: not a skinny-M shape (M <= %lld, N %% 8, K %% 64)", M, N, K,
+            kSkinnyMaxRows);
+    int m = 0, u = 0, st = 0;
+    REQUIRE(plan_skinny(M, N, K, num_sms, m, u, st), "no skinny-M plan fits one round over %d SMs", num_sms);
+    *mt = m;
+    *nu = u;
+    *stages = st;
+    *ctas = (int)(((M + 16LL * m - 1) / (16LL * m)) * ((N / 8 + u - 1) / u));
+    *smem_bytes = sk_smem_bytes(m, u, st);
+  });
 }
 
 int gdit_debug_wait_expiry(int device, unsigned long long limit_ns) {

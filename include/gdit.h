@@ -251,6 +251,16 @@ int gdit_debug_kv(gdit_handle* h, int layer, float* k_out, float* v_out, int* to
  * Allocates and frees one status word on the device; synchronous. */
 int gdit_debug_wait_expiry(int device, unsigned long long limit_ns);
 
+/* The plan of the skinny-M GEMM (the DiT linears of a few samples; a host
+ * computation, no GPU needed): for out[M, N] = X[M, K] W[N, K]^T on num_sms
+ * SMs, the row block (*mt m16 tiles), the units of 8 output features per
+ * item (*nu), the ring depth (*stages), the CTAs (*ctas: one item each) and a
+ * CTA's dynamic shared memory (*smem_bytes).  Returns GDIT_OK with a plan, or
+ * GDIT_EINVAL for a shape the kernel does not take or when no plan fits one
+ * item per SM (such a GEMM runs on the tensor-core kernel).  For tests. */
+int gdit_debug_skinny_plan(long long M, int N, int K, int num_sms, int* mt, int* nu, int* stages, int* ctas,
+                           int* smem_bytes);
+
 /* Range-checked build.  libgdit_checked.so is the same library compiled with
  * GDIT_CHECKED=1 (same entry points, same results):
  *   - every device allocation of a handle sits between two 4 KiB guard bands
