@@ -227,10 +227,11 @@ constexpr long long kSkinnyMaxRows = 160;
 constexpr double kSkinnyItemBytes = 64.0 * 1024;
 
 // Row block (16 mt rows) and units per item for an [M, K] x [N, K]^T GEMM:
-// the least bytes streamed by the busiest CTA, with a ring of at least 3
+// the least bytes streamed by the busiest CTA, with a ring of at least 2
 // stages and at most one item per SM.  False if none fits: with two rounds of
-// items (FF1 at 136 rows: 18.9 us against 15.6 us for the tensor-core GEMM)
-// the skinny kernel loses.
+// items (FF1 at 136 rows, 3-stage rings: 18.9 us against 15.6 us for the
+// tensor-core GEMM) the skinny kernel loses, while one round on a 2-stage
+// ring (48-row blocks of 11 units) wins (B = 8: 8.70 ms per call against 8.76).
 bool plan_skinny(long long M, int N, int K, int num_sms, int& mt, int& nu, int& stages) {
   double best = 0.0;
   bool found = false;
@@ -240,7 +241,7 @@ bool plan_skinny(long long M, int N, int K, int num_sms, int& mt, int& nu, int& 
     for (int u = 1; u <= sk_max_units(m); ++u) {
       const long long items = nrb * ((units + u - 1) / u);
       const int st = std::min(8, (kSkSmemMax - 1024 - sk_red_bytes(m, u) - 64) / sk_stage_bytes(m, u));
-      if (st < 3 || items > num_sms) continue;
+      if (st < 2 || items > num_sms) continue;
       const double cost = (double)(std::min(rows, M) + 8LL * u) * K * 2.0 + kSkinnyItemBytes;
       if (!found || cost < best) {
         found = true;

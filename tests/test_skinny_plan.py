@@ -5,7 +5,7 @@ of four 64-column boxes of 16 mt activation rows and of 8 nu weight rows
 (128-byte rows), the cross-warp partial sums (4 sets of mt x nu fragments of
 32 lanes x 16 bytes) and one 8-byte barrier per stage, within 226 KB.  The
 planner takes, among row blocks mt in {1, 2, 3, 5} and units 1 .. max(mt),
-the plans with at least 3 stages and at most one item per SM, the one whose
+the plans with at least 2 stages and at most one item per SM, the one whose
 CTA streams the fewest bytes (rows of its item times K, plus a fixed 64 KB per
 item); shapes of more than 160 rows, or with N not a multiple of 8 or K not a
 multiple of 64, are not skinny.
@@ -33,7 +33,7 @@ def brute_force(M, N, K, sms):
             items = nrb * -(-(N // 8) // nu)
             _, stage, red = layout(mt, nu, 0)
             stages = min(8, (SMEM - 1024 - red - 64) // stage)
-            if stages < 3 or items > sms:
+            if stages < 2 or items > sms:
                 continue
             cost = (min(16 * mt, M) + 8 * nu) * K * 2 + 64 * 1024
             if best is None or cost < best[0]:
@@ -60,15 +60,19 @@ def test_plans_fit_and_are_the_cheapest(B, shape):
     assert (plan["mt"], plan["nu"], plan["stages"], plan["ctas"]) == (mt, nu, stages, items)
     smem, _, _ = layout(mt, nu, stages)
     assert plan["smem_bytes"] == smem <= SMEM
-    assert plan["ctas"] <= 148 and plan["stages"] >= 3
+    assert plan["ctas"] <= 148 and plan["stages"] >= 2
 
 
 def test_known_choices():
     # eight samples' rows: the 1024-wide linears in 32-row blocks of 5 units (130 CTAs)
     assert fm.debug_skinny_plan(136, 1024, 1024) == {"mt": 2, "nu": 5, "stages": 5, "ctas": 130,
                                                      "smem_bytes": 205864}
-    # FF1 at 136 rows needs two rounds of items: the tensor-core GEMM keeps it
-    assert fm.debug_skinny_plan(136, 4096, 1024) is None
+    # FF1 at 136 rows: one round only with 48-row blocks of 11 units, on a 2-stage ring
+    assert fm.debug_skinny_plan(136, 4096, 1024) == {"mt": 3, "nu": 11, "stages": 2, "ctas": 141,
+                                                     "smem_bytes": 1024 + 2 * 4 * (48 + 88) * 128 + 4 * 3 * 11 * 512 + 16}
+    # 153 rows (nine samples): FF1 in two 80-row blocks of 7 units, one CTA per SM
+    p = fm.debug_skinny_plan(153, 4096, 1024)
+    assert (p["mt"], p["nu"], p["ctas"]) == (5, 7, 148)
     # a single 16-row block of a few units when there are few rows
     p = fm.debug_skinny_plan(34, 1024, 1024)
     assert p["mt"] == 1 and p["ctas"] <= 148
