@@ -65,20 +65,27 @@ def check_io_shapes(cfg, feats, mask, state, ids, noise, out, image_mask=None):
     return B, S
 
 
+def make_config(geom, max_batch: int, max_seq: int, device: int = 0, flags: int = 0):
+    """The gdit_config of a model geometry (any object with the config's
+    geometry fields as attributes) and a capacity."""
+    cfg = _lib.gdit_config()
+    for name in ("num_layers", "hidden", "num_heads", "head_dim", "mlp_hidden", "backbone_dim",
+                 "action_dim", "state_dim", "action_horizon", "num_embodiments", "time_freq_dim",
+                 "num_timestep_buckets"):
+        setattr(cfg, name, int(getattr(geom, name)))
+    cfg.ln_eps = float(geom.ln_eps)
+    cfg.max_batch = int(max_batch)
+    cfg.max_backbone_seq = int(max_seq)
+    cfg.flags = int(flags)
+    cfg.device = int(device)
+    cfg.attend_text_every_n_blocks = int(getattr(geom, "attend_text_every_n_blocks", 0))
+    return cfg
+
+
 class ActionHead:
     def __init__(self, geom, weights: Dict[str, np.ndarray], max_batch: int, max_seq: int,
                  device: int = 0, flags: int = 0):
-        cfg = _lib.gdit_config()
-        for name in ("num_layers", "hidden", "num_heads", "head_dim", "mlp_hidden", "backbone_dim",
-                     "action_dim", "state_dim", "action_horizon", "num_embodiments", "time_freq_dim",
-                     "num_timestep_buckets"):
-            setattr(cfg, name, int(getattr(geom, name)))
-        cfg.ln_eps = float(geom.ln_eps)
-        cfg.max_batch = int(max_batch)
-        cfg.max_backbone_seq = int(max_seq)
-        cfg.flags = int(flags)
-        cfg.device = int(device)
-        cfg.attend_text_every_n_blocks = int(getattr(geom, "attend_text_every_n_blocks", 0))
+        cfg = make_config(geom, max_batch, max_seq, device, flags)
         self.cfg = cfg
         keep = []
         arr = (_lib.gdit_tensor * len(weights))()
@@ -256,6 +263,18 @@ def gemm_static_scratch(A, B, bias, C=None, bn: int = 64, splits: int = 1, strea
     check(_lib.gdit_gemm_static_scratch(_ptr(A), _ptr(B), _ptr(bias) if bias is not None else None, _ptr(C),
                                         M, N, K, bn, splits, st), None)
     return C
+
+
+def debug_small_plan(geom, batch: int, num_steps: int = 4, num_sms: int = 148, max_seq: int = 600,
+                     flags: int = 0):
+    """Whether a call of `batch` samples runs the persistent loop
+    (gdit_debug_small_plan): dict(group_ctas, grouped), or None for the
+    per-layer kernels."""
+    cfg = make_config(geom, max(batch, 1), max_seq, 0, flags)
+    g, gr = ctypes.c_int(), ctypes.c_int()
+    check(_lib.gdit_debug_small_plan(ctypes.byref(cfg), int(batch), int(num_steps), int(num_sms),
+                                     ctypes.byref(g), ctypes.byref(gr)))
+    return None if g.value == 0 else {"group_ctas": g.value, "grouped": bool(gr.value)}
 
 
 def debug_skinny_plan(M: int, N: int, K: int, num_sms: int = 148):

@@ -72,6 +72,7 @@ _SIGS = {
     "gdit_gemm_static_scratch": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "gdit_debug_wait_expiry": (_I, [_I, ctypes.c_ulonglong]),
     "gdit_debug_skinny_plan": (_I, [ctypes.c_longlong, _I, _I, _I] + [ctypes.POINTER(_I)] * 5),
+    "gdit_debug_small_plan": (_I, [ctypes.POINTER(gdit_config), _I, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
     "gdit_get_action_vl": (_I, [_P, _P, _I, _P, _P, _P, _P, _P, _I, _P, _I, _I, _P]),
     "gdit_is_checked": (_I, []),
     "gdit_check_canaries": (_I, [_P, ctypes.POINTER(ctypes.c_longlong)]),
@@ -188,6 +189,10 @@ def gdit_debug_wait_expiry(device, limit_ns):
 
 def gdit_debug_skinny_plan(*a):
     return lib().gdit_debug_skinny_plan(*a)
+
+
+def gdit_debug_small_plan(*a):
+    return lib().gdit_debug_small_plan(*a)
 
 
 def gdit_is_checked():

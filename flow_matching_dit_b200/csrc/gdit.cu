@@ -1155,6 +1155,25 @@ bool small_loop_fits(const gdit_config& c, int N, int ctas) {
   return true;
 }
 
+// Whether a batch of B samples runs the K-step loop as the persistent kernel
+// (one sample, or up to kSmallMaxGroups with one CTA group of num_sms / B
+// CTAs per sample), its CTAs per group, and whether the grouped instantiation
+// (several groups, or a CTA with more than kSmallMaxUnits units of a linear)
+// runs.  False: the per-layer kernels.
+bool plan_small(const gdit_config& c, int B, int K, int num_sms, int& gsize, bool& grouped) {
+  const int N = c.action_horizon + 1, L = c.num_layers;
+  const long long D = c.hidden, F = c.mlp_hidden, A = c.action_dim;
+  gsize = B >= 1 ? num_sms / B : 0;
+  grouped = false;
+  if (B < 1 || B > kSmallMaxGroups || (c.flags & GDIT_FLAG_NO_SMALL) != 0 ||
+      (long long)B * small_phases_per_step(L) * K > kSmallMaxPhases || !small_loop_fits(c, N, gsize))
+    return false;
+  grouped = B > 1;
+  for (long long n_out : {A, D, 3 * D, F})
+    if ((n_out / kSmallUF + gsize - 1) / gsize > kSmallMaxUnits) grouped = true;
+  return true;
+}
+
 std::unique_ptr<Profile> build_profile(gdit_handle* h, int B, int S, int K, int bf16) {
   auto p = std::make_unique<Profile>();
   p->B = B;
@@ -1289,9 +1308,9 @@ std::unique_ptr<Profile> build_profile(gdit_handle* h, int B, int S, int K, int 
 
   // one sample, or up to kSmallMaxGroups: the K-step loop as one persistent
   // kernel whose CTAs form one group per sample
-  const int gsize = B >= 1 ? h->num_sms / B : 0;
-  p->small = B >= 1 && B <= kSmallMaxGroups && (h->cfg.flags & GDIT_FLAG_NO_SMALL) == 0 &&
-             (long long)B * small_phases_per_step(L) * K <= kSmallMaxPhases && small_loop_fits(h->cfg, N, gsize);
+  int gsize = 0;
+  bool grouped = false;
+  p->small = plan_small(h->cfg, B, K, h->num_sms, gsize, grouped);
   if (p->small) {
     const Tables& t = h->tables.at(K);
     SmallPlan sp;
@@ -1321,9 +1340,7 @@ std::unique_ptr<Profile> build_profile(gdit_handle* h, int B, int S, int K, int 
     p->small_phases = small_phases_per_step(L) * K;
     p->small_groups = B;
     p->small_gsize = gsize;
-    p->small_grouped = B > 1;
-    for (long long n_out : {(long long)A, (long long)D, 3LL * D, (long long)F})
-      if ((n_out / kSmallUF + gsize - 1) / gsize > kSmallMaxUnits) p->small_grouped = true;
+    p->small_grouped = grouped;
     // sample b (embodiment-sorted position) works on its own rows of the
     // batch buffers and on its own counters, descriptors and statistics
     std::vector<SmallPlan> plans((size_t)B, sp);
@@ -1960,6 +1977,22 @@ __global__ void wait_expiry_kernel(unsigned* status, unsigned long long limit_ns
   mbar_init(&bar, 1);
   fence_mbar_init();
   mbar_wait(&bar, 0, status, limit_ns);
+}
+
+int gdit_debug_small_plan(const gdit_config* cfg, int batch, int num_steps, int num_sms, int* group_ctas,
+                          int* grouped) {
+  g_create_error.clear();
+  return guarded(nullptr, [&] {
+    REQUIRE(cfg && group_ctas && grouped, "NULL argument");
+    validate_config(*cfg);
+    REQUIRE(batch >= 1 && num_steps >= 1 && num_sms >= 1, "batch %d, num_steps %d, num_sms %d", batch, num_steps,
+            num_sms);
+    int g = 0;
+    bool gr = false;
+    const bool small = plan_small(*cfg, batch, num_steps, num_sms, g, gr);
+    *group_ctas = small ? g : 0;
+    *grouped = small ? (gr ? 1 : 0) : 0;
+  });
 }
 
 int gdit_debug_skinny_plan(long long M, int N, int K, int num_sms, int* mt, int* nu, int* stages, int* ctas,

@@ -261,6 +261,16 @@ int gdit_debug_wait_expiry(int device, unsigned long long limit_ns);
 int gdit_debug_skinny_plan(long long M, int N, int K, int num_sms, int* mt, int* nu, int* stages, int* ctas,
                            int* smem_bytes);
 
+/* Whether a call of `batch` samples and num_steps Euler steps on a model of
+ * geometry *cfg runs the whole loop as the persistent kernel, on num_sms SMs
+ * (a host computation, no GPU needed): *group_ctas = CTAs per sample group
+ * (num_sms / batch), 0 when the call runs the per-layer kernels; *grouped = 1
+ * when the grouped instantiation runs (several samples, or a CTA with more
+ * than 4 units of 8 features in some linear).  GDIT_EINVAL for an invalid
+ * configuration or arguments.  For tests. */
+int gdit_debug_small_plan(const gdit_config* cfg, int batch, int num_steps, int num_sms, int* group_ctas,
+                          int* grouped);
+
 /* Range-checked build.  libgdit_checked.so is the same library compiled with
  * GDIT_CHECKED=1 (same entry points, same results):
  *   - every device allocation of a handle sits between two 4 KiB guard bands
