@@ -271,6 +271,18 @@ def test_device_call_path_validates_then_reaches_the_library(L):
                              inp["embodiment_id"], inp["init_noise"], 4)
 
 
+def test_binding_flags_and_codes_equal_the_header():
+    """Every GDIT_FLAG_* and status code the header defines has the same value
+    in the binding (the C ABI passes them as plain integers)."""
+    src = open(HEADER).read()
+    defs = dict((n, int(v)) for n, v in re.findall(r"#define\s+(GDIT_FLAG_[A-Z_]+)\s+(\d+)u", src))
+    assert len(defs) >= 6
+    codes = dict((n, int(v)) for n, v in re.findall(r"#define\s+(GDIT_(?:OK|E[A-Z]+))\s+\(?(-?\d+)\)?", src))
+    assert codes["GDIT_OK"] == 0 and len(codes) >= 8
+    for name, value in {**defs, **codes}.items():
+        assert getattr(_lib, name) == value, name
+
+
 def test_binding_forwards_every_entry_point_under_its_own_name():
     for name in _lib.exported_names():
         assert callable(getattr(_lib, name, None)), name
